@@ -1,0 +1,275 @@
+"""Seeded synthetic inputs for the int8 SSD chunk scan and its decode state update.
+
+This module only draws random numbers and quantizes the drawn activations to the int8
+inputs the op consumes; it holds none of the scan's arithmetic.  It is shared by the
+CPU oracle tests, the GPU parity tests and ``bench.py``; it imports neither side.
+
+Workloads follow the shapes the pages measure on (Mamba-2 1.3B / 2.7B / 8B SSD layers):
+
+* x, B, C arrive as int8 with static symmetric scales: per tensor (Quamba project page,
+  "static per-tensor quantization") or per head for x and per group for B/C
+  (SSDi8 page, Table 10 "quantization axis": per-H(G)).
+* x is head-structured with outlier channels (SSDi8 page, Figure 2; Quamba2 rebuttal,
+  channel persistence), stood in for by Laplace values with 1 % of the (h, p) channels
+  scaled x20, or a head-wise magnitude spread.
+* dt = softplus(N(-2, 0.5)), A_h = -exp(U(0, ln 16)), D ~ N(0, 1): typical Mamba-2 ranges.
+
+Random draws use numpy's PCG64 (``default_rng(seed)``), seed = 1000 + config index by
+default, in the fixed order A, D, dt, x, B, C, outlier mask, magnitude spread.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Optional
+
+import numpy as np
+
+__all__ = [
+    "PrefillCase",
+    "DecodeCase",
+    "PREFILL_CONFIGS",
+    "DECODE_CONFIG",
+    "quantize_symmetric",
+    "make_prefill",
+    "make_prefill_config",
+    "make_decode",
+    "make_decode_config",
+]
+
+F32 = np.float32
+
+
+@dataclasses.dataclass
+class PrefillCase:
+    """One prefill problem: int8 x/B/C plus fp32 dt, A, D and the static scales."""
+
+    name: str
+    batch: int
+    seqlen: int
+    nheads: int
+    headdim: int
+    dstate: int
+    ngroups: int
+    chunk_size: int
+    x: np.ndarray  # int8 [b, l, h, p]
+    B: np.ndarray  # int8 [b, l, g, n]
+    C: np.ndarray  # int8 [b, l, g, n]
+    dt: np.ndarray  # f32 [b, l, h]
+    A: np.ndarray  # f32 [h]
+    D: np.ndarray  # f32 [h]
+    x_scale: np.ndarray  # f32 [h]
+    B_scale: np.ndarray  # f32 [g]
+    C_scale: np.ndarray  # f32 [g]
+    out_dtype: str = "f16"  # "f32" | "f16" | "i8"
+    init_state: Optional[np.ndarray] = None  # f32 [b, h, p, n]
+
+    @property
+    def tokens(self) -> int:
+        return self.batch * self.seqlen
+
+
+@dataclasses.dataclass
+class DecodeCase:
+    """A sequence of single-token state updates on one fp32 state."""
+
+    name: str
+    batch: int
+    steps: int
+    nheads: int
+    headdim: int
+    dstate: int
+    ngroups: int
+    state: np.ndarray  # f32 [b, h, p, n]
+    x: np.ndarray  # int8 [steps, b, h, p]
+    B: np.ndarray  # int8 [steps, b, g, n]
+    C: np.ndarray  # int8 [steps, b, g, n]
+    dt: np.ndarray  # f32 [steps, b, h]
+    A: np.ndarray  # f32 [h]
+    D: np.ndarray  # f32 [h]
+    x_scale: np.ndarray  # f32 [h]
+    B_scale: np.ndarray  # f32 [g]
+    C_scale: np.ndarray  # f32 [g]
+    out_dtype: str = "f16"
+
+
+# name, batch, seqlen, nheads, headdim, dstate, ngroups, chunk, x/B/C law, scale axes, out dtype
+PREFILL_CONFIGS = {
+    0: dict(name="tiny-ssd-prefill b1 L256 h4 p64 n16 g1 Q64", batch=1, seqlen=256, nheads=4,
+            headdim=64, dstate=16, ngroups=1, chunk_size=64, law="normal", scales="tensor",
+            out_dtype="f16"),
+    1: dict(name="mamba2-1.3b-ssd-prefill b4 L2048 h64 p64 n128 g1 Q256", batch=4, seqlen=2048,
+            nheads=64, headdim=64, dstate=128, ngroups=1, chunk_size=256,
+            law="laplace_outliers_x", scales="head", out_dtype="f16"),
+    2: dict(name="mamba2-2.7b-ssd-prefill b8 L4096 h80 p64 n128 g1 Q256", batch=8, seqlen=4096,
+            nheads=80, headdim=64, dstate=128, ngroups=1, chunk_size=256,
+            law="laplace_spread", scales="head", out_dtype="f16"),
+    3: dict(name="mamba2-8b-ssd-long-prefill b2 L16384 h128 p64 n128 g8 Q256 int8-out", batch=2,
+            seqlen=16384, nheads=128, headdim=64, dstate=128, ngroups=8, chunk_size=256,
+            law="laplace_outliers_all", scales="head", out_dtype="i8"),
+}
+
+DECODE_CONFIG = dict(name="mamba2-8b-ssd-decode b128 x512 steps h128 p64 n128 g8", batch=128,
+                     steps=512, nheads=128, headdim=64, dstate=128, ngroups=8, out_dtype="f16")
+
+
+def quantize_symmetric(v: np.ndarray, scale_axis: Optional[int]) -> tuple[np.ndarray, np.ndarray]:
+    """Static symmetric int8 quantization: s = absmax / 127, q = clamp(rne(v / s), -127, 127).
+
+    ``scale_axis`` is the axis that keeps its own scale (per head / per group); ``None``
+    gives one per-tensor scale.  Returns (q int8, s f32[...]); s has one entry per index of
+    ``scale_axis`` (or a single entry).
+    """
+    v = np.asarray(v, dtype=F32)
+    if v.ndim == 0:
+        raise ValueError("quantize_symmetric expects an array")
+    shape = [1] * v.ndim
+    if scale_axis is None:
+        amax = np.array([np.abs(v).max() if v.size else 0.0], dtype=np.float64)
+    else:
+        axes = tuple(i for i in range(v.ndim) if i != scale_axis)
+        amax = (np.abs(v).max(axis=axes).astype(np.float64) if v.size
+                else np.zeros(v.shape[scale_axis]))
+        shape[scale_axis] = v.shape[scale_axis]
+    s = np.where(amax > 0, amax / 127.0, 1.0).astype(F32)
+    sb = s.reshape(shape)
+    q = np.empty(v.shape, dtype=np.int8)
+    # slabs along the first axis bound the host memory used at the large workloads
+    for i in range(v.shape[0]):
+        si = sb[i] if shape[0] > 1 else sb[0]
+        r = np.rint(v[i] / si)  # round half to even, in fp32
+        np.clip(r, -127, 127, out=r)
+        q[i] = r.astype(np.int8)
+    return q, s
+
+
+def _laplace(rng: np.random.Generator, shape) -> np.ndarray:
+    """Laplace(0, 1) in fp32: an Exp(1) magnitude with a fair random sign."""
+    out = np.empty(shape, dtype=F32)
+    rng.standard_exponential(dtype=F32, out=out)
+    sign = rng.integers(0, 2, size=shape, dtype=np.int8)
+    out *= (sign.astype(F32) * 2.0 - 1.0)
+    return out
+
+
+def _normal(rng: np.random.Generator, shape) -> np.ndarray:
+    out = np.empty(shape, dtype=F32)
+    rng.standard_normal(dtype=F32, out=out)
+    return out
+
+
+def _dt_A_D(rng: np.random.Generator, dt_shape, nheads: int):
+    A = (-np.exp(rng.uniform(0.0, math.log(16.0), size=nheads))).astype(F32)
+    D = rng.standard_normal(nheads).astype(F32)
+    raw = rng.normal(-2.0, 0.5, size=dt_shape)
+    dt = np.log1p(np.exp(raw)).astype(F32)  # softplus
+    return A, D, dt
+
+
+def make_prefill(batch: int, seqlen: int, nheads: int, headdim: int, dstate: int, ngroups: int,
+                 chunk_size: int, *, law: str = "normal", scales: str = "head",
+                 out_dtype: str = "f16", seed: int = 0, with_init_state: bool = False,
+                 name: Optional[str] = None) -> PrefillCase:
+    """Draw one seeded prefill problem.
+
+    law: "normal" (x, B, C ~ N(0,1)); "laplace_outliers_x" (x Laplace with 1 % outlier
+    channels x20 over (h,p); B, C ~ N(0,1)); "laplace_spread" (x, B, C Laplace, x scaled
+    per head and B, C per group by U(0.5, 8)); "laplace_outliers_all" (x, B, C Laplace with
+    1 % outlier channels x20: x over (h,p), B and C over (g,n)).
+    scales: "tensor" (one scale per tensor, broadcast) or "head" (x per head, B/C per group).
+    """
+    if nheads % ngroups:
+        raise ValueError("nheads must be a multiple of ngroups")
+    rng = np.random.default_rng(seed)
+    A, D, dt = _dt_A_D(rng, (batch, seqlen, nheads), nheads)
+    xs = (batch, seqlen, nheads, headdim)
+    bs = (batch, seqlen, ngroups, dstate)
+    if law == "normal" or law == "laplace_outliers_x":
+        x = _laplace(rng, xs) if law == "laplace_outliers_x" else _normal(rng, xs)
+        Bf = _normal(rng, bs)
+        Cf = _normal(rng, bs)
+    elif law in ("laplace_spread", "laplace_outliers_all"):
+        x = _laplace(rng, xs)
+        Bf = _laplace(rng, bs)
+        Cf = _laplace(rng, bs)
+    else:
+        raise ValueError(f"unknown law {law!r}")
+    # outlier mask, then magnitude spread (fixed draw order)
+    if law in ("laplace_outliers_x", "laplace_outliers_all"):
+        xm = rng.random(nheads * headdim) < 0.01
+        x *= np.where(xm, 20.0, 1.0).astype(F32).reshape(1, 1, nheads, headdim)
+        if law == "laplace_outliers_all":
+            bm = rng.random(ngroups * dstate) < 0.01
+            cm = rng.random(ngroups * dstate) < 0.01
+            Bf *= np.where(bm, 20.0, 1.0).astype(F32).reshape(1, 1, ngroups, dstate)
+            Cf *= np.where(cm, 20.0, 1.0).astype(F32).reshape(1, 1, ngroups, dstate)
+    if law == "laplace_spread":
+        hs = rng.uniform(0.5, 8.0, size=nheads).astype(F32)
+        gs_b = rng.uniform(0.5, 8.0, size=ngroups).astype(F32)
+        gs_c = rng.uniform(0.5, 8.0, size=ngroups).astype(F32)
+        x *= hs.reshape(1, 1, nheads, 1)
+        Bf *= gs_b.reshape(1, 1, ngroups, 1)
+        Cf *= gs_c.reshape(1, 1, ngroups, 1)
+    if scales == "tensor":
+        xq, sx = quantize_symmetric(x, None)
+        Bq, sb = quantize_symmetric(Bf, None)
+        Cq, sc = quantize_symmetric(Cf, None)
+        sx = np.full(nheads, sx[0], dtype=F32)
+        sb = np.full(ngroups, sb[0], dtype=F32)
+        sc = np.full(ngroups, sc[0], dtype=F32)
+    elif scales == "head":
+        xq, sx = quantize_symmetric(x, 2)
+        Bq, sb = quantize_symmetric(Bf, 2)
+        Cq, sc = quantize_symmetric(Cf, 2)
+    else:
+        raise ValueError(f"unknown scales {scales!r}")
+    del x, Bf, Cf
+    init = None
+    if with_init_state:
+        init = (0.1 * rng.standard_normal((batch, nheads, headdim, dstate))).astype(F32)
+    return PrefillCase(
+        name=name or f"prefill b{batch} L{seqlen} h{nheads} p{headdim} n{dstate} g{ngroups} Q{chunk_size}",
+        batch=batch, seqlen=seqlen, nheads=nheads, headdim=headdim, dstate=dstate,
+        ngroups=ngroups, chunk_size=chunk_size, x=xq, B=Bq, C=Cq, dt=dt, A=A, D=D,
+        x_scale=sx, B_scale=sb, C_scale=sc, out_dtype=out_dtype, init_state=init)
+
+
+def make_prefill_config(index: int, seed: Optional[int] = None, **overrides) -> PrefillCase:
+    """The prefill workload ``index`` (0..3) with its default seed 1000 + index."""
+    spec = dict(PREFILL_CONFIGS[index])
+    spec.update(overrides)
+    name = spec.pop("name")
+    return make_prefill(seed=1000 + index if seed is None else seed, name=name, **spec)
+
+
+def make_decode(batch: int, steps: int, nheads: int, headdim: int, dstate: int, ngroups: int, *,
+                out_dtype: str = "f16", seed: int = 0, name: Optional[str] = None) -> DecodeCase:
+    """Draw a seeded decode run: an fp32 state ~ N(0, 0.1^2) and ``steps`` fresh tokens.
+
+    Per step x, B, C ~ N(0, 1), quantized with static scales (x per head, B/C per group)
+    calibrated over all steps; dt, A, D as in the prefill workloads.
+    """
+    if nheads % ngroups:
+        raise ValueError("nheads must be a multiple of ngroups")
+    rng = np.random.default_rng(seed)
+    A, D, dt = _dt_A_D(rng, (steps, batch, nheads), nheads)
+    x = _normal(rng, (steps, batch, nheads, headdim))
+    Bf = _normal(rng, (steps, batch, ngroups, dstate))
+    Cf = _normal(rng, (steps, batch, ngroups, dstate))
+    state = (0.1 * _normal(rng, (batch, nheads, headdim, dstate))).astype(F32)
+    xq, sx = quantize_symmetric(x, 2)
+    Bq, sb = quantize_symmetric(Bf, 2)
+    Cq, sc = quantize_symmetric(Cf, 2)
+    return DecodeCase(
+        name=name or f"decode b{batch} x{steps} h{nheads} p{headdim} n{dstate} g{ngroups}",
+        batch=batch, steps=steps, nheads=nheads, headdim=headdim, dstate=dstate,
+        ngroups=ngroups, state=state, x=xq, B=Bq, C=Cq, dt=dt, A=A, D=D, x_scale=sx,
+        B_scale=sb, C_scale=sc, out_dtype=out_dtype)
+
+
+def make_decode_config(seed: Optional[int] = None, **overrides) -> DecodeCase:
+    """The decode workload (batch 128, 512 steps, Mamba-2-8B head shape), seed 1004."""
+    spec = dict(DECODE_CONFIG)
+    spec.update(overrides)
+    name = spec.pop("name")
+    return make_decode(seed=1004 if seed is None else seed, name=name, **spec)
