@@ -1,0 +1,417 @@
+"""Benchmark of the int8 SSD chunk scan (and its decode state update) on B200.
+
+One JSON line on rank 0.  A "step" is one ``ssd_i8_chunk_scan`` call over the Mamba-2-8B
+shaped long prefill (batch 2 x 16384 tokens, 128 heads x 64, dstate 128, 8 groups, chunk
+256, int8 output): chunk_cumsum, ChunkBMM, chunk_state, state passing, chunk_scan and the
+requantizing epilogue.  ``value`` = tokens/s with inputs resident in HBM; ``e2e`` = the same
+through the public call with pinned-host inputs copied in and the int8 output copied back in
+every step.  The decode state update (batch 128, 512 steps) is reported beside it under
+``decode``.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 launch under torch.distributed.run; every rank scans its own batch (weak scaling,
+no collective on the data path; the only collective is the max-over-ranks of the timings).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from quantized_mamba_ssd_b200 import workloads as W  # noqa: E402
+
+PREFILL_CFG = 3
+METRIC = "SSD scan tokens/s (int8 in) at 1 B200; achieved fraction of HBM/int8 roofline"
+UNIT = "tokens/s"
+INT8_PER_BF16 = 2.0  # nominal dense int8 : bf16 tensor throughput ratio on B200 (4.5 : 2.25)
+
+
+# ------------------------------------------------------------------------------------------
+# algorithmic work of one call (bytes moved once, int8 MMA ops of the causal contractions)
+# ------------------------------------------------------------------------------------------
+def prefill_alg_bytes(c: W.PrefillCase, out_bytes: int, final_state: bool) -> int:
+    b, L, H, P, N, G = c.batch, c.seqlen, c.nheads, c.headdim, c.dstate, c.ngroups
+    n = b * L * H * P  # x in (int8)
+    n += 2 * b * L * G * N  # B, C in (int8)
+    n += 4 * b * L * H  # dt (f32)
+    n += out_bytes * b * L * H * P  # y out
+    if final_state:
+        n += 4 * b * H * P * N
+    return n
+
+
+def prefill_alg_ops(c: W.PrefillCase) -> float:
+    """2 x MACs: causal CB per group, causal M.x, chunk state B^T x and C.H_prev per head."""
+    b, L, H, P, N, G, Q = c.batch, c.seqlen, c.nheads, c.headdim, c.dstate, c.ngroups, c.chunk_size
+    nch = -(-L // Q)
+    causal = Q * (Q + 1) / 2
+    cb = b * nch * G * causal * N
+    mx = b * nch * H * causal * P
+    st = b * L * H * P * N
+    ch = b * L * H * N * P
+    return 2.0 * (cb + mx + st + ch)
+
+
+def decode_alg_bytes(d: W.DecodeCase, out_bytes: int) -> int:
+    b, H, P, N, G = d.batch, d.nheads, d.headdim, d.dstate, d.ngroups
+    return 2 * 4 * b * H * P * N + b * H * P + 2 * b * G * N + 4 * b * H + out_bytes * b * H * P
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", 0)), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only; nothing is changed)
+# ------------------------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = self._handle(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # NVML missing: report clocks as unavailable
+            self.ok = False
+
+    def _handle(self, device_index):
+        import torch
+        pynvml = self.nvml
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            return pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid).encode())
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(device_index)
+
+    def _run(self):
+        pynvml = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(pynvml.nvmlDeviceGetClockInfo(self.handle, pynvml.NVML_CLOCK_SM))
+                self.reasons |= pynvml.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        reasons = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------------------------
+# CPU baseline / reference arm: the oracle on a bounded sample of the same workload
+# ------------------------------------------------------------------------------------------
+def oracle_tokens_per_s(case: W.PrefillCase, target_s: float = 15.0):
+    import oracle
+    oracle.build()
+    probe = min(case.seqlen, 64)
+
+    def run(Ls):
+        t0 = time.perf_counter()
+        _, _, nt = oracle.scan(case.x[:, :Ls], case.B[:, :Ls], case.C[:, :Ls], case.dt[:, :Ls],
+                               case.A, case.D, case.x_scale, case.B_scale, case.C_scale,
+                               want_final_state=False)
+        return time.perf_counter() - t0, nt
+
+    tp, _ = run(probe)
+    Ls = int(min(case.seqlen, max(probe, probe * target_s / max(tp, 1e-6))))
+    t, nt = run(Ls)
+    tokens = case.batch * Ls
+    return tokens / t, nt, (f"first {Ls} of {case.seqlen} tokens of every (batch, head) pair of "
+                            f"the workload ({tokens} tokens x {case.nheads} heads), fp64 oracle")
+
+
+def reference_arm(args, case: W.PrefillCase):
+    """--impl reference: the fp64 CPU oracle, as it stands, on bounded samples."""
+    import oracle
+    oracle.build()
+    Ls = min(case.seqlen, 512)
+    xs = (case.x[:, :Ls], case.B[:, :Ls], case.C[:, :Ls], case.dt[:, :Ls])
+    times = []
+    nt = 0
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        _, _, nt = oracle.scan(*xs, case.A, case.D, case.x_scale, case.B_scale, case.C_scale,
+                               want_final_state=False)
+        dtm = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dtm)
+    tot = sum(times)
+    tokens = case.batch * Ls * len(times)
+    value = tokens / tot
+    sample = (f"first {Ls} of {case.seqlen} tokens of every (batch, head) pair per step "
+              f"({case.batch * Ls} tokens x {case.nheads} heads), fp64 oracle")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded, shapes and value laws of the workload)",
+        "config": {"workload": case.name, "global_batch": case.batch, "seq_len": case.seqlen,
+                   "sample_seq_len": Ls, "parallelism": "cpu threads over (batch, head)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": nt, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------------
+# our arm
+# ------------------------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--decode-passes", type=int, default=3,
+                    help="timed passes of the 512-step decode run (0 skips the decode report)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        reference_arm(args, W.make_prefill_config(PREFILL_CFG))
+        return
+
+    import torch
+    import torch.distributed as dist
+    from quantized_mamba_ssd_b200 import ssd_i8
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    ssd_i8.library()
+
+    hbm_peak, bf16_peak, bf16_sus, peak_kind = load_peaks()
+    int8_peak_tops = bf16_peak * INT8_PER_BF16
+
+    # ---- prefill workload: this rank's own batch (seeded per rank) ----
+    case = W.make_prefill_config(PREFILL_CFG, seed=1000 + PREFILL_CFG + 97 * rank)
+    x, B, C = (torch.from_numpy(a).to(dev) for a in (case.x, case.B, case.C))
+    dt = torch.from_numpy(case.dt).to(dev)
+    A, Dp, sx, sb, sc = (torch.from_numpy(a).to(dev) for a in
+                         (case.A, case.D, case.x_scale, case.B_scale, case.C_scale))
+    bsz, L, H, P, N, G, Q = (case.batch, case.seqlen, case.nheads, case.headdim, case.dstate,
+                             case.ngroups, case.chunk_size)
+    y = torch.empty((bsz, L, H, P), dtype=torch.int8, device=dev)
+    fs = torch.empty((bsz, H, P, N), dtype=torch.float32, device=dev)
+    ws = torch.empty(ssd_i8.ssd_i8_chunk_scan_workspace_size(bsz, L, H, P, N, G, Q),
+                     dtype=torch.uint8, device=dev)
+    # static output scale: a fixed calibration constant for the int8 output (the parity tests
+    # calibrate it on the oracle; here it only sets the clamp range)
+    y_scale = 0.05
+
+    def step():
+        ssd_i8.ssd_i8_chunk_scan(x, B, C, dt, A, Dp, sx, sb, sc, Q, final_state=fs, y=y,
+                                 y_dtype="i8", y_scale=y_scale, workspace=ws)
+
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clocks:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    t = torch.tensor([ms], device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    tokens_all = bsz * L * world
+    value = tokens_all / (ms_max * 1e-3)
+
+    # ---- end to end: pinned host inputs in, int8 output back, every step ----
+    hx, hB, hC, hdt = (torch.from_numpy(a).pin_memory() for a in (case.x, case.B, case.C, case.dt))
+    hy = torch.empty((bsz, L, H, P), dtype=torch.int8).pin_memory()
+    h2d = sum(t_.numel() * t_.element_size() for t_ in (hx, hB, hC, hdt))
+    d2h = hy.numel() * hy.element_size()
+
+    def e2e_step():
+        x.copy_(hx, non_blocking=True)
+        B.copy_(hB, non_blocking=True)
+        C.copy_(hC, non_blocking=True)
+        dt.copy_(hdt, non_blocking=True)
+        step()
+        hy.copy_(y, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    ev0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    t = torch.tensor([ev0.elapsed_time(ev1) / e2e_steps], device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_value = tokens_all / (float(t.item()) * 1e-3)
+
+    # ---- roofline of the timed call ----
+    alg_bytes = prefill_alg_bytes(case, 1, True)
+    alg_ops = prefill_alg_ops(case)
+    t_hbm = alg_bytes / (hbm_peak * 1e9)
+    t_ops = alg_ops / (int8_peak_tops * 1e12)
+    bound = "hbm" if t_hbm >= t_ops else "tensor"
+    achieved_gbs = alg_bytes / (ms * 1e-3) / 1e9
+    roofline = {
+        "bound": bound, "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+        "frac": achieved_gbs / hbm_peak, "traffic": None,
+        "peak_kind": f"{peak_kind} HBM copy bandwidth",
+        "alg_bytes_per_launch": alg_bytes, "alg_int8_ops_per_launch": alg_ops,
+        "roofline_us": 1e6 * max(t_hbm, t_ops), "frac_of_roofline_time": 1e6 * max(t_hbm, t_ops) / (ms * 1e3),
+        "int8_peak_tops": int8_peak_tops,
+    }
+
+    # ---- decode state update, 512 steps of batch 128 (CUDA graph replay) ----
+    decode = None
+    if args.decode_passes > 0:
+        d = W.make_decode_config(seed=1004 + 97 * rank)
+        st = torch.from_numpy(d.state).to(dev)
+        dx, dB, dC, ddt = (torch.from_numpy(a).to(dev) for a in (d.x, d.B, d.C, d.dt))
+        dA, dD, dsx, dsb, dsc = (torch.from_numpy(a).to(dev) for a in
+                                 (d.A, d.D, d.x_scale, d.B_scale, d.C_scale))
+        dy = torch.empty((d.steps, d.batch, d.nheads, d.headdim), dtype=torch.float16, device=dev)
+
+        def decode_pass():
+            for s in range(d.steps):
+                ssd_i8.ssd_i8_state_update(st, dx[s], dB[s], dC[s], ddt[s], dA, dD, dsx, dsb, dsc,
+                                           y=dy[s], y_dtype="f16")
+
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            decode_pass()  # warm up on the capture stream
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            decode_pass()
+        for _ in range(max(1, args.warmup // 2)):
+            graph.replay()
+        torch.cuda.synchronize()
+        barrier()
+        ev0.record(stream)
+        for _ in range(args.decode_passes):
+            graph.replay()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        t = torch.tensor([ev0.elapsed_time(ev1) / args.decode_passes], device=dev)
+        if world > 1:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dms = float(t.item())
+        dbytes = decode_alg_bytes(d, 2) * d.steps
+        dgbs = dbytes / (dms * 1e-3) / 1e9
+        decode = {
+            "metric": "SSD decode state-update tokens/s (int8 in, fp32 state)",
+            "value": d.batch * d.steps * world / (dms * 1e-3), "unit": UNIT,
+            "ms_per_512_steps": dms, "us_per_step": 1e3 * dms / d.steps,
+            "workload": d.name, "gpu_launches_per_pass": d.steps,
+            "roofline": {"bound": "hbm", "achieved": dgbs, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": dgbs / hbm_peak, "traffic": None,
+                         "alg_bytes_per_launch": decode_alg_bytes(d, 2)},
+        }
+        del graph
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, nt, sample = oracle_tokens_per_s(case)
+        cpu = {"value": v, "unit": UNIT, "cores": nt, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8",
+            "data": "synthetic (seeded; shapes and value laws of the Mamba-2-8B SSD workload)",
+            "config": {"workload": case.name, "global_batch": bsz * world, "seq_len": L,
+                       "nheads": H, "headdim": P, "dstate": N, "ngroups": G, "chunk_size": Q,
+                       "out_dtype": "i8", "parallelism": f"batch-sharded x{world}, no collective",
+                       "l2": "inputs larger than L2 (x 268 MB + B,C 67 MB + dt 17 MB per rank)"},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps * ssd_i8.KERNELS_PER_CHUNK_SCAN,
+            "clocks": clocks.summary(),
+            "decode": decode,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

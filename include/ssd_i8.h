@@ -1,0 +1,128 @@
+/*
+ * ssd_i8.h -- C ABI of the B200 (sm_100a) int8-input Mamba-2 SSD library.
+ *
+ * The operation (per batch b and head h, head h reading group g = h / (nheads/ngroups)):
+ *
+ *   x_t = s_x[h] * xq[b,t,h,:]     B_t = s_B[g] * Bq[b,t,g,:]     C_t = s_C[g] * Cq[b,t,g,:]
+ *   h_t = exp(dt_t * A[h]) * h_{t-1} + dt_t * x_t B_t^T            (state [headdim, dstate])
+ *   y_t = h_t C_t + D[h] * x_t                                      (output [headdim])
+ *
+ * Sources: the SSM recurrence h_t = Abar_t h_{t-1} + Bbar_t x_t ("Ternary Mamba: Grouped
+ * Quantization-Aware Training of W1.58A16 State Space Models", section 1); x, B and C as
+ * int8 SSD inputs with static scales ("Quamba2" OpenReview rebuttal, response on quantizing
+ * the SSD inputs (B, C, x); "Quamba" project page, static per-tensor quantization; "SSDi8"
+ * page, Table 10, per-H(G) scale axes); the chunked evaluation with a persistent int8 path
+ * ("SSDi8" page, Abstract, Figure 1(b), Figure 3(a) ChunkState, Table 5 ChunkBMM).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; tensors are dense,
+ *     row-major (C order) with the shapes given in brackets.  The library allocates nothing.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *     Argument errors are detected on the host and returned before anything is launched;
+ *     launch failures return SSD_ERR_CUDA.  No entry point throws or aborts.
+ *   - Output dtype codes: SSD_OUT_F32 (float), SSD_OUT_F16 (IEEE half), SSD_OUT_I8 (int8,
+ *     q = clamp(round_half_even(y / y_scale), -127, 127); y_scale > 0 is used only for I8).
+ */
+#ifndef SSD_I8_H
+#define SSD_I8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SSD_API __attribute__((visibility("default")))
+#else
+#define SSD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum ssd_status {
+    SSD_OK = 0,
+    SSD_ERR_INVALID_ARG = 1, /* null pointer, negative size, H % G != 0, bad dtype code ... */
+    SSD_ERR_UNSUPPORTED = 2, /* shape outside what the kernels implement (see each call)   */
+    SSD_ERR_WORKSPACE = 3,   /* workspace missing, too small or misaligned                  */
+    SSD_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed                 */
+    SSD_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up (reported by a kernel)   */
+} ssd_status;
+
+typedef enum ssd_out_dtype { SSD_OUT_F32 = 0, SSD_OUT_F16 = 1, SSD_OUT_I8 = 2 } ssd_out_dtype;
+
+/* Version of this ABI; bumped when a signature or a layout changes. */
+SSD_API int ssd_i8_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+SSD_API const char *ssd_status_string(ssd_status status);
+
+/*
+ * Bytes of device workspace that ssd_i8_chunk_scan needs for this problem (0 on invalid
+ * sizes).  The workspace holds the per-chunk states of the chunked scan; its contents do not
+ * need to be initialised and are scratch between calls.  One workspace per concurrently
+ * running call.
+ */
+SSD_API size_t ssd_i8_chunk_scan_workspace_size(int batch, int seqlen, int nheads, int headdim,
+                                        int dstate, int ngroups, int chunk_size);
+
+/*
+ * Chunked SSD scan over a prefill (SSDi8 page: ChunkState, state passing, ChunkScan with the
+ * ChunkBMM product CB = C B^T kept in exact int32).
+ *
+ *   x          int8  [batch, seqlen, nheads, headdim]
+ *   B, C       int8  [batch, seqlen, ngroups, dstate]
+ *   dt         float [batch, seqlen, nheads]   (already discretised / softplus'ed, >= 0)
+ *   A, D       float [nheads]                   (A <= 0)
+ *   x_scale    float [nheads];  B_scale, C_scale float [ngroups]   (static scales)
+ *   chunk_size Q: 64, 128 or 256.  The result does not depend on Q beyond rounding.
+ *   init_state float [batch, nheads, headdim, dstate] or NULL (zero initial state)
+ *   final_state float [batch, nheads, headdim, dstate] or NULL (not written)
+ *   y          [batch, seqlen, nheads, headdim] of y_dtype
+ *   workspace  device memory of at least ssd_i8_chunk_scan_workspace_size(...) bytes,
+ *              256-byte aligned.
+ * Supported: headdim == 64; dstate in {16, 32, 64, 128}; seqlen >= 0 (seqlen == 0 only copies
+ * init_state to final_state); batch >= 0; nheads % ngroups == 0.
+ */
+SSD_API ssd_status ssd_i8_chunk_scan(const int8_t *x, const int8_t *B, const int8_t *C, const float *dt,
+                             const float *A, const float *D, const float *x_scale,
+                             const float *B_scale, const float *C_scale, int batch, int seqlen,
+                             int nheads, int headdim, int dstate, int ngroups, int chunk_size,
+                             const float *init_state, float *final_state, void *y, int y_dtype,
+                             float y_scale, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Single-token decode state update, in place (the "SSD update" of the Quamba2 rebuttal's
+ * generation-time discussion, Tables R7/R8): one step of the recurrence above.
+ *
+ *   state      float [batch, nheads, headdim, dstate]   read and overwritten with h_t
+ *   x          int8  [batch, nheads, headdim]
+ *   B, C       int8  [batch, ngroups, dstate]
+ *   dt         float [batch, nheads]
+ *   A, D, x_scale float [nheads]; B_scale, C_scale float [ngroups]
+ *   y          [batch, nheads, headdim] of y_dtype
+ * Supported: dstate in {16, 32, 64, 128, 256}; 1 <= headdim <= 256; nheads % ngroups == 0.
+ */
+SSD_API ssd_status ssd_i8_state_update(float *state, const int8_t *x, const int8_t *B, const int8_t *C,
+                               const float *dt, const float *A, const float *D,
+                               const float *x_scale, const float *B_scale, const float *C_scale,
+                               int batch, int nheads, int headdim, int dstate, int ngroups,
+                               void *y, int y_dtype, float y_scale, void *stream);
+
+/*
+ * ChunkBMM of SSDi8 (Table 5): the exact int32 products CB[b, c, g, t, s] =
+ * sum_n Cq[b, c*Q+t, g, n] * Bq[b, c*Q+s, g, n] for every chunk c of length Q, the full
+ * Q x Q block (no causal mask), zero where c*Q+t or c*Q+s >= seqlen.  Computed by the same
+ * device code the chunk scan uses for its intra-chunk term; exposed so that the integer part
+ * of the scan can be checked bit for bit.
+ *
+ *   C, B int8 [batch, seqlen, ngroups, dstate];  cb int32 [batch, ceil(seqlen/Q), ngroups, Q, Q]
+ * Supported: as ssd_i8_chunk_scan for dstate and chunk_size.
+ */
+SSD_API ssd_status ssd_i8_chunk_cb(const int8_t *C, const int8_t *B, int batch, int seqlen, int ngroups,
+                           int dstate, int chunk_size, int32_t *cb, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSD_I8_H */

@@ -1,0 +1,134 @@
+// extern "C" entry points of libssd_i8.so: argument checks, then one launch sequence on the
+// caller's stream.  Declarations and their documentation live in include/ssd_i8.h.
+#include <cmath>
+#include <cstdint>
+
+#include "../../include/ssd_i8.h"
+#include "ssd_kernels.h"
+
+namespace {
+
+constexpr int kAbiVersion = 1;
+constexpr size_t kWorkspaceAlign = 256;
+
+bool valid_out_dtype(int d) { return d == SSD_OUT_F32 || d == SSD_OUT_F16 || d == SSD_OUT_I8; }
+
+bool chunk_dstate_ok(int n) { return n == 16 || n == 32 || n == 64 || n == 128; }
+
+bool chunk_size_ok(int q) { return q == 64 || q == 128 || q == 256; }
+
+// Output scale handling shared by both entry points: I8 needs y_scale > 0 (finite); the
+// kernels multiply by its fp32 reciprocal.
+bool out_scale(int y_dtype, float y_scale, float* inv) {
+    *inv = 1.f;
+    if (y_dtype != SSD_OUT_I8) return true;
+    if (!(y_scale > 0.f) || !std::isfinite(y_scale)) return false;
+    *inv = 1.f / y_scale;
+    return std::isfinite(*inv);
+}
+
+}  // namespace
+
+extern "C" {
+
+int ssd_i8_abi_version(void) { return kAbiVersion; }
+
+const char* ssd_status_string(ssd_status s) {
+    switch (s) {
+        case SSD_OK: return "SSD_OK";
+        case SSD_ERR_INVALID_ARG: return "SSD_ERR_INVALID_ARG: invalid argument";
+        case SSD_ERR_UNSUPPORTED: return "SSD_ERR_UNSUPPORTED: shape not supported by the kernels";
+        case SSD_ERR_WORKSPACE: return "SSD_ERR_WORKSPACE: workspace missing, too small or misaligned";
+        case SSD_ERR_CUDA: return "SSD_ERR_CUDA: CUDA runtime or launch failure";
+        case SSD_ERR_TIMEOUT: return "SSD_ERR_TIMEOUT: a bounded device-side wait gave up";
+        default: return "SSD_ERR_UNKNOWN";
+    }
+}
+
+size_t ssd_i8_chunk_scan_workspace_size(int batch, int seqlen, int nheads, int headdim,
+                                        int dstate, int ngroups, int chunk_size) {
+    if (batch < 0 || seqlen < 0 || nheads <= 0 || headdim <= 0 || dstate <= 0 || ngroups <= 0 ||
+        chunk_size <= 0)
+        return 0;
+    const size_t n = ssd::chunk_scan_workspace_bytes(batch, seqlen, nheads, headdim, dstate,
+                                                     chunk_size);
+    return (n + kWorkspaceAlign - 1) / kWorkspaceAlign * kWorkspaceAlign;
+}
+
+ssd_status ssd_i8_chunk_scan(const int8_t* x, const int8_t* B, const int8_t* C, const float* dt,
+                             const float* A, const float* D, const float* x_scale,
+                             const float* B_scale, const float* C_scale, int batch, int seqlen,
+                             int nheads, int headdim, int dstate, int ngroups, int chunk_size,
+                             const float* init_state, float* final_state, void* y, int y_dtype,
+                             float y_scale, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+    if (batch < 0 || seqlen < 0 || nheads <= 0 || headdim <= 0 || dstate <= 0 || ngroups <= 0 ||
+        chunk_size <= 0 || nheads % ngroups != 0 || !valid_out_dtype(y_dtype))
+        return SSD_ERR_INVALID_ARG;
+    if (!A || !D || !x_scale || !B_scale || !C_scale) return SSD_ERR_INVALID_ARG;
+    if (headdim != 64 || !chunk_dstate_ok(dstate) || !chunk_size_ok(chunk_size))
+        return SSD_ERR_UNSUPPORTED;
+    float inv = 1.f;
+    if (!out_scale(y_dtype, y_scale, &inv)) return SSD_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t state_bytes = (size_t)batch * nheads * headdim * dstate * sizeof(float);
+    if (batch == 0) return SSD_OK;
+    if (seqlen == 0) {
+        // nothing to scan: the final state is the initial state
+        if (final_state) {
+            cudaError_t e = init_state ? cudaMemcpyAsync(final_state, init_state, state_bytes,
+                                                         cudaMemcpyDeviceToDevice, st)
+                                       : cudaMemsetAsync(final_state, 0, state_bytes, st);
+            if (e != cudaSuccess) return SSD_ERR_CUDA;
+        }
+        return SSD_OK;
+    }
+    if (!x || !B || !C || !dt || !y) return SSD_ERR_INVALID_ARG;
+    const size_t need = ssd_i8_chunk_scan_workspace_size(batch, seqlen, nheads, headdim, dstate,
+                                                         ngroups, chunk_size);
+    if (!workspace || workspace_bytes < need ||
+        reinterpret_cast<uintptr_t>(workspace) % kWorkspaceAlign != 0)
+        return SSD_ERR_WORKSPACE;
+    ssd::ChunkScanArgs a{x, B, C, dt, A, D, x_scale, B_scale, C_scale, batch, seqlen, nheads,
+                         headdim, dstate, ngroups, chunk_size, init_state, final_state, y,
+                         y_dtype, inv, workspace};
+    return ssd::launch_chunk_scan(a, st) == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
+ssd_status ssd_i8_state_update(float* state, const int8_t* x, const int8_t* B, const int8_t* C,
+                               const float* dt, const float* A, const float* D,
+                               const float* x_scale, const float* B_scale, const float* C_scale,
+                               int batch, int nheads, int headdim, int dstate, int ngroups,
+                               void* y, int y_dtype, float y_scale, void* stream) {
+    if (batch < 0 || nheads <= 0 || headdim <= 0 || dstate <= 0 || ngroups <= 0 ||
+        nheads % ngroups != 0 || !valid_out_dtype(y_dtype))
+        return SSD_ERR_INVALID_ARG;
+    if (!(dstate == 16 || dstate == 32 || dstate == 64 || dstate == 128 || dstate == 256) ||
+        headdim > 256)
+        return SSD_ERR_UNSUPPORTED;
+    float inv = 1.f;
+    if (!out_scale(y_dtype, y_scale, &inv)) return SSD_ERR_INVALID_ARG;
+    if (batch == 0) return SSD_OK;
+    if (!state || !x || !B || !C || !dt || !A || !D || !x_scale || !B_scale || !C_scale || !y)
+        return SSD_ERR_INVALID_ARG;
+    ssd::StateUpdateArgs a{state, x, B, C, dt, A, D, x_scale, B_scale, C_scale, batch, nheads,
+                           headdim, dstate, ngroups, y, y_dtype, inv};
+    return ssd::launch_state_update(a, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? SSD_OK
+               : SSD_ERR_CUDA;
+}
+
+ssd_status ssd_i8_chunk_cb(const int8_t* C, const int8_t* B, int batch, int seqlen, int ngroups,
+                           int dstate, int chunk_size, int32_t* cb, void* stream) {
+    if (batch < 0 || seqlen < 0 || ngroups <= 0 || dstate <= 0 || chunk_size <= 0)
+        return SSD_ERR_INVALID_ARG;
+    if (!chunk_dstate_ok(dstate) || !chunk_size_ok(chunk_size)) return SSD_ERR_UNSUPPORTED;
+    if (batch == 0 || seqlen == 0) return SSD_OK;
+    if (!C || !B || !cb) return SSD_ERR_INVALID_ARG;
+    return ssd::launch_chunk_cb(C, B, batch, seqlen, ngroups, dstate, chunk_size, cb,
+                                static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? SSD_OK
+               : SSD_ERR_CUDA;
+}
+
+}  // extern "C"

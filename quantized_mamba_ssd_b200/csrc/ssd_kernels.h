@@ -1,0 +1,53 @@
+// Internal launcher interface between the C ABI (abi.cu) and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace ssd {
+
+struct ChunkScanArgs {
+    const int8_t* x;
+    const int8_t* B;
+    const int8_t* C;
+    const float* dt;
+    const float* A;
+    const float* D;
+    const float* x_scale;
+    const float* B_scale;
+    const float* C_scale;
+    int batch, seqlen, nheads, headdim, dstate, ngroups, chunk_size;
+    const float* init_state;
+    float* final_state;
+    void* y;
+    int y_dtype;
+    float inv_y_scale;
+    void* workspace;
+};
+
+struct StateUpdateArgs {
+    float* state;
+    const int8_t* x;
+    const int8_t* B;
+    const int8_t* C;
+    const float* dt;
+    const float* A;
+    const float* D;
+    const float* x_scale;
+    const float* B_scale;
+    const float* C_scale;
+    int batch, nheads, headdim, dstate, ngroups;
+    void* y;
+    int y_dtype;
+    float inv_y_scale;
+};
+
+size_t chunk_scan_workspace_bytes(int batch, int seqlen, int nheads, int headdim, int dstate,
+                                  int chunk_size);
+cudaError_t launch_chunk_scan(const ChunkScanArgs& a, cudaStream_t stream);
+cudaError_t launch_chunk_cb(const int8_t* C, const int8_t* B, int batch, int seqlen, int ngroups,
+                            int dstate, int chunk_size, int32_t* cb, cudaStream_t stream);
+cudaError_t launch_state_update(const StateUpdateArgs& a, cudaStream_t stream);
+
+}  // namespace ssd

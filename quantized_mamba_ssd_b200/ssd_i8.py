@@ -1,0 +1,206 @@
+"""Python binding of ``libssd_i8.so``: argument marshalling only.
+
+Each function takes torch CUDA tensors, checks dtype / shape / contiguity, and passes their
+device pointers to the C entry point of the same name (declared in ``include/ssd_i8.h``) on
+the current torch stream.  All arithmetic runs in the library's CUDA kernels; if the library
+is missing or fails to load, the calls raise -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libssd_i8.so")
+
+SSD_OK = 0
+STATUS_NAMES = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED",
+                3: "SSD_ERR_WORKSPACE", 4: "SSD_ERR_CUDA", 5: "SSD_ERR_TIMEOUT"}
+OUT_DTYPES = {"f32": (0, torch.float32), "f16": (1, torch.float16), "i8": (2, torch.int8)}
+
+# names of every extern "C" symbol include/ssd_i8.h declares
+EXPORTED = ("ssd_i8_abi_version", "ssd_status_string", "ssd_i8_chunk_scan_workspace_size",
+            "ssd_i8_chunk_scan", "ssd_i8_state_update", "ssd_i8_chunk_cb")
+
+# kernels one ssd_i8_chunk_scan call launches (chunk_state, state_passing, chunk_scan); the
+# benchmark reports launches from it and a GPU test checks it against a profiler count
+KERNELS_PER_CHUNK_SCAN = 3
+KERNELS_PER_STATE_UPDATE = 1
+
+_lock = threading.Lock()
+_lib: Optional[ctypes.CDLL] = None
+
+
+class SSDError(RuntimeError):
+    """A non-OK status returned by the library."""
+
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn} failed: {msg}")
+        self.status = status
+
+
+def library() -> ctypes.CDLL:
+    """Load ``libssd_i8.so`` (built by ``quantized_mamba_ssd_b200.build``) and declare types."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m quantized_mamba_ssd_b200.build` (no fallback exists)")
+        lib = ctypes.CDLL(LIB_PATH)
+        vp, ci, cf, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        lib.ssd_i8_abi_version.restype = ci
+        lib.ssd_i8_abi_version.argtypes = []
+        lib.ssd_status_string.restype = ctypes.c_char_p
+        lib.ssd_status_string.argtypes = [ci]
+        lib.ssd_i8_chunk_scan_workspace_size.restype = sz
+        lib.ssd_i8_chunk_scan_workspace_size.argtypes = [ci] * 7
+        lib.ssd_i8_chunk_scan.restype = ci
+        lib.ssd_i8_chunk_scan.argtypes = [vp] * 9 + [ci] * 7 + [vp, vp, vp, ci, cf, vp, sz, vp]
+        lib.ssd_i8_state_update.restype = ci
+        lib.ssd_i8_state_update.argtypes = [vp] * 10 + [ci] * 5 + [vp, ci, cf, vp]
+        lib.ssd_i8_chunk_cb.restype = ci
+        lib.ssd_i8_chunk_cb.argtypes = [vp, vp] + [ci] * 5 + [vp, vp]
+        _lib = lib
+        return lib
+
+
+def _check(fn: str, status: int) -> None:
+    if status != SSD_OK:
+        msg = library().ssd_status_string(status).decode()
+        raise SSDError(fn, status, msg)
+
+
+def _ptr(t: Optional[torch.Tensor], name: str, dtype: torch.dtype, shape=None) -> Optional[int]:
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t.data_ptr() if t.numel() else None
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def ssd_i8_chunk_scan_workspace_size(batch: int, seqlen: int, nheads: int, headdim: int,
+                                     dstate: int, ngroups: int, chunk_size: int) -> int:
+    return int(library().ssd_i8_chunk_scan_workspace_size(batch, seqlen, nheads, headdim, dstate,
+                                                          ngroups, chunk_size))
+
+
+def ssd_i8_chunk_scan(x: torch.Tensor, B: torch.Tensor, C: torch.Tensor, dt: torch.Tensor,
+                      A: torch.Tensor, D: torch.Tensor, x_scale: torch.Tensor,
+                      B_scale: torch.Tensor, C_scale: torch.Tensor, chunk_size: int, *,
+                      init_state: Optional[torch.Tensor] = None,
+                      final_state: Optional[torch.Tensor] = None,
+                      y: Optional[torch.Tensor] = None, y_dtype: str = "f16",
+                      y_scale: float = 1.0, workspace: Optional[torch.Tensor] = None,
+                      stream=None) -> torch.Tensor:
+    """Chunked int8 SSD scan (see ``ssd_i8_chunk_scan`` in include/ssd_i8.h).
+
+    x int8 [b,l,h,p]; B, C int8 [b,l,g,n]; dt f32 [b,l,h]; A, D, x_scale f32 [h];
+    B_scale, C_scale f32 [g]; optional init_state / final_state f32 [b,h,p,n]; returns y
+    [b,l,h,p] of ``y_dtype`` ("f32", "f16" or "i8"; "i8" uses ``y_scale``).  ``workspace`` is
+    a uint8 CUDA tensor of at least ``ssd_i8_chunk_scan_workspace_size`` bytes; one is
+    allocated through torch when omitted.
+    """
+    if x.dim() != 4 or B.dim() != 4:
+        raise ValueError("x must be [b,l,h,p] and B/C [b,l,g,n]")
+    bsz, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    code, tdt = OUT_DTYPES[y_dtype]
+    if y is None:
+        y = torch.empty((bsz, L, H, P), dtype=tdt, device=x.device)
+    need = ssd_i8_chunk_scan_workspace_size(bsz, L, H, P, N, G, chunk_size)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    args = [
+        _ptr(x, "x", torch.int8, (bsz, L, H, P)),
+        _ptr(B, "B", torch.int8, (bsz, L, G, N)),
+        _ptr(C, "C", torch.int8, (bsz, L, G, N)),
+        _ptr(dt, "dt", torch.float32, (bsz, L, H)),
+        _ptr(A, "A", torch.float32, (H,)),
+        _ptr(D, "D", torch.float32, (H,)),
+        _ptr(x_scale, "x_scale", torch.float32, (H,)),
+        _ptr(B_scale, "B_scale", torch.float32, (G,)),
+        _ptr(C_scale, "C_scale", torch.float32, (G,)),
+        bsz, L, H, P, N, G, int(chunk_size),
+        _ptr(init_state, "init_state", torch.float32, (bsz, H, P, N)),
+        _ptr(final_state, "final_state", torch.float32, (bsz, H, P, N)),
+        _ptr(y, "y", tdt, (bsz, L, H, P)),
+        code, float(y_scale),
+        _ptr(workspace, "workspace", torch.uint8),
+        workspace.numel(),
+        _stream(stream),
+    ]
+    _check("ssd_i8_chunk_scan", library().ssd_i8_chunk_scan(*args))
+    return y
+
+
+def ssd_i8_state_update(state: torch.Tensor, x: torch.Tensor, B: torch.Tensor, C: torch.Tensor,
+                        dt: torch.Tensor, A: torch.Tensor, D: torch.Tensor,
+                        x_scale: torch.Tensor, B_scale: torch.Tensor, C_scale: torch.Tensor, *,
+                        y: Optional[torch.Tensor] = None, y_dtype: str = "f16",
+                        y_scale: float = 1.0, stream=None) -> torch.Tensor:
+    """One decode step, state f32 [b,h,p,n] updated in place; x int8 [b,h,p]; B, C int8
+    [b,g,n]; dt f32 [b,h].  Returns y [b,h,p] of ``y_dtype``."""
+    bsz, H, P, N = state.shape
+    G = B.shape[1]
+    code, tdt = OUT_DTYPES[y_dtype]
+    if y is None:
+        y = torch.empty((bsz, H, P), dtype=tdt, device=state.device)
+    args = [
+        _ptr(state, "state", torch.float32, (bsz, H, P, N)),
+        _ptr(x, "x", torch.int8, (bsz, H, P)),
+        _ptr(B, "B", torch.int8, (bsz, G, N)),
+        _ptr(C, "C", torch.int8, (bsz, G, N)),
+        _ptr(dt, "dt", torch.float32, (bsz, H)),
+        _ptr(A, "A", torch.float32, (H,)),
+        _ptr(D, "D", torch.float32, (H,)),
+        _ptr(x_scale, "x_scale", torch.float32, (H,)),
+        _ptr(B_scale, "B_scale", torch.float32, (G,)),
+        _ptr(C_scale, "C_scale", torch.float32, (G,)),
+        bsz, H, P, N, G,
+        _ptr(y, "y", tdt, (bsz, H, P)),
+        code, float(y_scale),
+        _stream(stream),
+    ]
+    _check("ssd_i8_state_update", library().ssd_i8_state_update(*args))
+    return y
+
+
+def ssd_i8_chunk_cb(C: torch.Tensor, B: torch.Tensor, chunk_size: int, *,
+                    cb: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """ChunkBMM export: int32 [b, ceil(l/Q), g, Q, Q] = Cq Bq^T per chunk and group."""
+    bsz, L, G, N = C.shape
+    Q = int(chunk_size)
+    nch = (L + Q - 1) // Q
+    if cb is None:
+        cb = torch.empty((bsz, nch, G, Q, Q), dtype=torch.int32, device=C.device)
+    args = [
+        _ptr(C, "C", torch.int8, (bsz, L, G, N)),
+        _ptr(B, "B", torch.int8, (bsz, L, G, N)),
+        bsz, L, G, N, Q,
+        _ptr(cb, "cb", torch.int32, (bsz, nch, G, Q, Q)),
+        _stream(stream),
+    ]
+    _check("ssd_i8_chunk_cb", library().ssd_i8_chunk_cb(*args))
+    return cb
