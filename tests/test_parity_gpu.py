@@ -26,6 +26,12 @@ def _lib():
     ssd_i8.library()
 
 
+def mk(b, L, H, G, N, Q, **kw):
+    """A prefill case with headdim 64, sizes given as (batch, seqlen, heads, groups, dstate,
+    chunk)."""
+    return W.make_prefill(b, L, H, 64, N, G, Q, **kw)
+
+
 def dev(a, dtype=None):
     t = torch.from_numpy(np.ascontiguousarray(a))
     if dtype is not None:
@@ -76,7 +82,7 @@ def test_small_prefill_matches_oracle(b, L, H, G, N, Q, law, scales, init, out):
 
 @pytest.mark.parametrize("Q", [64, 256])
 def test_small_prefill_int8_output(Q):
-    case = W.make_prefill(2, 400, 8, 2, 128, Q, law="laplace_outliers_all", scales="head",
+    case = mk(2, 400, 8, 2, 128, Q, law="laplace_outliers_all", scales="head",
                           seed=77, with_init_state=True)
     yr, _ = oracle_scan(case)
     s_y = float(np.abs(yr).max() / 127.0)
@@ -86,7 +92,7 @@ def test_small_prefill_int8_output(Q):
 
 def test_int8_output_is_the_fp32_output_requantized():
     # the int8 epilogue must be q = clamp(rint(y * fp32(1/s_y))) of the very y the f32 path writes
-    case = W.make_prefill(1, 333, 4, 2, 128, 128, law="laplace_outliers_all", seed=5)
+    case = mk(1, 333, 4, 2, 128, 128, law="laplace_outliers_all", seed=5)
     y32, _ = gpu_scan(case, y_dtype="f32")
     s_y = np.float32(np.abs(y32).max() / 100.0)
     yq, _ = gpu_scan(case, y_dtype="i8", y_scale=float(s_y))
@@ -172,7 +178,7 @@ def test_chunk_cb_bit_exact_at_workload_size():
 # invariants and edge cases
 # ---------------------------------------------------------------------------------------
 def test_chunk_size_does_not_change_the_result():
-    case = W.make_prefill(2, 700, 4, 2, 128, 64, law="laplace_outliers_all", seed=9,
+    case = mk(2, 700, 4, 2, 128, 64, law="laplace_outliers_all", seed=9,
                           with_init_state=True)
     ys = [gpu_scan(case, chunk_size=q) for q in (64, 128, 256)]
     yr, fr = oracle_scan(case)
@@ -184,7 +190,7 @@ def test_chunk_size_does_not_change_the_result():
 
 @pytest.mark.parametrize("split", [200, 256])
 def test_split_prefill_hands_state_on(split):
-    case = W.make_prefill(2, 600, 4, 2, 128, 128, law="laplace_outliers_all", seed=10,
+    case = mk(2, 600, 4, 2, 128, 128, law="laplace_outliers_all", seed=10,
                           with_init_state=True)
     y, fs = gpu_scan(case)
     import copy
@@ -216,7 +222,7 @@ def test_decode_step_equals_length_one_prefill():
 
 
 def test_deterministic():
-    case = W.make_prefill(2, 513, 8, 2, 128, 256, law="laplace_outliers_all", seed=13,
+    case = mk(2, 513, 8, 2, 128, 256, law="laplace_outliers_all", seed=13,
                           with_init_state=True)
     y1, f1 = gpu_scan(case)
     y2, f2 = gpu_scan(case)
@@ -224,7 +230,7 @@ def test_deterministic():
 
 
 def test_empty_sequence_copies_initial_state():
-    case = W.make_prefill(2, 8, 4, 2, 128, 64, seed=14, with_init_state=True)
+    case = mk(2, 8, 4, 2, 128, 64, seed=14, with_init_state=True)
     fs = torch.full((2, 4, 64, 128), 7.0, device=DEV)
     z8 = torch.empty((2, 0, 4, 64), dtype=torch.int8, device=DEV)
     zb = torch.empty((2, 0, 2, 128), dtype=torch.int8, device=DEV)
@@ -238,7 +244,7 @@ def test_empty_sequence_copies_initial_state():
 
 
 def test_special_inputs_zero_dt_and_strong_decay():
-    case = W.make_prefill(1, 300, 4, 2, 128, 128, seed=15, with_init_state=True)
+    case = mk(1, 300, 4, 2, 128, 128, seed=15, with_init_state=True)
     case.dt[:, :100] = 0.0   # no update: state carries over unchanged
     case.dt[:, 200:] = 6.0   # exp(dt A) underflows towards zero
     y, fs = gpu_scan(case)
@@ -248,7 +254,7 @@ def test_special_inputs_zero_dt_and_strong_decay():
 
 
 def test_workspace_too_small_is_reported():
-    case = W.make_prefill(1, 100, 4, 2, 128, 64, seed=16)
+    case = mk(1, 100, 4, 2, 128, 64, seed=16)
     with pytest.raises(ssd_i8.SSDError) as ei:
         ssd_i8.ssd_i8_chunk_scan(dev(case.x), dev(case.B), dev(case.C), dev(case.dt), dev(case.A),
                                  dev(case.D), dev(case.x_scale), dev(case.B_scale),
@@ -317,3 +323,23 @@ def test_decode_workload_sampled():
                                     d.B_scale[g:g + 1], d.C_scale[g:g + 1])[0, 0])
         check_close(got, np.stack(refs), f"decode y (b={b}, h={h})")
         check_close(final[b, h], ref[0, 0], f"decode state (b={b}, h={h})")
+
+
+def test_launch_count_claim():
+    """The benchmark reports KERNELS_PER_CHUNK_SCAN launches per call; count them."""
+    from torch.profiler import ProfilerActivity, profile
+    case = mk(1, 300, 4, 2, 128, 128, seed=17)
+    ins = [dev(a) for a in (case.x, case.B, case.C, case.dt, case.A, case.D, case.x_scale,
+                            case.B_scale, case.C_scale)]
+    y = torch.empty((1, 300, 4, 64), dtype=torch.float16, device=DEV)
+    ws = torch.empty(ssd_i8.ssd_i8_chunk_scan_workspace_size(1, 300, 4, 64, 128, 2, 128),
+                     dtype=torch.uint8, device=DEV)
+    ssd_i8.ssd_i8_chunk_scan(*ins, 128, y=y, workspace=ws)
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        ssd_i8.ssd_i8_chunk_scan(*ins, 128, y=y, workspace=ws)
+        torch.cuda.synchronize()
+    kernels = [e.name for e in prof.events()
+               if e.device_type == torch.autograd.DeviceType.CUDA
+               and "Memcpy" not in e.name and "Memset" not in e.name]
+    assert len(kernels) == ssd_i8.KERNELS_PER_CHUNK_SCAN, kernels
