@@ -91,6 +91,36 @@ SSD_API ssd_status ssd_i8_chunk_scan(const int8_t *x, const int8_t *B, const int
                              float y_scale, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Allocation-free variant of ssd_i8_chunk_scan.  The pages have no counterpart: this entry point
+ * exists for callers that cannot allocate device memory when they run the scan -- code working
+ * inside a memory pool reserved in full up front, code that must not risk the device
+ * synchronisation a cudaMalloc can cause, or a plug-in whose host owns every allocation.
+ *
+ * Arguments, supported shapes and results are those of ssd_i8_chunk_scan without the workspace:
+ * the scratch comes from one array of 16 MiB compiled into the library as device memory, which
+ * every GPU that loads the library holds until the process exits.  The call allocates nothing
+ * (no cudaMalloc / cudaFree, no allocating library routine).
+ *   - Size limit: problems whose ssd_i8_chunk_scan_workspace_size(...) exceeds 16 MiB
+ *     (16777216 bytes) are rejected with SSD_ERR_WORKSPACE before anything is launched.
+ *   - Device: the scratch of the device that is current at the call is used; `stream` must
+ *     belong to that device.  The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) and caches it; make that first call before any stream capture.
+ *   - Sharing: all calls on a device share the one array and it keeps the last call's
+ *     contents.  Nothing in it needs to start at zero (every word a call reads is written
+ *     earlier in the same call), but calls whose execution overlaps on the GPU -- on different
+ *     streams, or from different host threads -- race on it and give wrong results; serialise
+ *     them (one stream, or events).
+ */
+SSD_API ssd_status ssd_i8_chunk_scan_noalloc(const int8_t *x, const int8_t *B, const int8_t *C,
+                                             const float *dt, const float *A, const float *D,
+                                             const float *x_scale, const float *B_scale,
+                                             const float *C_scale, int batch, int seqlen,
+                                             int nheads, int headdim, int dstate, int ngroups,
+                                             int chunk_size, const float *init_state,
+                                             float *final_state, void *y, int y_dtype,
+                                             float y_scale, void *stream);
+
+/*
  * Single-token decode state update, in place (the "SSD update" of the Quamba2 rebuttal's
  * generation-time discussion, Tables R7/R8): one step of the recurrence above.
  *

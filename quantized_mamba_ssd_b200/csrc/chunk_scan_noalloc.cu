@@ -1,0 +1,70 @@
+// ssd_i8_chunk_scan_noalloc: the chunk scan for callers that cannot allocate device memory.
+//
+// Some callers cannot call cudaMalloc at the point where they run the scan: code executing
+// under a fixed memory budget that was reserved up front (an inference engine that hands out
+// every byte of its pool before serving), code that must not synchronise the device (a
+// cudaMalloc can), and plug-ins of hosts that own all allocation.  For them this entry point
+// takes the scan's scratch from a fixed array compiled into the library instead of a
+// caller-provided workspace.  Everything else -- inputs, outputs, stream -- is the caller's, as
+// for ssd_i8_chunk_scan, and the same kernels run.
+//
+// The array is a file-scope __device__ variable: every GPU that loads the library holds its
+// kScratchBytes until the process exits.  In host code its name is only a host-side stand-in,
+// so its device address is looked up once per device with cudaGetSymbolAddress (with that
+// device current) and cached.
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/ssd_i8.h"
+
+namespace {
+
+// Built-in scratch: enough for the per-chunk states of problems with
+// batch * ceil(seqlen / chunk) * nheads * headdim * dstate * 4 bytes up to 16 MiB (e.g. one
+// sequence of 8192 tokens with 16 heads of 64 x 128 at chunk 256).
+constexpr size_t kScratchBytes = size_t(16) << 20;
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
+
+std::mutex g_mutex;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_scratch on the current device; looked up on the first call per device.
+ssd_status scratch_on_current_device(void** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SSD_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return SSD_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (g_scratch_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || p == nullptr) return SSD_ERR_CUDA;
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return SSD_OK;
+}
+
+}  // namespace
+
+extern "C" ssd_status ssd_i8_chunk_scan_noalloc(
+    const int8_t* x, const int8_t* B, const int8_t* C, const float* dt, const float* A,
+    const float* D, const float* x_scale, const float* B_scale, const float* C_scale, int batch,
+    int seqlen, int nheads, int headdim, int dstate, int ngroups, int chunk_size,
+    const float* init_state, float* final_state, void* y, int y_dtype, float y_scale,
+    void* stream) {
+    const size_t need = ssd_i8_chunk_scan_workspace_size(batch, seqlen, nheads, headdim, dstate,
+                                                         ngroups, chunk_size);
+    if (need > kScratchBytes) return SSD_ERR_WORKSPACE;  // problem too large for the built-in scratch
+    void* scratch = nullptr;
+    if (need > 0) {
+        const ssd_status s = scratch_on_current_device(&scratch);
+        if (s != SSD_OK) return s;
+    }
+    // Nothing in the scratch has to start at zero for this launch sequence: every word the
+    // kernels read is written earlier in the same call, so the previous call's leftovers are
+    // never observed.
+    return ssd_i8_chunk_scan(x, B, C, dt, A, D, x_scale, B_scale, C_scale, batch, seqlen, nheads,
+                             headdim, dstate, ngroups, chunk_size, init_state, final_state, y,
+                             y_dtype, y_scale, scratch, kScratchBytes, stream);
+}

@@ -24,7 +24,11 @@ OUT_DTYPES = {"f32": (0, torch.float32), "f16": (1, torch.float16), "i8": (2, to
 
 # names of every extern "C" symbol include/ssd_i8.h declares
 EXPORTED = ("ssd_i8_abi_version", "ssd_status_string", "ssd_i8_chunk_scan_workspace_size",
-            "ssd_i8_chunk_scan", "ssd_i8_state_update", "ssd_i8_chunk_cb")
+            "ssd_i8_chunk_scan", "ssd_i8_state_update", "ssd_i8_chunk_cb",
+            "ssd_i8_chunk_scan_noalloc")
+
+# built-in scratch of ssd_i8_chunk_scan_noalloc (bytes); larger problems are refused
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 # kernels one ssd_i8_chunk_scan call launches (chunk_state, state_passing, chunk_scan); the
 # benchmark reports launches from it and a GPU test checks it against a profiler count
@@ -66,6 +70,8 @@ def library() -> ctypes.CDLL:
         lib.ssd_i8_state_update.argtypes = [vp] * 10 + [ci] * 5 + [vp, ci, cf, vp]
         lib.ssd_i8_chunk_cb.restype = ci
         lib.ssd_i8_chunk_cb.argtypes = [vp, vp] + [ci] * 5 + [vp, vp]
+        lib.ssd_i8_chunk_scan_noalloc.restype = ci
+        lib.ssd_i8_chunk_scan_noalloc.argtypes = [vp] * 9 + [ci] * 7 + [vp, vp, vp, ci, cf, vp]
         _lib = lib
         return lib
 
@@ -204,3 +210,43 @@ def ssd_i8_chunk_cb(C: torch.Tensor, B: torch.Tensor, chunk_size: int, *,
     ]
     _check("ssd_i8_chunk_cb", library().ssd_i8_chunk_cb(*args))
     return cb
+
+
+def ssd_i8_chunk_scan_noalloc(x: torch.Tensor, B: torch.Tensor, C: torch.Tensor,
+                              dt: torch.Tensor, A: torch.Tensor, D: torch.Tensor,
+                              x_scale: torch.Tensor, B_scale: torch.Tensor,
+                              C_scale: torch.Tensor, chunk_size: int, *,
+                              init_state: Optional[torch.Tensor] = None,
+                              final_state: Optional[torch.Tensor] = None,
+                              y: Optional[torch.Tensor] = None, y_dtype: str = "f16",
+                              y_scale: float = 1.0, stream=None) -> torch.Tensor:
+    """The chunk scan without a workspace, for callers that cannot allocate device memory:
+    the library's built-in 16 MiB scratch (shared by all calls on a device) is used instead.
+    Pass ``y`` to keep the call itself free of allocations; larger problems raise SSDError
+    (SSD_ERR_WORKSPACE).  See ``ssd_i8_chunk_scan_noalloc`` in include/ssd_i8.h."""
+    if x.dim() != 4 or B.dim() != 4:
+        raise ValueError("x must be [b,l,h,p] and B/C [b,l,g,n]")
+    bsz, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    code, tdt = OUT_DTYPES[y_dtype]
+    if y is None:
+        y = torch.empty((bsz, L, H, P), dtype=tdt, device=x.device)
+    args = [
+        _ptr(x, "x", torch.int8, (bsz, L, H, P)),
+        _ptr(B, "B", torch.int8, (bsz, L, G, N)),
+        _ptr(C, "C", torch.int8, (bsz, L, G, N)),
+        _ptr(dt, "dt", torch.float32, (bsz, L, H)),
+        _ptr(A, "A", torch.float32, (H,)),
+        _ptr(D, "D", torch.float32, (H,)),
+        _ptr(x_scale, "x_scale", torch.float32, (H,)),
+        _ptr(B_scale, "B_scale", torch.float32, (G,)),
+        _ptr(C_scale, "C_scale", torch.float32, (G,)),
+        bsz, L, H, P, N, G, int(chunk_size),
+        _ptr(init_state, "init_state", torch.float32, (bsz, H, P, N)),
+        _ptr(final_state, "final_state", torch.float32, (bsz, H, P, N)),
+        _ptr(y, "y", tdt, (bsz, L, H, P)),
+        code, float(y_scale),
+        _stream(stream),
+    ]
+    _check("ssd_i8_chunk_scan_noalloc", library().ssd_i8_chunk_scan_noalloc(*args))
+    return y
