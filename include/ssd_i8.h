@@ -58,9 +58,10 @@ SSD_API const char *ssd_status_string(ssd_status status);
 
 /*
  * Bytes of device workspace that ssd_i8_chunk_scan needs for this problem (0 on invalid
- * sizes).  The workspace holds the per-chunk states of the chunked scan; its contents do not
- * need to be initialised and are scratch between calls.  One workspace per concurrently
- * running call.
+ * sizes): a status word, hand-off flags and one 32 KiB state slot per CTA of the persistent
+ * kernel (at most 256 CTAs, so at most about 8.4 MB).  Its contents need no initialisation:
+ * every flag and the status word are tagged with a per-call 64-bit epoch.  One workspace per
+ * concurrently running call.
  */
 SSD_API size_t ssd_i8_chunk_scan_workspace_size(int batch, int seqlen, int nheads, int headdim,
                                         int dstate, int ngroups, int chunk_size);
@@ -81,7 +82,11 @@ SSD_API size_t ssd_i8_chunk_scan_workspace_size(int batch, int seqlen, int nhead
  *   workspace  device memory of at least ssd_i8_chunk_scan_workspace_size(...) bytes,
  *              256-byte aligned.
  * Supported: headdim == 64; dstate in {16, 32, 64, 128}; seqlen >= 0 (seqlen == 0 only copies
- * init_state to final_state); batch >= 0; nheads % ngroups == 0.
+ * init_state to final_state); batch >= 0; nheads % ngroups == 0; x, B, C and y 16-byte
+ * aligned.  Expected ranges: A <= 0 and dt >= 0 (a decaying state); other values are computed
+ * but without the range guarantees the f16 operand scaling relies on.
+ * Device-side failures (a bounded wait that gave up) do not change the return value of this
+ * asynchronous call; ssd_i8_chunk_scan_status reports them.
  */
 SSD_API ssd_status ssd_i8_chunk_scan(const int8_t *x, const int8_t *B, const int8_t *C, const float *dt,
                              const float *A, const float *D, const float *x_scale,
@@ -91,25 +96,35 @@ SSD_API ssd_status ssd_i8_chunk_scan(const int8_t *x, const int8_t *B, const int
                              float y_scale, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Status of the last ssd_i8_chunk_scan call that ran on `workspace`: synchronises `stream`,
+ * then returns SSD_ERR_TIMEOUT if a device-side wait of that call gave up (a CTA waiting for its
+ * predecessor's state hand-off, or for a tensor-core / TMA completion) and SSD_OK otherwise.
+ * Every wait inside the kernels is bounded (about one second), so a failed call still
+ * terminates; its outputs are then undefined.
+ */
+SSD_API ssd_status ssd_i8_chunk_scan_status(const void *workspace, void *stream);
+
+/*
  * Allocation-free variant of ssd_i8_chunk_scan.  The pages have no counterpart: this entry point
  * exists for callers that cannot allocate device memory when they run the scan -- code working
  * inside a memory pool reserved in full up front, code that must not risk the device
  * synchronisation a cudaMalloc can cause, or a plug-in whose host owns every allocation.
  *
  * Arguments, supported shapes and results are those of ssd_i8_chunk_scan without the workspace:
- * the scratch comes from one array of 16 MiB compiled into the library as device memory, which
+ * the scratch comes from one array of 4 MiB compiled into the library as device memory, which
  * every GPU that loads the library holds until the process exits.  The call allocates nothing
  * (no cudaMalloc / cudaFree, no allocating library routine).
- *   - Size limit: problems whose ssd_i8_chunk_scan_workspace_size(...) exceeds 16 MiB
- *     (16777216 bytes) are rejected with SSD_ERR_WORKSPACE before anything is launched.
+ *   - Size limit: problems whose ssd_i8_chunk_scan_workspace_size(...) exceeds 4 MiB
+ *     (4194304 bytes; up to 127 batch x head x chunk work items) are rejected with
+ *     SSD_ERR_WORKSPACE before anything is launched.
  *   - Device: the scratch of the device that is current at the call is used; `stream` must
  *     belong to that device.  The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) and caches it; make that first call before any stream capture.
  *   - Sharing: all calls on a device share the one array and it keeps the last call's
- *     contents.  Nothing in it needs to start at zero (every word a call reads is written
- *     earlier in the same call), but calls whose execution overlaps on the GPU -- on different
- *     streams, or from different host threads -- race on it and give wrong results; serialise
- *     them (one stream, or events).
+ *     contents.  Nothing in it needs to start at zero (its flags carry a per-call epoch), but
+ *     calls whose execution overlaps on the GPU -- on different streams, or from different
+ *     host threads -- race on it and give wrong results; serialise them (one stream, or
+ *     events).
  */
 SSD_API ssd_status ssd_i8_chunk_scan_noalloc(const int8_t *x, const int8_t *B, const int8_t *C,
                                              const float *dt, const float *A, const float *D,

@@ -17,6 +17,8 @@ bool chunk_dstate_ok(int n) { return n == 16 || n == 32 || n == 64 || n == 128; 
 
 bool chunk_size_ok(int q) { return q == 64 || q == 128 || q == 256; }
 
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
 // Output scale handling shared by both entry points: I8 needs y_scale > 0 (finite); the
 // kernels multiply by its fp32 reciprocal.
 bool out_scale(int y_dtype, float y_scale, float* inv) {
@@ -84,6 +86,7 @@ ssd_status ssd_i8_chunk_scan(const int8_t* x, const int8_t* B, const int8_t* C, 
         return SSD_OK;
     }
     if (!x || !B || !C || !dt || !y) return SSD_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(B) || !aligned16(C) || !aligned16(y)) return SSD_ERR_INVALID_ARG;
     const size_t need = ssd_i8_chunk_scan_workspace_size(batch, seqlen, nheads, headdim, dstate,
                                                          ngroups, chunk_size);
     if (!workspace || workspace_bytes < need ||
@@ -125,10 +128,24 @@ ssd_status ssd_i8_chunk_cb(const int8_t* C, const int8_t* B, int batch, int seql
     if (!chunk_dstate_ok(dstate) || !chunk_size_ok(chunk_size)) return SSD_ERR_UNSUPPORTED;
     if (batch == 0 || seqlen == 0) return SSD_OK;
     if (!C || !B || !cb) return SSD_ERR_INVALID_ARG;
+    if (!aligned16(C) || !aligned16(B)) return SSD_ERR_INVALID_ARG;
     return ssd::launch_chunk_cb(C, B, batch, seqlen, ngroups, dstate, chunk_size, cb,
                                 static_cast<cudaStream_t>(stream)) == cudaSuccess
                ? SSD_OK
                : SSD_ERR_CUDA;
+}
+
+ssd_status ssd_i8_chunk_scan_status(const void* workspace, void* stream) {
+    if (!workspace) return SSD_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return SSD_ERR_CUDA;
+    unsigned long long w[3] = {0, 0, 0};
+    if (cudaMemcpy(w, workspace, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return SSD_ERR_CUDA;
+    // w[0]: epoch of the call that recorded a failure, w[1]: failure code, w[2]: epoch of the
+    // last call that ran on this workspace
+    if (w[1] != 0 && w[0] == w[2]) return SSD_ERR_TIMEOUT;
+    return SSD_OK;
 }
 
 }  // extern "C"

@@ -19,10 +19,9 @@
 
 namespace {
 
-// Built-in scratch: enough for the per-chunk states of problems with
-// batch * ceil(seqlen / chunk) * nheads * headdim * dstate * 4 bytes up to 16 MiB (e.g. one
-// sequence of 8192 tokens with 16 heads of 64 x 128 at chunk 256).
-constexpr size_t kScratchBytes = size_t(16) << 20;
+// Built-in scratch: 4 MiB, the workspace of problems with up to 127 (batch x head x chunk) work
+// items (the chunk scan hands states between CTAs through one 32 KiB slot per CTA).
+constexpr size_t kScratchBytes = size_t(4) << 20;
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
@@ -61,9 +60,9 @@ extern "C" ssd_status ssd_i8_chunk_scan_noalloc(
         const ssd_status s = scratch_on_current_device(&scratch);
         if (s != SSD_OK) return s;
     }
-    // Nothing in the scratch has to start at zero for this launch sequence: every word the
-    // kernels read is written earlier in the same call, so the previous call's leftovers are
-    // never observed.
+    // Nothing in the scratch has to start at zero: the hand-off flags and the status word are
+    // tagged with a per-call 64-bit epoch, so a previous call's leftovers never match, and a
+    // state slot is read only after its flag carries this call's epoch.
     return ssd_i8_chunk_scan(x, B, C, dt, A, D, x_scale, B_scale, C_scale, batch, seqlen, nheads,
                              headdim, dstate, ngroups, chunk_size, init_state, final_state, y,
                              y_dtype, y_scale, scratch, kScratchBytes, stream);

@@ -25,14 +25,14 @@ OUT_DTYPES = {"f32": (0, torch.float32), "f16": (1, torch.float16), "i8": (2, to
 # names of every extern "C" symbol include/ssd_i8.h declares
 EXPORTED = ("ssd_i8_abi_version", "ssd_status_string", "ssd_i8_chunk_scan_workspace_size",
             "ssd_i8_chunk_scan", "ssd_i8_state_update", "ssd_i8_chunk_cb",
-            "ssd_i8_chunk_scan_noalloc")
+            "ssd_i8_chunk_scan_noalloc", "ssd_i8_chunk_scan_status")
 
 # built-in scratch of ssd_i8_chunk_scan_noalloc (bytes); larger problems are refused
-NOALLOC_SCRATCH_BYTES = 16 << 20
+NOALLOC_SCRATCH_BYTES = 4 << 20
 
-# kernels one ssd_i8_chunk_scan call launches (chunk_state, state_passing, chunk_scan); the
-# benchmark reports launches from it and a GPU test checks it against a profiler count
-KERNELS_PER_CHUNK_SCAN = 3
+# kernels one ssd_i8_chunk_scan call launches (the fused persistent scan); the benchmark
+# reports launches from it and a GPU test checks it against a profiler count
+KERNELS_PER_CHUNK_SCAN = 1
 KERNELS_PER_STATE_UPDATE = 1
 
 _lock = threading.Lock()
@@ -70,6 +70,8 @@ def library() -> ctypes.CDLL:
         lib.ssd_i8_state_update.argtypes = [vp] * 10 + [ci] * 5 + [vp, ci, cf, vp]
         lib.ssd_i8_chunk_cb.restype = ci
         lib.ssd_i8_chunk_cb.argtypes = [vp, vp] + [ci] * 5 + [vp, vp]
+        lib.ssd_i8_chunk_scan_status.restype = ci
+        lib.ssd_i8_chunk_scan_status.argtypes = [vp, vp]
         lib.ssd_i8_chunk_scan_noalloc.restype = ci
         lib.ssd_i8_chunk_scan_noalloc.argtypes = [vp] * 9 + [ci] * 7 + [vp, vp, vp, ci, cf, vp]
         _lib = lib
@@ -212,6 +214,14 @@ def ssd_i8_chunk_cb(C: torch.Tensor, B: torch.Tensor, chunk_size: int, *,
     return cb
 
 
+def ssd_i8_chunk_scan_status(workspace: torch.Tensor, stream=None) -> None:
+    """Raise SSDError (SSD_ERR_TIMEOUT) if the last chunk scan on ``workspace`` reported a
+    device-side wait that gave up; synchronises the stream."""
+    _check("ssd_i8_chunk_scan_status",
+           library().ssd_i8_chunk_scan_status(_ptr(workspace, "workspace", torch.uint8),
+                                              _stream(stream)))
+
+
 def ssd_i8_chunk_scan_noalloc(x: torch.Tensor, B: torch.Tensor, C: torch.Tensor,
                               dt: torch.Tensor, A: torch.Tensor, D: torch.Tensor,
                               x_scale: torch.Tensor, B_scale: torch.Tensor,
@@ -221,7 +231,7 @@ def ssd_i8_chunk_scan_noalloc(x: torch.Tensor, B: torch.Tensor, C: torch.Tensor,
                               y: Optional[torch.Tensor] = None, y_dtype: str = "f16",
                               y_scale: float = 1.0, stream=None) -> torch.Tensor:
     """The chunk scan without a workspace, for callers that cannot allocate device memory:
-    the library's built-in 16 MiB scratch (shared by all calls on a device) is used instead.
+    the library's built-in 4 MiB scratch (shared by all calls on a device) is used instead.
     Pass ``y`` to keep the call itself free of allocations; larger problems raise SSDError
     (SSD_ERR_WORKSPACE).  See ``ssd_i8_chunk_scan_noalloc`` in include/ssd_i8.h."""
     if x.dim() != 4 or B.dim() != 4:

@@ -62,13 +62,14 @@ def test_workspace_size(lib):
     n = f(2, 16384, 128, 64, 128, 8, 256)
     assert n > 0 and n % 256 == 0
     assert f(-1, 10, 4, 64, 16, 1, 64) == 0
-    assert f(1, 0, 4, 64, 16, 1, 64) == 0
+    assert f(1, 0, 4, 64, 16, 1, 64) < 4096  # no work: status word and flags only
+    assert f(2, 16384, 128, 64, 128, 8, 256) <= 9 << 20  # bounded by the CTA count, not L
 
 
 def _scan_args(**over):
-    a = dict(x=1, B=1, C=1, dt=1, A=1, D=1, xs=1, bs=1, cs=1, batch=1, L=8, H=4, P=64, N=16,
-             G=1, Q=64, init=None, final=None, y=1, yd=1, ys=1.0, ws=256, wsb=1 << 20,
-             stream=None)
+    a = dict(x=256, B=256, C=256, dt=256, A=256, D=256, xs=256, bs=256, cs=256, batch=1, L=8, H=4,
+             P=64, N=16, G=1, Q=64, init=None, final=None, y=256, yd=1, ys=1.0, ws=256,
+             wsb=1 << 24, stream=None)
     a.update(over)
     return [a[k] for k in ("x", "B", "C", "dt", "A", "D", "xs", "bs", "cs", "batch", "L", "H",
                            "P", "N", "G", "Q", "init", "final", "y", "yd", "ys", "ws", "wsb",
@@ -87,6 +88,8 @@ def _scan_args(**over):
     (dict(wsb=16), 3),            # workspace too small
     (dict(ws=257), 3),            # workspace misaligned
     (dict(batch=-1), 1),
+    (dict(x=264), 1),             # x not 16-byte aligned (TMA source)
+    (dict(y=1032), 1),            # y not 16-byte aligned (vector stores)
 ])
 def test_chunk_scan_rejects_bad_arguments_on_host(lib, over, status):
     assert lib.ssd_i8_chunk_scan(*_scan_args(**over)) == status
@@ -108,9 +111,14 @@ def test_state_update_rejects_bad_arguments_on_host(lib):
 
 def test_chunk_cb_rejects_bad_arguments_on_host(lib):
     f = lib.ssd_i8_chunk_cb
-    assert f(1, 1, 1, 8, 1, 16, 100, 1, None) == 2
-    assert f(None, 1, 1, 8, 1, 16, 64, 1, None) == 1
-    assert f(1, 1, -1, 8, 1, 16, 64, 1, None) == 1
+    assert f(256, 256, 1, 8, 1, 16, 100, 256, None) == 2
+    assert f(None, 256, 1, 8, 1, 16, 64, 256, None) == 1
+    assert f(256, 256, -1, 8, 1, 16, 64, 256, None) == 1
+    assert f(264, 256, 1, 8, 1, 16, 64, 256, None) == 1  # misaligned C
+
+
+def test_status_query_rejects_null_workspace(lib):
+    assert lib.ssd_i8_chunk_scan_status(None, None) == 1
 
 
 def test_binding_refuses_cpu_tensors(lib):

@@ -253,6 +253,30 @@ def test_special_inputs_zero_dt_and_strong_decay():
     check_close(fs, fr, "final_state")
 
 
+def test_status_query_after_a_clean_call():
+    case = mk(2, 300, 8, 2, 128, 64, seed=18, with_init_state=True)
+    ws = torch.empty(ssd_i8.ssd_i8_chunk_scan_workspace_size(2, 300, 8, 64, 128, 2, 64),
+                     dtype=torch.uint8, device=DEV)
+    ssd_i8.ssd_i8_chunk_scan(dev(case.x), dev(case.B), dev(case.C), dev(case.dt), dev(case.A),
+                             dev(case.D), dev(case.x_scale), dev(case.B_scale), dev(case.C_scale),
+                             64, workspace=ws)
+    ssd_i8.ssd_i8_chunk_scan_status(ws)  # raises on a device-side timeout
+
+
+@pytest.mark.parametrize("b,L,H,G,Q", [(1, 4096, 2, 1, 256), (3, 1000, 50, 5, 128),
+                                       (1, 64 * 300, 1, 1, 64)])
+def test_range_split_hand_offs(b, L, H, G, Q):
+    # work lists whose per-CTA ranges split sequences mid-way (one unit over many CTAs, and
+    # ranges covering several units) exercise the state hand-off between CTAs
+    case = mk(b, L, H, G, 128, Q, law="laplace_outliers_all", seed=L + H, with_init_state=True)
+    y, fs = gpu_scan(case)
+    pairs = [(0, 0), (b - 1, H - 1)]
+    for bb, hh in pairs:
+        yr, fr, _ = oracle.scan(**head_subset(case, [hh], batches=[bb]))
+        check_close(y[bb, :, hh, :], yr[0, :, 0, :], f"y[b={bb},h={hh}]")
+        check_close(fs[bb, hh], fr[0, 0], f"final_state[b={bb},h={hh}]")
+
+
 def test_workspace_too_small_is_reported():
     case = mk(1, 100, 4, 2, 128, 64, seed=16)
     with pytest.raises(ssd_i8.SSDError) as ei:
