@@ -211,6 +211,10 @@ def main():
     ap.add_argument("--decode-passes", type=int, default=3,
                     help="timed passes of the 512-step decode run (0 skips the decode report)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) leg")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="sequences per rank (default: the workload's batch of 2); a smaller "
+                         "batch of the same shape serves profiling captures")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -241,7 +245,8 @@ def main():
     int8_peak_tops = bf16_peak * INT8_PER_BF16
 
     # ---- prefill workload: this rank's own batch (seeded per rank) ----
-    case = W.make_prefill_config(PREFILL_CFG, seed=1000 + PREFILL_CFG + 97 * rank)
+    overrides = {} if args.batch is None else {"batch": args.batch}
+    case = W.make_prefill_config(PREFILL_CFG, seed=1000 + PREFILL_CFG + 97 * rank, **overrides)
     x, B, C = (torch.from_numpy(a).to(dev) for a in (case.x, case.B, case.C))
     dt = torch.from_numpy(case.dt).to(dev)
     A, Dp, sx, sb, sc = (torch.from_numpy(a).to(dev) for a in
@@ -301,21 +306,24 @@ def main():
         step()
         hy.copy_(y, non_blocking=True)
 
-    e2e_steps = max(3, min(args.steps, 10))
-    for _ in range(3):
-        e2e_step()
-    torch.cuda.synchronize()
-    barrier()
-    ev0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    t = torch.tensor([ev0.elapsed_time(ev1) / e2e_steps], device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_value = tokens_all / (float(t.item()) * 1e-3)
+    e2e = None
+    if not args.no_e2e:
+        e2e_steps = max(3, min(args.steps, 10))
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        ev0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        t = torch.tensor([ev0.elapsed_time(ev1) / e2e_steps], device=dev)
+        if world > 1:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e = {"value": tokens_all / (float(t.item()) * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     # ---- roofline of the timed call ----
     alg_bytes = prefill_alg_bytes(case, 1, True)
@@ -401,8 +409,7 @@ def main():
                        "l2": "inputs larger than L2 (x 268 MB + B,C 67 MB + dt 17 MB per rank)"},
             "roofline": roofline,
             "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
+            "e2e": e2e,
             "gpu_launches": args.steps * ssd_i8.KERNELS_PER_CHUNK_SCAN,
             "clocks": clocks.summary(),
             "decode": decode,

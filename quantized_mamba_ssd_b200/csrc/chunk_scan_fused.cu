@@ -1,25 +1,37 @@
-// Fused int8 SSD chunk scan for sm_100a: one persistent CTA per SM, tcgen05 tensor cores,
-// TMA-staged int8 tiles, the running state kept in tensor memory.
+// Fused int8 SSD chunk scan for sm_100a: one persistent, warp-specialised CTA per SM, tcgen05
+// tensor cores, TMA-staged int8 tiles, the running state kept in tensor memory.
 //
-// Work: units u = (batch, head), each a sequence of nch = ceil(L / Q) chunks.  The flattened
-// (unit, chunk) list is cut into one contiguous range per CTA, so every SM gets the same
-// number of chunks.  A range holds at most one unit piece that starts mid-sequence (its first)
-// and one that ends mid-sequence (its last).  The CTA runs its last piece first and publishes
-// the state at its end to a workspace slot; it runs its first piece last, after reading the
-// predecessor CTA's slot (a bounded wait).  With at least nch chunks per CTA the slot is
-// always ready by then.
+// Work: units u = (batch, head), each a sequence of nblk = ceil(L / 128) blocks of 128 tokens.
+// The flattened (unit, block) list is cut into one contiguous range per CTA, so every SM gets
+// the same number of blocks.  A range holds at most one unit piece that starts mid-sequence
+// (its first) and one that ends mid-sequence (its last).  The CTA runs its last piece first and
+// publishes the state at its end to a workspace slot; it runs its first piece last, after
+// reading the predecessor CTA's slot (a bounded wait).  With at least nblk blocks per CTA the
+// slot is always ready by then.
 //
-// Per chunk of Q tokens and one head (SSDi8 page: ChunkState, state path, ChunkScan,
-// ChunkBMM of Table 5; X_scaled of Figure 3(a)):
-//   Acum_t = sum_{k<=t} dt_k A_h                     block scan, fp32
-//   CB     = Cq Bq^T                                  tcgen05 kind::i8, exact int32 in TMEM
-//   M'     = CB * exp(Acum_t - Acum_s) * dt_s / kappa  (s <= t), f16, written over CB in TMEM
-//   acc    = C' H'^T + M' x                           tcgen05 kind::f16, A from TMEM
-//            C'[t,n] = Cq[t,n] exp(Acum_t),  H' = H / kappa
-//   y      = s_C s_x s_B kappa acc + D s_x xq           fused epilogue (f32 / f16 / int8)
-//   H     <- exp(Acum_end) H + B'^T x,  B'[t,n] = Bq[t,n] dt_t exp(Acum_end - Acum_t)
-// H is kept in units of s_x s_B.  Only the operands that are not int8 (M', C', B', H') are
-// rounded, once each, to f16 (relative 2^-12); kappa keeps them inside f16 range.
+// The chunked scan is evaluated in blocks of 128 tokens (SSDi8 page: ChunkState, state path,
+// ChunkScan, ChunkBMM of Table 5; X_scaled of Figure 3(a)).  This is the same recurrence for
+// any chunk length, so the result depends on the caller's chunk size only through rounding.
+// Per block and head, with Acum_t = sum_{k<=t} dt_k A_h inside the block:
+//   CB    = Cq Bq^T                                   tcgen05 kind::i8, exact int32 in TMEM
+//   M'    = CB * exp(Acum_t - Acum_s) * dt_s / kappa   (s <= t), plus D s_x / rho on the
+//           diagonal; f16, written over CB in TMEM
+//   acc   = C' H'^T + M' x                             tcgen05 kind::f16, A from TMEM
+//           C'[t,n] = Cq[t,n] exp(Acum_t),  H' = (H / s_x s_B) / kappa
+//   y     = rho * acc,  rho = s_C s_x s_B kappa (a power of two)
+//   H    <- exp(Acum_end) H + B'^T x,  B'[t,n] = Bq[t,n] dt_t exp(Acum_end - Acum_t) / U
+// H lives in TMEM in units of s_x s_B U, U a per-block power of two that keeps B' inside f16
+// range; kappa comes from a running bound on |H| so that no reduction over the state is
+// needed.  Only the non-int8 operands (M', C', B', H') are rounded, once each, to f16.
+//
+// Warp roles, coupled only through mbarriers (buffers alternate with the block parity j):
+//   warp 8      TMA: x, B, C tiles of block k into stage j            (waits: stage free)
+//   warp 9      MMA issue: CB(k); state(k), C'H(k); M'x(k)            (waits: tiles, operands)
+//   warps 0-3   prep: block scan of dt*A, state hand-over (H', decay), x / B' / C' conversions,
+//               piece start / end (initial state, hand-off slot, final state)
+//   warps 4-7   M' from CB(k); output of block k-1 while the tensor core runs block k
+// Every wait is bounded; a timeout sets a status word and turns the remaining waits into
+// no-ops so that the kernel still ends (its outputs are then undefined).
 #include <algorithm>
 #include <atomic>
 #include <mutex>
@@ -34,36 +46,54 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 128;  // one warpgroup: thread i <-> TMEM lane i
-constexpr int kP = 64;         // headdim
-constexpr int kTB = 128;       // rows of a t-block (MMA M)
+constexpr int kThreads = 320;   // 10 warps (see the role table above)
+constexpr int kWarpTma = 8, kWarpMma = 9;
+constexpr int kP = 64;          // headdim
+constexpr int kBlk = 128;       // tokens per block (MMA M)
 constexpr long long kWaitCycles = 1ll << 31;  // bound of every device-side wait (~1 s)
-constexpr int kMaxCtas = 256;  // workspace slots
+constexpr int kMaxCtas = 256;   // workspace slots
+constexpr float kF16Range = 16384.f;  // target magnitude of the f16 operands (2^14)
 
 // tensor memory columns (512 allocated)
-constexpr uint32_t kColCB = 0;     // 256: CB int32; M' f16 pairs written over it
-constexpr uint32_t kColAcc = 256;  // 64: y accumulator f32 [t][p]
-constexpr uint32_t kColC = 320;    // 64: C' f16 pairs [t][n]
-constexpr uint32_t kColH = 384;    // 64: state f32 [n][p]
+constexpr uint32_t kColCB = 0;     // 2 x 128: CB int32 per buffer; M' f16 pairs over cols 0..63
+constexpr uint32_t kColAcc = 256;  // 2 x 64: y accumulator f32 [t][p]
+constexpr uint32_t kColC = 384;    // 64: C' f16 pairs [t][n]
+constexpr uint32_t kColH = 448;    // 64: state f32 [n][p]
 constexpr uint32_t kTmemCols = 512;
 
-template <int Q>
-struct Layout {
-    static constexpr int kC = 0;                        // Cq  [Q][128 B], 128B swizzle
-    static constexpr int kB = kC + Q * 128;             // Bq  [Q][128 B], 128B swizzle
-    static constexpr int kXf = kB + Q * 128;            // x f16 [Q][64] (MN-major, swizzled)
-    static constexpr int kBp = kXf + Q * 128;           // B' f16 2 x [Q][64] (MN-major)
-    static constexpr int kHp = kBp + 2 * Q * 128;       // H' f16 [128 n][64 p] (MN-major)
-    static constexpr int kX = kHp + 128 * 128;          // xq [Q][64 B], dense
-    static constexpr int kDt = kX + Q * 64;             // dt [256] f32
-    static constexpr int kAcum = kDt + 256 * 4;         // Acum [256] f32
-    static constexpr int kRed = kAcum + 256 * 4;        // reduction scratch [64] f32
-    static constexpr int kBar = kRed + 64 * 4;          // 4 mbarriers
-    static constexpr int kMisc = kBar + 4 * 8;          // tmem base, abort flag
-    static constexpr int kBytes = kMisc + 16;
-    static constexpr int kAlloc = kBytes + 1024;        // + alignment slack
-    static_assert(kXf % 1024 == 0 && kBp % 1024 == 0 && kHp % 1024 == 0 && kB % 1024 == 0,
-                  "swizzled tiles must be 1024-byte aligned");
+// shared memory (offsets from a 1024-byte aligned base)
+constexpr int kStageBytes = 40960;  // C [128][128 B], B [128][128 B] (128B swizzle), X [128][64 B]
+constexpr int kStC = 0, kStB = 16384, kStX = 32768;
+constexpr int kOffXf = 2 * kStageBytes;         // x f16 [128 t][64 p] MN-major, 2 buffers
+constexpr int kOffBp = kOffXf + 2 * 16384;      // B' f16 2 x [128 t][64 n] MN-major, 2 buffers
+constexpr int kOffHp = kOffBp + 2 * 32768;      // H' f16 [128 n][64 p] MN-major, 2 buffers
+constexpr int kOffColf = kOffHp + 2 * 16384;    // column factors [2][4][128] f32
+constexpr int kOffDt = kOffColf + 2 * 2048;     // dt [2][128]
+constexpr int kOffAcum = kOffDt + 2 * 512;      // Acum [2][128]
+constexpr int kOffInfo = kOffAcum + 2 * 512;    // per-block info [2]
+constexpr int kOffRed = kOffInfo + 2 * 64;      // prep scratch [32] f32
+constexpr int kOffBar = kOffRed + 128;          // mbarriers [16]
+constexpr int kOffMisc = kOffBar + 16 * 8;      // TMEM base, abort flag
+constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+static_assert(kOffXf % 1024 == 0 && kOffBp % 1024 == 0 && kOffHp % 1024 == 0, "alignment");
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+
+enum {
+    kBarFull0 = 0, kBarFull1,      // tiles of stage j landed (TMA transaction count)
+    kBarEmpty0, kBarEmpty1,        // stage j consumed: prep arrival + ChunkBMM commit
+    kBarCb0, kBarCb1,              // CB(k) in TMEM buffer j
+    kBarPrep0, kBarPrep1,          // operands of block k ready (prep warpgroup)
+    kBarMp0, kBarMp1,              // M'(k) in TMEM buffer j
+    kBarAcc0, kBarAcc1,            // accumulator j complete (M'x(k) done)
+    kBarAccFree0, kBarAccFree1,    // accumulator j read out
+    kBarState,                     // state update of the last issued block done
+    kBarCh,                        // C'.H' of the last issued block done (C' columns free)
+    kNumBars
+};
+
+struct BlockInfo {  // handed from the prep warpgroup to the M' / output warpgroup
+    float rho, inv_kappa, dterm, pad;
+    int b, h, c, valid;
 };
 
 struct FusedParams {
@@ -78,17 +108,70 @@ struct FusedParams {
     void* y;
     int y_dtype;
     float inv_y_scale;
-    int batch, L, H, G, N, nch, nctas;
-    long long total;  // batch * H * nch
-    float* slots;     // [nctas][128 n][64 p] handed-off states (units of s_x s_B)
+    int batch, L, H, G, N, nblk, nctas;
+    long long total;             // batch * H * nblk
+    float* slots;                // [nctas][128 n][64 p] handed-off states, units of s_x s_B
     unsigned long long* flags;   // [nctas] epoch of the published slot
     unsigned long long* status;  // [3]: epoch and code of a device-side failure, last epoch
     unsigned long long epoch;
 };
 
+// the pieces of this CTA's range, in processing order (last piece first, first piece last)
+struct Range {
+    long long ws, we, u_first, u_last;
+    int nseg, nblk, H;
+    __device__ void init(const FusedParams& p) {
+        const long long W = p.total;
+        ws = W * blockIdx.x / p.nctas;
+        we = W * (blockIdx.x + 1) / p.nctas;
+        nblk = p.nblk;
+        H = p.H;
+        u_first = ws / nblk;
+        u_last = we > ws ? (we - 1) / nblk : u_first;
+        nseg = we > ws ? static_cast<int>(u_last - u_first + 1) : 0;
+    }
+    __device__ void seg(int k, int& b, int& h, int& c_begin, int& c_end) const {
+        const long long u = (k == 0) ? u_last : (k == nseg - 1 ? u_first : u_first + k);
+        c_begin = static_cast<int>(u == u_first ? ws - u * nblk : 0);
+        c_end = static_cast<int>(u == u_last ? we - u * nblk : nblk);
+        b = static_cast<int>(u / H);
+        h = static_cast<int>(u % H);
+    }
+};
+
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
     const __half2 h = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+__device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, __half2 s) {
+    __half2 v = *reinterpret_cast<__half2*>(&a);
+    v = __hmul2(v, s);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// four int8 (one word) -> two f16x2, exact: (b ^ 0x80) placed in the mantissa of 1024.0,
+// minus 1152 (= 1024 + 128)
+__device__ __forceinline__ void i8x4_to_h2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    const uint32_t u = w ^ 0x80808080u;
+    uint32_t a = __byte_perm(u, 0x64646464u, 0x4140);
+    uint32_t b = __byte_perm(u, 0x64646464u, 0x4342);
+    const __half2 bias = __half2half2(__ushort_as_half(0x6480));
+    __half2 ha = __hsub2(*reinterpret_cast<__half2*>(&a), bias);
+    __half2 hb = __hsub2(*reinterpret_cast<__half2*>(&b), bias);
+    lo = *reinterpret_cast<uint32_t*>(&ha);
+    hi = *reinterpret_cast<uint32_t*>(&hb);
+}
+
+// exact int32 -> float for |v| < 2^22 (ChunkBMM entries: |CB| <= 127^2 * 128)
+__device__ __forceinline__ float i32_to_f32_small(uint32_t v) {
+    return __int_as_float(static_cast<int>(v) + 0x4B400000) - 12582912.0f;
+}
+
+// fp32 -> int8 code: round half to even, clamp to [-127, 127]
+__device__ __forceinline__ uint32_t q8(float v) {
+    v = fminf(fmaxf(v, -127.f), 127.f);
+    return __float_as_uint(v + 12582912.0f) & 0xffu;
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
@@ -101,22 +184,16 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
         : "memory");
 }
 
-// int8x4 (one 32-bit word) -> 4 floats
-__device__ __forceinline__ void i8x4_to_f32(uint32_t w, float* f) {
-    f[0] = static_cast<float>(static_cast<int8_t>(w & 0xff));
-    f[1] = static_cast<float>(static_cast<int8_t>((w >> 8) & 0xff));
-    f[2] = static_cast<float>(static_cast<int8_t>((w >> 16) & 0xff));
-    f[3] = static_cast<float>(static_cast<int8_t>(w >> 24));
+// barrier among the 128 threads of one warpgroup (id 1: prep, id 2: M' / output)
+__device__ __forceinline__ void wg_sync(int id) {
+    asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
 }
 
-__device__ __forceinline__ float block_max(float v, float* red) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    const int warp = threadIdx.x / 32;
-    __syncthreads();
-    if ((threadIdx.x & 31) == 0) red[warp] = v;
-    __syncthreads();
-    return fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+// smallest power of two >= v (v > 0, finite)
+__device__ __forceinline__ float pow2_ceil(float v) {
+    int e;
+    const float m = frexpf(v, &e);  // v = m * 2^e, m in [0.5, 1)
+    return ldexpf(1.f, m == 0.5f ? e - 1 : e);
 }
 
 __device__ void report_failure(const FusedParams& p, unsigned long long code) {
@@ -125,9 +202,25 @@ __device__ void report_failure(const FusedParams& p, unsigned long long code) {
     atomicExch(p.status, p.epoch);
 }
 
-// Issue the ChunkBMM MMAs: D[tmem] = C rows [t0, t0+128) x B rows [0, ncols), K = 128 (int8).
+// Bounded wait that gives up at once after any failure of the CTA.
+__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity,
+                                           volatile uint32_t* abort_flag, const FusedParams& p) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort_flag) return false;
+        if (clock64() - t0 > kWaitCycles) {
+            *abort_flag = 1;
+            report_failure(p, 1);
+            return false;
+        }
+    }
+    return true;
+}
+
+// ChunkBMM MMAs: D[tmem] = C rows [t0, t0+128) x B rows [0, ncols), K = 128 (int8).
 __device__ __forceinline__ void issue_cb(uint32_t d, uint32_t sC, uint32_t sB, int t0, int ncols) {
-    const uint32_t id = idesc_i8(kTB, ncols, false, false);
+    const uint32_t id = idesc_i8(kBlk, ncols, false, false);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         const uint64_t a = smem_desc(sC + t0 * 128 + 32 * k, 16, 1024, kSwizzle128B);
@@ -136,47 +229,29 @@ __device__ __forceinline__ void issue_cb(uint32_t d, uint32_t sC, uint32_t sB, i
     }
 }
 
-template <int Q>
 __global__ void __launch_bounds__(kThreads, 1)
 fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                         const __grid_constant__ CUtensorMap map_B,
                         const __grid_constant__ CUtensorMap map_C, const FusedParams p) {
-    using Lay = Layout<Q>;
-    constexpr int NTB = Q > kTB ? Q / kTB : 1;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint8_t* sC = smem + Lay::kC;
-    uint8_t* sB = smem + Lay::kB;
-    uint8_t* sXf = smem + Lay::kXf;
-    uint8_t* sBp = smem + Lay::kBp;
-    uint8_t* sHp = smem + Lay::kHp;
-    const uint8_t* sX = smem + Lay::kX;
-    float* dts = reinterpret_cast<float*>(smem + Lay::kDt);
-    float* acum = reinterpret_cast<float*>(smem + Lay::kAcum);
-    float* red = reinterpret_cast<float*>(smem + Lay::kRed);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
-    uint64_t* bar_tma = bars + 0;
-    uint64_t* bar_cb = bars + 1;
-    uint64_t* bar_acc = bars + 2;
-    uint64_t* bar_state = bars + 3;
-    uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lay::kMisc);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+    uint32_t* misc = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile uint32_t* abort_flag = misc + 1;
+    BlockInfo* info = reinterpret_cast<BlockInfo*>(smem + kOffInfo);
 
     const int tid = threadIdx.x;
-    const int warp = tid / 32;
-    const uint32_t lane_base = static_cast<uint32_t>(warp) * 32u;
+    const int warp = tid >> 5, lane = tid & 31;
 
     if (tid == 0) {
-        for (int i = 0; i < 4; ++i) mbar_init(bars + i, 1);
+        for (int i = 0; i < kNumBars; ++i)
+            mbar_init(bars + i, (i == kBarEmpty0 || i == kBarEmpty1) ? 2 : 1);
         fence_mbar_init();
         *abort_flag = 0;
         if (blockIdx.x == 0) p.status[2] = p.epoch;  // the call the status word refers to
-        tma_prefetch_map(&map_x);
-        tma_prefetch_map(&map_B);
-        tma_prefetch_map(&map_C);
     }
-    if (warp == 0) {
+    if (warp == kWarpMma) {
         tmem_alloc(misc, kTmemCols);
         tmem_relinquish();
     }
@@ -184,406 +259,501 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = misc[0];
-    uint32_t ph_tma = 0, ph_cb = 0, ph_acc = 0, ph_state = 0;
-    bool tma_in_flight = false;
+    Range rg;
+    rg.init(p);
+    const int nb_total = static_cast<int>(rg.we - rg.ws);
 
-    // wait helper: every thread waits; a timeout raises the CTA-wide abort flag
-    auto wait_bar = [&](uint64_t* bar, uint32_t& phase) {
-        if (!mbar_wait(bar, phase, kWaitCycles)) *abort_flag = 1;
-        phase ^= 1u;
-    };
-
-    const long long W = p.total;
-    const int cta = blockIdx.x;
-    const long long ws = W * cta / p.nctas, we = W * (cta + 1) / p.nctas;
-    const int nch = p.nch;
-    const long long u_first = ws / nch, u_last = (we - 1) / nch;
-    const int nseg = we > ws ? static_cast<int>(u_last - u_first + 1) : 0;
-
-    for (int k = 0; k < nseg && !*abort_flag; ++k) {
-        const long long u = (k == 0) ? u_last : (k == nseg - 1 ? u_first : u_first + k);
-        const int c_begin = static_cast<int>(u == u_first ? ws - u * nch : 0);
-        const int c_end = static_cast<int>(u == u_last ? we - u * nch : nch);
-        const int b = static_cast<int>(u / p.H), h = static_cast<int>(u % p.H);
-        const int g = h / (p.H / p.G);
-        const float sx = p.x_scale[h], sBg = p.B_scale[g], sCg = p.C_scale[g];
-        const float sigma = sx * sBg;
-        const float A_h = p.A[h], Dsx = p.D[h] * sx;
-        const int N = p.N;
-        const int n = tid;  // state row owned by this thread (TMEM lane)
-
-        // ---- initial state of the piece -> H (TMEM lanes = n, columns = p) ----
-        {
-            const float* src = nullptr;
-            float scale = 1.f / sigma;
-            if (c_begin == 0) {
-                if (p.init_state) src = p.init_state + ((size_t)b * p.H + h) * kP * N;
-            } else {
-                if (tid == 0) {
-                    const unsigned long long* f = p.flags + (cta - 1);
-                    const long long t0 = clock64();
-                    unsigned long long v;
-                    for (;;) {
-                        asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(f) : "memory");
-                        if (v == p.epoch) break;
-                        if (clock64() - t0 > kWaitCycles) {
-                            report_failure(p, 2);
-                            *abort_flag = 1;
-                            break;
-                        }
-                        __nanosleep(256);
-                    }
+    if (warp == kWarpTma) {
+        // ============================== TMA producer ==============================
+        if (lane == 0) {
+            tma_prefetch_map(&map_x);
+            tma_prefetch_map(&map_B);
+            tma_prefetch_map(&map_C);
+            int kb = 0;
+            for (int k = 0; k < rg.nseg; ++k) {
+                int b, h, cb, ce;
+                rg.seg(k, b, h, cb, ce);
+                const int g = h / (p.H / p.G);
+                for (int c = cb; c < ce; ++c, ++kb) {
+                    const int s = kb & 1;
+                    if (kb >= 2) wait_phase(bars + kBarEmpty0 + s, ((kb >> 1) - 1) & 1, abort_flag, p);
+                    uint8_t* stage = smem + s * kStageBytes;
+                    uint64_t* bar = bars + kBarFull0 + s;
+                    mbar_arrive_expect_tx(bar, kStageBytes);
+                    tma_load_4d(stage + kStX, &map_x, 0, h, c * kBlk, b, bar);
+                    tma_load_4d(stage + kStB, &map_B, 0, g, c * kBlk, b, bar);
+                    tma_load_4d(stage + kStC, &map_C, 0, g, c * kBlk, b, bar);
                 }
-                __syncthreads();
-                if (*abort_flag) break;
-                src = p.slots + (size_t)(cta - 1) * 128 * kP;
-                scale = 1.f;
             }
-            uint32_t r[32];
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int pp = half * 32 + j;
-                    float v = 0.f;
-                    if (src != nullptr && n < N)
-                        v = (c_begin == 0) ? src[(size_t)pp * N + n] * scale : __ldcg(src + n * kP + pp);
-                    r[j] = __float_as_uint(v);
-                }
-                tmem_st32(tmem_addr(tmem, lane_base, kColH + half * 32), r);
-            }
-            tmem_st_wait();
+            // drain: both stages' last loads must have landed before the CTA exits
+            for (int kb2 = nb_total > 2 ? nb_total - 2 : 0; kb2 < nb_total; ++kb2)
+                mbar_wait(bars + kBarFull0 + (kb2 & 1), (kb2 >> 1) & 1, kWaitCycles);
         }
-
-        for (int c = c_begin; c < c_end; ++c) {
-            const int t_base = c * Q;
-            const int valid = min(Q, p.L - t_base);
-            // ---- TMA: x, B, C tiles of the chunk (zero past the sequence end) ----
-            if (tid == 0) {
-                mbar_arrive_expect_tx(bar_tma, Q * 128 * 2 + Q * 64);
-                tma_load_4d(smem + Lay::kX, &map_x, 0, h, t_base, b, bar_tma);
-                tma_load_4d(sB, &map_B, 0, g, t_base, b, bar_tma);
-                tma_load_4d(sC, &map_C, 0, g, t_base, b, bar_tma);
-            }
-            tma_in_flight = true;
-            // ---- chunk_cumsum: Acum_t (inclusive), two tokens per thread ----
-            float dmax;
-            {
-                const int t0 = 2 * tid, t1 = 2 * tid + 1;
-                const float* dtp = p.dt + ((size_t)b * p.L + t_base) * p.H + h;
-                const float d0 = (t0 < valid) ? dtp[(size_t)t0 * p.H] : 0.f;
-                const float d1 = (t1 < valid) ? dtp[(size_t)t1 * p.H] : 0.f;
-                const float a0 = d0 * A_h, a1 = d1 * A_h;
-                const float incl = block_inclusive_scan(a0 + a1, red);
-                const float excl = incl - (a0 + a1);
-                if (t0 < Q) {
-                    dts[t0] = d0;
-                    acum[t0] = excl + a0;
-                }
-                if (t1 < Q) {
-                    dts[t1] = d1;
-                    acum[t1] = excl + a0 + a1;
-                }
-                dmax = block_max(fmaxf(d0, d1), red + 32);
-            }
-            __syncthreads();
-            const float a_end = acum[Q - 1];
-            const float decay_end = __expf(a_end);
-
-            // ---- chunk boundary: H' = f16(H / kappa) for C'.H', then H <- exp(Acum_end) H ----
-            float kappa;
-            {
-                uint32_t hv[2][32];
-                tmem_ld32(tmem_addr(tmem, lane_base, kColH), hv[0]);
-                tmem_ld32(tmem_addr(tmem, lane_base, kColH + 32), hv[1]);
-                tmem_ld_wait();
-                float m = 0.f;
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(__uint_as_float(hv[hh][j])));
-                const float hmax = block_max(m, red + 40);
-                kappa = fmaxf(hmax, 16129.f * static_cast<float>(N) * dmax) * (1.f / 16384.f);
-                if (!(kappa > 1e-30f) || !isfinite(kappa)) kappa = 1.f;
-                const float inv_k = 1.f / kappa;
-                // H' row n: 64 f16 = 128 bytes, 8 swizzled 16-byte chunks
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    const int hh = ch / 4, j0 = (ch % 4) * 8;
-                    uint4 v;
-                    v.x = pack_f16x2(__uint_as_float(hv[hh][j0 + 0]) * inv_k, __uint_as_float(hv[hh][j0 + 1]) * inv_k);
-                    v.y = pack_f16x2(__uint_as_float(hv[hh][j0 + 2]) * inv_k, __uint_as_float(hv[hh][j0 + 3]) * inv_k);
-                    v.z = pack_f16x2(__uint_as_float(hv[hh][j0 + 4]) * inv_k, __uint_as_float(hv[hh][j0 + 5]) * inv_k);
-                    v.w = pack_f16x2(__uint_as_float(hv[hh][j0 + 6]) * inv_k, __uint_as_float(hv[hh][j0 + 7]) * inv_k);
-                    *reinterpret_cast<uint4*>(sHp + sw128(n, ch * 16)) = v;
-                }
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        hv[hh][j] = __float_as_uint(__uint_as_float(hv[hh][j]) * decay_end);
-                    tmem_st32(tmem_addr(tmem, lane_base, kColH + hh * 32), hv[hh]);
-                }
-                tmem_st_wait();
-            }
-
-            // ---- wait for the tiles, then convert x -> f16 and B -> B' (f16) ----
-            wait_bar(bar_tma, ph_tma);
-            tma_in_flight = false;
-            for (int t = tid; t < Q; t += kThreads) {
-                // x row t: 64 int8 (dense) -> 64 f16 (swizzled 128-byte row)
-                const uint4* xs = reinterpret_cast<const uint4*>(sX + t * 64);
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const uint4 w = xs[q4];
-                    const uint32_t ws4[4] = {w.x, w.y, w.z, w.w};
-                    float f[16];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) i8x4_to_f32(ws4[i], f + 4 * i);
-                    uint4 o0, o1;
-                    o0.x = pack_f16x2(f[0], f[1]);   o0.y = pack_f16x2(f[2], f[3]);
-                    o0.z = pack_f16x2(f[4], f[5]);   o0.w = pack_f16x2(f[6], f[7]);
-                    o1.x = pack_f16x2(f[8], f[9]);   o1.y = pack_f16x2(f[10], f[11]);
-                    o1.z = pack_f16x2(f[12], f[13]); o1.w = pack_f16x2(f[14], f[15]);
-                    *reinterpret_cast<uint4*>(sXf + sw128(t, q4 * 32)) = o0;
-                    *reinterpret_cast<uint4*>(sXf + sw128(t, q4 * 32 + 16)) = o1;
-                }
-                // B row t (128-byte swizzled int8) scaled by w_t -> B' (two 64-column blocks)
-                const float w_t = (t < valid) ? dts[t] * __expf(a_end - acum[t]) : 0.f;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint4 w = *reinterpret_cast<const uint4*>(sB + sw128(t, j * 16));
-                    const uint32_t ws4[4] = {w.x, w.y, w.z, w.w};
-                    float f[16];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) i8x4_to_f32(ws4[i], f + 4 * i);
-                    uint4 o0, o1;
-                    o0.x = pack_f16x2(f[0] * w_t, f[1] * w_t);   o0.y = pack_f16x2(f[2] * w_t, f[3] * w_t);
-                    o0.z = pack_f16x2(f[4] * w_t, f[5] * w_t);   o0.w = pack_f16x2(f[6] * w_t, f[7] * w_t);
-                    o1.x = pack_f16x2(f[8] * w_t, f[9] * w_t);   o1.y = pack_f16x2(f[10] * w_t, f[11] * w_t);
-                    o1.z = pack_f16x2(f[12] * w_t, f[13] * w_t); o1.w = pack_f16x2(f[14] * w_t, f[15] * w_t);
-                    uint8_t* blk = sBp + (j / 4) * (Q * 128);
-                    *reinterpret_cast<uint4*>(blk + sw128(t, (j % 4) * 32)) = o0;
-                    *reinterpret_cast<uint4*>(blk + sw128(t, (j % 4) * 32 + 16)) = o1;
-                }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncthreads();
-            tc_fence_after();
-            if (*abort_flag) break;
-
-            // ---- state update MMA: H += B'^T x  (M = 128 n, N = 64 p, K = Q) ----
-            if (tid == 0) {
-                const uint32_t id = idesc_f16(128, kP, true, true);
-#pragma unroll 4
-                for (int kk = 0; kk < Q / 16; ++kk) {
-                    const uint64_t a = smem_desc(smem_u32(sBp) + 2048 * kk, Q * 128, 1024, kSwizzle128B);
-                    const uint64_t bd = smem_desc(smem_u32(sXf) + 2048 * kk, 16, 1024, kSwizzle128B);
-                    mma_f16_ss(tmem + kColH, a, bd, id, 1);
-                }
-                tc_commit(bar_state);
-            }
-
-            // ---- t-blocks of 128 rows ----
-            const float rho = sCg * sigma * kappa;
-            const float inv_kappa = 1.f / kappa;
-            for (int tb = 0; tb < NTB; ++tb) {
-                const int t0 = tb * kTB;
-                const int ncols = (Q <= kTB) ? Q : (tb + 1) * kTB;
-                const int t = t0 + tid;  // this thread's row
-                // C' row t -> TMEM (64 columns of f16 pairs); rows past Q are zero
-                {
-                    const float f = (t < Q) ? __expf(acum[t]) : 0.f;
-                    uint32_t r[32];
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-#pragma unroll
-                        for (int j4 = 0; j4 < 4; ++j4) {
-                            const int j = half * 4 + j4;  // 16-byte chunk of the int8 row
-                            uint4 w = make_uint4(0, 0, 0, 0);
-                            if (t < Q) w = *reinterpret_cast<const uint4*>(sC + sw128(t, j * 16));
-                            const uint32_t ws4[4] = {w.x, w.y, w.z, w.w};
-                            float fv[16];
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) i8x4_to_f32(ws4[i], fv + 4 * i);
-#pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                r[j4 * 8 + i] = pack_f16x2(fv[2 * i] * f, fv[2 * i + 1] * f);
-                        }
-                        tmem_st32(tmem_addr(tmem, lane_base, kColC + half * 32), r);
-                    }
-                    tmem_st_wait();
-                }
-                tc_fence_before();
-                __syncthreads();
+    } else if (warp == kWarpMma) {
+        // ============================== MMA issue ==============================
+        if (lane == 0 && nb_total > 0) {
+            const uint32_t id_st = idesc_f16(kBlk, kP, true, true);
+            const uint32_t id_y = idesc_f16(kBlk, kP, false, true);
+            auto issue_cb_block = [&](int kb) {
+                const int j = kb & 1;
+                wait_phase(bars + kBarFull0 + j, (kb >> 1) & 1, abort_flag, p);
+                if (kb >= 2) wait_phase(bars + kBarAcc0 + j, ((kb >> 1) - 1) & 1, abort_flag, p);
                 tc_fence_after();
-                if (tid == 0) {
-                    issue_cb(tmem + kColCB, smem_u32(sC), smem_u32(sB), t0, ncols);
-                    tc_commit(bar_cb);
-                    const uint32_t id = idesc_f16(kTB, kP, false, true);
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_f16_ts(tmem + kColAcc, tmem + kColC + 8 * kk,
-                                   smem_desc(smem_u32(sHp) + 2048 * kk, 16, 1024, kSwizzle128B), id,
-                                   kk > 0);
-                }
-                wait_bar(bar_cb, ph_cb);
+                uint8_t* stage = smem + j * kStageBytes;
+                issue_cb(tmem + kColCB + 128u * j, smem_u32(stage + kStC), smem_u32(stage + kStB),
+                         0, kBlk);
+                tc_commit(bars + kBarCb0 + j);
+                tc_commit(bars + kBarEmpty0 + j);
+            };
+            issue_cb_block(0);
+            for (int kb = 0; kb < nb_total; ++kb) {
+                const int j = kb & 1;
+                const uint32_t xf = smem_u32(smem + kOffXf + j * 16384);
+                const uint32_t bp = smem_u32(smem + kOffBp + j * 32768);
+                const uint32_t hp = smem_u32(smem + kOffHp + j * 16384);
+                wait_phase(bars + kBarPrep0 + j, (kb >> 1) & 1, abort_flag, p);
+                if (kb >= 2) wait_phase(bars + kBarAccFree0 + j, ((kb >> 1) - 1) & 1, abort_flag, p);
                 tc_fence_after();
-                // M' over CB, in place: columns [32 sc, 32 sc + 32) -> f16 pairs at [16 sc, 16 sc + 16)
-                {
-                    const float at = (t < Q) ? acum[t] : 0.f;
-                    const bool row_ok = t < valid;
-                    for (int sc = 0; sc < ncols / 32; ++sc) {
-                        uint32_t r[32];
-                        tmem_ld32(tmem_addr(tmem, lane_base, kColCB + 32 * sc), r);
-                        tmem_ld_wait();
-                        uint32_t o[16];
+                // state: H += B'^T x   (M = 128 n, N = 64 p, K = 128 t)
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            float mv[2];
+                for (int kk = 0; kk < kBlk / 16; ++kk)
+                    mma_f16_ss(tmem + kColH,
+                               smem_desc(bp + 2048 * kk, 16384, 1024, kSwizzle128B),
+                               smem_desc(xf + 2048 * kk, 16, 1024, kSwizzle128B), id_st, 1);
+                tc_commit(bars + kBarState);
+                // acc = C' H'^T   (A = C' from TMEM, K = 128 n)
 #pragma unroll
-                            for (int e = 0; e < 2; ++e) {
-                                const int s = 32 * sc + 2 * i + e;
-                                float v = 0.f;
-                                if (row_ok && s <= t)
-                                    v = static_cast<float>(static_cast<int>(r[2 * i + e])) *
-                                        __expf(at - acum[s]) * dts[s] * inv_kappa;
-                                mv[e] = v;
-                            }
-                            o[i] = pack_f16x2(mv[0], mv[1]);
-                        }
-                        tmem_st16(tmem_addr(tmem, lane_base, kColCB + 16 * sc), o);
-                    }
-                    tmem_st_wait();
-                }
-                tc_fence_before();
-                __syncthreads();
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_f16_ts(tmem + kColAcc + 64 * j, tmem + kColC + 8 * kk,
+                               smem_desc(hp + 2048 * kk, 16, 1024, kSwizzle128B), id_y, kk > 0);
+                tc_commit(bars + kBarCh);
+                // acc += M' x   (A = M' from TMEM, K = 128 s)
+                wait_phase(bars + kBarMp0 + j, (kb >> 1) & 1, abort_flag, p);
                 tc_fence_after();
-                if (*abort_flag) break;
-                if (tid == 0) {
-                    const uint32_t id = idesc_f16(kTB, kP, false, true);
-                    for (int kk = 0; kk < ncols / 16; ++kk)
-                        mma_f16_ts(tmem + kColAcc, tmem + kColCB + 8 * kk,
-                                   smem_desc(smem_u32(sXf) + 2048 * kk, 16, 1024, kSwizzle128B), id,
-                                   1);
-                    tc_commit(bar_acc);
-                }
-                wait_bar(bar_acc, ph_acc);
-                tc_fence_after();
-                // ---- epilogue: y = rho * acc + D s_x xq ----
-                {
-                    uint32_t r[2][32];
-                    tmem_ld32(tmem_addr(tmem, lane_base, kColAcc), r[0]);
-                    tmem_ld32(tmem_addr(tmem, lane_base, kColAcc + 32), r[1]);
-                    tmem_ld_wait();
-                    if (t < valid) {
-                        const size_t ybase = (((size_t)b * p.L + t_base + t) * p.H + h) * kP;
-                        const int8_t* xr = reinterpret_cast<const int8_t*>(sX + t * 64);
-                        float out[kP];
 #pragma unroll
-                        for (int pp = 0; pp < kP; ++pp)
-                            out[pp] = rho * __uint_as_float(r[pp / 32][pp % 32]) +
-                                      Dsx * static_cast<float>(xr[pp]);
-                        if (p.y_dtype == SSD_OUT_I8) {
-                            int8_t* yo = static_cast<int8_t*>(p.y) + ybase;
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                uint32_t wv[4];
-#pragma unroll
-                                for (int i = 0; i < 4; ++i) {
-                                    uint32_t acc = 0;
-#pragma unroll
-                                    for (int e = 0; e < 4; ++e) {
-                                        float rr = rintf(out[q * 16 + i * 4 + e] * p.inv_y_scale);
-                                        rr = fminf(fmaxf(rr, -127.f), 127.f);
-                                        acc |= (static_cast<uint32_t>(static_cast<int>(rr)) & 0xffu) << (8 * e);
-                                    }
-                                    wv[i] = acc;
-                                }
-                                reinterpret_cast<uint4*>(yo)[q] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-                            }
-                        } else if (p.y_dtype == SSD_OUT_F16) {
-                            __half* yo = static_cast<__half*>(p.y) + ybase;
-#pragma unroll
-                            for (int q = 0; q < 8; ++q)
-                                reinterpret_cast<uint4*>(yo)[q] = make_uint4(
-                                    pack_f16x2(out[q * 8 + 0], out[q * 8 + 1]), pack_f16x2(out[q * 8 + 2], out[q * 8 + 3]),
-                                    pack_f16x2(out[q * 8 + 4], out[q * 8 + 5]), pack_f16x2(out[q * 8 + 6], out[q * 8 + 7]));
-                        } else {
-                            float* yo = static_cast<float*>(p.y) + ybase;
-#pragma unroll
-                            for (int q = 0; q < 16; ++q)
-                                reinterpret_cast<float4*>(yo)[q] =
-                                    make_float4(out[q * 4], out[q * 4 + 1], out[q * 4 + 2], out[q * 4 + 3]);
-                        }
-                    }
-                }
-                tc_fence_before();
-                __syncthreads();
-                tc_fence_after();
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_f16_ts(tmem + kColAcc + 64 * j, tmem + kColCB + 128u * j + 8 * kk,
+                               smem_desc(xf + 2048 * kk, 16, 1024, kSwizzle128B), id_y, 1);
+                tc_commit(bars + kBarAcc0 + j);
+                if (kb + 1 < nb_total) issue_cb_block(kb + 1);
             }
-            // the state MMA of this chunk must be done before the next boundary step reads H
-            wait_bar(bar_state, ph_state);
-            tc_fence_after();
-            __syncthreads();
-            if (*abort_flag) break;
         }
-        if (*abort_flag) break;
-
-        // ---- end of the piece: final state and / or hand-off slot ----
-        {
+        __syncwarp();
+    } else if (warp < 4) {
+        // ============================== prep warpgroup ==============================
+        const int row = tid;  // block row t / state row n (TMEM lane)
+        const uint32_t lane_base = static_cast<uint32_t>(warp) * 32u;
+        float* red = reinterpret_cast<float*>(smem + kOffRed);
+        int kb = 0;
+        // previous piece, whose state is stored once its last update is done
+        int pv_b = 0, pv_h = 0, pv_cta_end = 0;
+        bool pv_valid = false, pv_final = false;
+        float pv_out = 1.f;  // H_true / s_x s_B = pv_out * H_tmem
+        auto store_piece = [&]() {
             uint32_t hv[2][32];
             tmem_ld32(tmem_addr(tmem, lane_base, kColH), hv[0]);
             tmem_ld32(tmem_addr(tmem, lane_base, kColH + 32), hv[1]);
             tmem_ld_wait();
-            if (c_end == nch) {
-                if (p.final_state != nullptr && n < N) {
-                    float* dst = p.final_state + ((size_t)b * p.H + h) * kP * N;
+            if (pv_final) {
+                if (p.final_state != nullptr && row < p.N) {
+                    float* dst = p.final_state + ((size_t)pv_b * p.H + pv_h) * kP * p.N;
+                    const float s = pv_out * p.x_scale[pv_h] * p.B_scale[pv_h / (p.H / p.G)];
 #pragma unroll
-                    for (int pp = 0; pp < kP; ++pp)
-                        dst[(size_t)pp * N + n] = sigma * __uint_as_float(hv[pp / 32][pp % 32]);
+                    for (int j = 0; j < 64; ++j)
+                        dst[(size_t)j * p.N + row] = s * __uint_as_float(hv[j / 32][j % 32]);
                 }
-            } else {
-                float4* dst = reinterpret_cast<float4*>(p.slots + ((size_t)cta * 128 + n) * kP);
+            } else if (pv_cta_end) {
+                float4* dst = reinterpret_cast<float4*>(p.slots + ((size_t)blockIdx.x * 128 + row) * kP);
 #pragma unroll
-                for (int q = 0; q < kP / 4; ++q)
-                    dst[q] = make_float4(__uint_as_float(hv[(4 * q) / 32][(4 * q) % 32]),
-                                         __uint_as_float(hv[(4 * q + 1) / 32][(4 * q + 1) % 32]),
-                                         __uint_as_float(hv[(4 * q + 2) / 32][(4 * q + 2) % 32]),
-                                         __uint_as_float(hv[(4 * q + 3) / 32][(4 * q + 3) % 32]));
+                for (int q = 0; q < 16; ++q)
+                    dst[q] = make_float4(pv_out * __uint_as_float(hv[(4 * q) / 32][(4 * q) % 32]),
+                                         pv_out * __uint_as_float(hv[(4 * q + 1) / 32][(4 * q + 1) % 32]),
+                                         pv_out * __uint_as_float(hv[(4 * q + 2) / 32][(4 * q + 2) % 32]),
+                                         pv_out * __uint_as_float(hv[(4 * q + 3) / 32][(4 * q + 3) % 32]));
                 __threadfence();
-                __syncthreads();
-                if (tid == 0) {
-                    unsigned long long* f = p.flags + cta;
+                wg_sync(1);
+                if (row == 0) {
+                    unsigned long long* f = p.flags + blockIdx.x;
                     asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(f), "l"(p.epoch) : "memory");
                 }
             }
-            tc_fence_before();
-            __syncthreads();
-            tc_fence_after();
+        };
+        for (int k = 0; k < rg.nseg; ++k) {
+            int b, h, c_begin, c_end;
+            rg.seg(k, b, h, c_begin, c_end);
+            const int g = h / (p.H / p.G);
+            const float sx = p.x_scale[h], sBg = p.B_scale[g], sCg = p.C_scale[g];
+            const float sigma = sx * sBg;
+            const float A_h = p.A[h], D_h = p.D[h];
+            const float* dt_bh = p.dt + (size_t)b * p.L * p.H + h;
+            float U = 1.f;   // H_true / sigma = U * H_tmem
+            float hb = 0.f;  // running bound on max |H_true| / sigma
+            for (int c = c_begin; c < c_end; ++c, ++kb) {
+                const int j = kb & 1;
+                uint8_t* stage = smem + j * kStageBytes;
+                uint8_t* xf = smem + kOffXf + j * 16384;
+                uint8_t* bp = smem + kOffBp + j * 32768;
+                uint8_t* hp = smem + kOffHp + j * 16384;
+                float* colf = reinterpret_cast<float*>(smem + kOffColf) + j * 512;
+                float* dts = reinterpret_cast<float*>(smem + kOffDt) + j * 128;
+                float* acum = reinterpret_cast<float*>(smem + kOffAcum) + j * 128;
+                const int valid = min(kBlk, p.L - c * kBlk);
+                // dt of this token (in flight during the waits below)
+                const float d = row < valid ? dt_bh[(size_t)(c * kBlk + row) * p.H] : 0.f;
+                // (a) the previous block's state update is done: H, hp[j], xf[j], bp[j] free
+                if (kb >= 1) wait_phase(bars + kBarState, (kb - 1) & 1, abort_flag, p);
+                tc_fence_after();
+                // (b) piece start: store the previous piece's state, load this piece's
+                if (c == c_begin) {
+                    if (pv_valid) store_piece();
+                    const float* src = nullptr;
+                    bool from_slot = false;
+                    if (c_begin == 0) {
+                        if (p.init_state) src = p.init_state + ((size_t)b * p.H + h) * kP * p.N;
+                    } else {
+                        if (row == 0) {
+                            const unsigned long long* f = p.flags + (blockIdx.x - 1);
+                            const long long t0 = clock64();
+                            unsigned long long v;
+                            for (;;) {
+                                asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(f) : "memory");
+                                if (v == p.epoch || *abort_flag) break;
+                                if (clock64() - t0 > kWaitCycles) {
+                                    *abort_flag = 1;
+                                    report_failure(p, 2);
+                                    break;
+                                }
+                                __nanosleep(256);
+                            }
+                        }
+                        wg_sync(1);
+                        src = p.slots + (size_t)(blockIdx.x - 1) * 128 * kP;
+                        from_slot = true;
+                    }
+                    uint32_t r[2][32];
+                    float m = 0.f;
+#pragma unroll
+                    for (int jj = 0; jj < 64; ++jj) {
+                        float v = 0.f;
+                        if (src != nullptr && row < p.N)
+                            v = from_slot ? __ldcg(src + row * kP + jj) : src[(size_t)jj * p.N + row] / sigma;
+                        m = fmaxf(m, fabsf(v));
+                        r[jj / 32][jj % 32] = __float_as_uint(v);
+                    }
+                    tmem_st32(tmem_addr(tmem, lane_base, kColH), r[0]);
+                    tmem_st32(tmem_addr(tmem, lane_base, kColH + 32), r[1]);
+                    tmem_st_wait();
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                    if (lane == 0) red[16 + warp] = m;
+                    wg_sync(1);
+                    hb = fmaxf(fmaxf(red[16], red[17]), fmaxf(red[18], red[19]));
+                    U = 1.f;
+                }
+                // (c) block scan of dt * A, with the block's max dt and sum dt
+                float incl, dmax, dsum;
+                {
+                    const float a = d * A_h;
+                    float v = a, mx = d, sm = d;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const float u = __shfl_up_sync(0xffffffffu, v, o);
+                        if (lane >= o) v += u;
+                    }
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) {
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                        sm += __shfl_xor_sync(0xffffffffu, sm, o);
+                    }
+                    if (lane == 31) red[warp] = v;
+                    if (lane == 0) {
+                        red[4 + warp] = mx;
+                        red[8 + warp] = sm;
+                    }
+                    wg_sync(1);
+                    float pre = 0.f;
+                    for (int w = 0; w < warp; ++w) pre += red[w];
+                    incl = v + pre;
+                    dmax = fmaxf(fmaxf(red[4], red[5]), fmaxf(red[6], red[7]));
+                    dsum = (red[8] + red[9]) + (red[10] + red[11]);
+                    dts[row] = d;
+                    acum[row] = incl;
+                }
+                wg_sync(1);  // acum complete; red[] free again
+                const float a_end = acum[kBlk - 1];
+                // (d) scales of this block
+                float need = fmaxf(fmaxf(hb, 16129.f * static_cast<float>(p.N) * dmax),
+                                   fabsf(D_h) / (sCg * sBg)) * (1.f / kF16Range);
+                if (!(need > 1e-30f) || !isfinite(need)) need = 1.f;
+                const float rho = pow2_ceil(sCg * sigma * need);
+                const float kappa = rho / (sCg * sigma);
+                const float U_new = dmax > 0.f ? pow2_ceil(127.f * dmax * (1.f / kF16Range)) : U;
+                const float e_end = __expf(a_end);
+                // (e) state hand-over: H' = H / kappa (f16) for C'.H', then decay + rescale
+                {
+                    const float to_hp = U / kappa;
+                    const float to_h = e_end * (U / U_new);
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t hv[32];
+                        tmem_ld32(tmem_addr(tmem, lane_base, kColH + 32 * hh), hv);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint4 v;
+                            v.x = pack_f16x2(__uint_as_float(hv[8 * q + 0]) * to_hp, __uint_as_float(hv[8 * q + 1]) * to_hp);
+                            v.y = pack_f16x2(__uint_as_float(hv[8 * q + 2]) * to_hp, __uint_as_float(hv[8 * q + 3]) * to_hp);
+                            v.z = pack_f16x2(__uint_as_float(hv[8 * q + 4]) * to_hp, __uint_as_float(hv[8 * q + 5]) * to_hp);
+                            v.w = pack_f16x2(__uint_as_float(hv[8 * q + 6]) * to_hp, __uint_as_float(hv[8 * q + 7]) * to_hp);
+                            *reinterpret_cast<uint4*>(hp + sw128(row, 64 * hh + 16 * q)) = v;
+                        }
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) hv[i] = __float_as_uint(__uint_as_float(hv[i]) * to_h);
+                        tmem_st32(tmem_addr(tmem, lane_base, kColH + 32 * hh), hv);
+                    }
+                    U = U_new;
+                    hb = hb * e_end + 16129.f * dsum;  // bound after this block's update
+                }
+                // (f) conversions of the block's tiles
+                wait_phase(bars + kBarFull0 + j, (kb >> 1) & 1, abort_flag, p);
+                {
+                    // x row -> f16 (64 values)
+                    const uint4* xs = reinterpret_cast<const uint4*>(stage + kStX + row * 64);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint4 w = xs[q];
+                        uint4 o0, o1;
+                        i8x4_to_h2x2(w.x, o0.x, o0.y);
+                        i8x4_to_h2x2(w.y, o0.z, o0.w);
+                        i8x4_to_h2x2(w.z, o1.x, o1.y);
+                        i8x4_to_h2x2(w.w, o1.z, o1.w);
+                        *reinterpret_cast<uint4*>(xf + sw128(row, 32 * q)) = o0;
+                        *reinterpret_cast<uint4*>(xf + sw128(row, 32 * q + 16)) = o1;
+                    }
+                    // B row scaled by w_t / U -> B' (two MN blocks of 64 n)
+                    const float wt = row < valid ? d * __expf(a_end - incl) / U : 0.f;
+                    const __half2 w2 = __float2half2_rn(wt);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const uint4 w = *reinterpret_cast<const uint4*>(stage + kStB + sw128(row, 16 * q));
+                        uint4 o0, o1;
+                        i8x4_to_h2x2(w.x, o0.x, o0.y);
+                        i8x4_to_h2x2(w.y, o0.z, o0.w);
+                        i8x4_to_h2x2(w.z, o1.x, o1.y);
+                        i8x4_to_h2x2(w.w, o1.z, o1.w);
+                        o0.x = hmul2_u32(o0.x, w2); o0.y = hmul2_u32(o0.y, w2);
+                        o0.z = hmul2_u32(o0.z, w2); o0.w = hmul2_u32(o0.w, w2);
+                        o1.x = hmul2_u32(o1.x, w2); o1.y = hmul2_u32(o1.y, w2);
+                        o1.z = hmul2_u32(o1.z, w2); o1.w = hmul2_u32(o1.w, w2);
+                        uint8_t* blk = bp + (q / 4) * 16384;
+                        *reinterpret_cast<uint4*>(blk + sw128(row, 32 * (q % 4))) = o0;
+                        *reinterpret_cast<uint4*>(blk + sw128(row, 32 * (q % 4) + 16)) = o1;
+                    }
+                    // C row scaled by exp(Acum_t) -> C' in TMEM, once the previous C'.H' is done
+                    if (kb >= 1) wait_phase(bars + kBarCh, (kb - 1) & 1, abort_flag, p);
+                    tc_fence_after();
+                    const __half2 f2 = __float2half2_rn(__expf(incl));
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t r[32];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const uint4 w = *reinterpret_cast<const uint4*>(stage + kStC + sw128(row, 16 * (4 * hh + q)));
+                            i8x4_to_h2x2(w.x, r[8 * q + 0], r[8 * q + 1]);
+                            i8x4_to_h2x2(w.y, r[8 * q + 2], r[8 * q + 3]);
+                            i8x4_to_h2x2(w.z, r[8 * q + 4], r[8 * q + 5]);
+                            i8x4_to_h2x2(w.w, r[8 * q + 6], r[8 * q + 7]);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) r[8 * q + i] = hmul2_u32(r[8 * q + i], f2);
+                        }
+                        tmem_st32(tmem_addr(tmem, lane_base, kColC + 32 * hh), r);
+                    }
+                    // column factors exp(Acum_{32 q} - Acum_s) dt_s / kappa for s < 32 q
+                    for (int idx = row; idx < 192; idx += kBlk) {
+                        const int q = idx < 32 ? 1 : (idx < 96 ? 2 : 3);
+                        const int s = idx - (q == 1 ? 0 : (q == 2 ? 32 : 96));
+                        colf[q * 128 + s] = __expf(acum[32 * q] - acum[s]) * dts[s] / kappa;
+                    }
+                    if (row == 0) {
+                        BlockInfo bi;
+                        bi.rho = rho;
+                        bi.inv_kappa = 1.f / kappa;
+                        bi.dterm = D_h * sx / rho;
+                        bi.pad = 0.f;
+                        bi.b = b;
+                        bi.h = h;
+                        bi.c = c;
+                        bi.valid = valid;
+                        info[j] = bi;
+                    }
+                }
+                fence_proxy_async_smem();
+                tmem_st_wait();
+                tc_fence_before();
+                wg_sync(1);
+                if (row == 0) {
+                    mbar_arrive(bars + kBarEmpty0 + j);
+                    mbar_arrive(bars + kBarPrep0 + j);
+                }
+            }
+            // this piece's state is stored when the next piece starts (or below)
+            pv_valid = true;
+            pv_b = b;
+            pv_h = h;
+            pv_final = (c_end == p.nblk);
+            pv_cta_end = (c_end != p.nblk);
+            pv_out = U;
         }
+        if (pv_valid) {
+            wait_phase(bars + kBarState, (kb - 1) & 1, abort_flag, p);
+            tc_fence_after();
+            store_piece();
+        }
+    } else {
+        // ============================== M' and output warpgroup ==============================
+        const int quad = warp & 3;
+        const int row = quad * 32 + lane;
+        const uint32_t lane_base = static_cast<uint32_t>(quad) * 32u;
+        // output of the previous block
+        int pv_j = 0, pv_b = 0, pv_h = 0, pv_c = 0, pv_valid = 0;
+        float pv_rho = 1.f;
+        auto output = [&](int kb) {
+            wait_phase(bars + kBarAcc0 + pv_j, (kb >> 1) & 1, abort_flag, p);
+            tc_fence_after();
+            uint32_t r[2][32];
+            tmem_ld32(tmem_addr(tmem, lane_base, kColAcc + 64 * pv_j), r[0]);
+            tmem_ld32(tmem_addr(tmem, lane_base, kColAcc + 64 * pv_j + 32), r[1]);
+            tmem_ld_wait();
+            tc_fence_before();
+            wg_sync(2);
+            if (row == 0 + 0 && quad == 0 && lane == 0) mbar_arrive(bars + kBarAccFree0 + pv_j);
+            if (row < pv_valid) {
+                const size_t ybase = (((size_t)pv_b * p.L + (size_t)pv_c * kBlk + row) * p.H + pv_h) * kP;
+                if (p.y_dtype == SSD_OUT_I8) {
+                    const float sc = pv_rho * p.inv_y_scale;
+                    uint32_t wv[16];
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        const uint32_t* rr = &r[q / 8][(q % 8) * 4];
+                        wv[q] = q8(__uint_as_float(rr[0]) * sc) | (q8(__uint_as_float(rr[1]) * sc) << 8) |
+                                (q8(__uint_as_float(rr[2]) * sc) << 16) | (q8(__uint_as_float(rr[3]) * sc) << 24);
+                    }
+                    uint4* yo = reinterpret_cast<uint4*>(static_cast<int8_t*>(p.y) + ybase);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) yo[q] = make_uint4(wv[4 * q], wv[4 * q + 1], wv[4 * q + 2], wv[4 * q + 3]);
+                } else if (p.y_dtype == SSD_OUT_F16) {
+                    uint4* yo = reinterpret_cast<uint4*>(static_cast<__half*>(p.y) + ybase);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const uint32_t* rr = &r[q / 4][(q % 4) * 8];
+                        yo[q] = make_uint4(pack_f16x2(__uint_as_float(rr[0]) * pv_rho, __uint_as_float(rr[1]) * pv_rho),
+                                           pack_f16x2(__uint_as_float(rr[2]) * pv_rho, __uint_as_float(rr[3]) * pv_rho),
+                                           pack_f16x2(__uint_as_float(rr[4]) * pv_rho, __uint_as_float(rr[5]) * pv_rho),
+                                           pack_f16x2(__uint_as_float(rr[6]) * pv_rho, __uint_as_float(rr[7]) * pv_rho));
+                    }
+                } else {
+                    float4* yo = reinterpret_cast<float4*>(static_cast<float*>(p.y) + ybase);
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        const uint32_t* rr = &r[q / 8][(q % 8) * 4];
+                        yo[q] = make_float4(__uint_as_float(rr[0]) * pv_rho, __uint_as_float(rr[1]) * pv_rho,
+                                            __uint_as_float(rr[2]) * pv_rho, __uint_as_float(rr[3]) * pv_rho);
+                    }
+                }
+            }
+        };
+        for (int kb = 0; kb < nb_total; ++kb) {
+            const int j = kb & 1;
+            const float* colf = reinterpret_cast<const float*>(smem + kOffColf) + j * 512;
+            const float* dts = reinterpret_cast<const float*>(smem + kOffDt) + j * 128;
+            const float* acum = reinterpret_cast<const float*>(smem + kOffAcum) + j * 128;
+            const uint32_t col_cb = kColCB + 128u * j;
+            wait_phase(bars + kBarPrep0 + j, (kb >> 1) & 1, abort_flag, p);
+            const BlockInfo bi = info[j];
+            wait_phase(bars + kBarCb0 + j, (kb >> 1) & 1, abort_flag, p);
+            tc_fence_after();
+            // ---- M' in place over CB, one 32-column chunk at a time (increasing order) ----
+            {
+                const bool row_ok = row < bi.valid;
+                const float at = acum[row];
+                const float rowf = row_ok ? __expf(at - acum[32 * quad]) : 0.f;
+                for (int sc = 0; sc < 4; ++sc) {
+                    uint32_t o[16];
+                    if (sc <= quad) {
+                        uint32_t cbv[32];
+                        tmem_ld32(tmem_addr(tmem, lane_base, col_cb + 32 * sc), cbv);
+                        tmem_ld_wait();
+                        if (sc < quad) {
+                            const float* cf = colf + quad * 128 + 32 * sc;
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                const float2 f = *reinterpret_cast<const float2*>(cf + 2 * e);
+                                o[e] = pack_f16x2(i32_to_f32_small(cbv[2 * e]) * f.x * rowf,
+                                                  i32_to_f32_small(cbv[2 * e + 1]) * f.y * rowf);
+                            }
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                float mv[2];
+#pragma unroll
+                                for (int z = 0; z < 2; ++z) {
+                                    const int s = 32 * sc + 2 * e + z;
+                                    float v = 0.f;
+                                    if (row_ok && s <= row)
+                                        v = i32_to_f32_small(cbv[2 * e + z]) * __expf(at - acum[s]) *
+                                            dts[s] * bi.inv_kappa;
+                                    if (row_ok && s == row) v += bi.dterm;
+                                    mv[z] = v;
+                                }
+                                o[e] = pack_f16x2(mv[0], mv[1]);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) o[e] = 0u;
+                    }
+                    tmem_st16(tmem_addr(tmem, lane_base, col_cb + 16 * sc), o);
+                }
+                tmem_st_wait();
+            }
+            tc_fence_before();
+            wg_sync(2);
+            if (tid == 128) mbar_arrive(bars + kBarMp0 + j);
+            // ---- output of the previous block while the tensor core runs this one ----
+            if (kb >= 1) output(kb - 1);
+            pv_j = j;
+            pv_b = bi.b;
+            pv_h = bi.h;
+            pv_c = bi.c;
+            pv_valid = bi.valid;
+            pv_rho = bi.rho;
+        }
+        if (nb_total >= 1) output(nb_total - 1);
     }
 
-    // ---- teardown: nothing of ours may still be in flight when TMEM is released ----
-    if (*abort_flag) {
-        if (tid == 0) report_failure(p, 1);
-        if (tma_in_flight) mbar_wait(bar_tma, ph_tma, kWaitCycles);
-        if (tid == 0) tc_commit(bar_acc);
-        mbar_wait(bar_acc, ph_acc, kWaitCycles);
-    }
-    tc_fence_before();
+    // ---- teardown: nothing of ours may be in flight when TMEM is released ----
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+    if (warp == kWarpMma) {
+        if (lane == 0 && nb_total > 0) {
+            tc_commit(bars + kBarCh);  // completes once every MMA issued above is done
+            // the commit count of kBarCh so far is nb_total; wait for one more phase
+            mbar_wait(bars + kBarCh, nb_total & 1, kWaitCycles);
+        }
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
 }
 
-// ChunkBMM export with the same device code the fused scan uses: one CTA per
-// (chunk, group, batch), t-blocks of 128 rows, every s column of the chunk.
+// ChunkBMM export with the device code the fused scan uses (issue_cb): one CTA per
+// (chunk, group, batch), 128-row t-blocks, every s column of the chunk.
+constexpr int kCbThreads = 128;
+
 template <int Q>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kCbThreads, 1)
 chunk_cb_tc_kernel(const __grid_constant__ CUtensorMap map_B, const __grid_constant__ CUtensorMap map_C,
                    int nch, int G, int32_t* __restrict__ cb) {
-    constexpr int NTB = Q > kTB ? Q / kTB : 1;
+    constexpr int NTB = Q > kBlk ? Q / kBlk : 1;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -616,13 +786,14 @@ chunk_cb_tc_kernel(const __grid_constant__ CUtensorMap map_B, const __grid_const
     int32_t* out = cb + (((size_t)b * nch + c) * G + g) * Q * Q;
     for (int tb = 0; tb < NTB && ok; ++tb) {
         if (tid == 0) {
-            issue_cb(tmem, smem_u32(sC), smem_u32(sB), tb * kTB, Q);
+            tc_fence_after();
+            issue_cb(tmem, smem_u32(sC), smem_u32(sB), tb * kBlk, Q);
             tc_commit(bars + 1);
         }
         ok = mbar_wait(bars + 1, ph, kWaitCycles);
         ph ^= 1u;
         tc_fence_after();
-        const int t = tb * kTB + tid;
+        const int t = tb * kBlk + tid;
         for (int sc = 0; sc < Q / 32; ++sc) {
             uint32_t r[32];
             tmem_ld32(tmem_addr(tmem, warp * 32, 32 * sc), r);
@@ -662,15 +833,15 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 4-D int8 map over [batch][L][rows2][inner] with box {box0, 1, Q, 1}.
+// 4-D int8 map over [batch][L][rows2][inner] with box {box0, 1, rows, 1}.
 bool make_map(CUtensorMap* m, const void* base, int inner, int rows2, int L, int batch, int box0,
-              int Q, CUtensorMapSwizzle sw) {
+              int rows, CUtensorMapSwizzle sw) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[4] = {(cuuint64_t)inner, (cuuint64_t)rows2, (cuuint64_t)L, (cuuint64_t)batch};
     cuuint64_t strides[3] = {(cuuint64_t)inner, (cuuint64_t)inner * rows2,
                              (cuuint64_t)inner * rows2 * L};
-    cuuint32_t box[4] = {(cuuint32_t)box0, 1, (cuuint32_t)Q, 1};
+    cuuint32_t box[4] = {(cuuint32_t)box0, 1, (cuuint32_t)rows, 1};
     cuuint32_t es[4] = {1, 1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, es,
               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -693,39 +864,6 @@ int num_sms() {
 }
 
 template <int Q>
-cudaError_t launch_fused_q(const ChunkScanArgs& a, cudaStream_t st) {
-    CUtensorMap mx, mB, mC;
-    if (!make_map(&mx, a.x, kP, a.nheads, a.seqlen, a.batch, kP, Q, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map(&mB, a.B, a.dstate, a.ngroups, a.seqlen, a.batch, 128, Q, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mC, a.C, a.dstate, a.ngroups, a.seqlen, a.batch, 128, Q, CU_TENSOR_MAP_SWIZZLE_128B))
-        return cudaErrorInvalidValue;
-    FusedParams p{};
-    p.dt = a.dt; p.A = a.A; p.D = a.D; p.x_scale = a.x_scale; p.B_scale = a.B_scale;
-    p.C_scale = a.C_scale; p.init_state = a.init_state; p.final_state = a.final_state;
-    p.y = a.y; p.y_dtype = a.y_dtype; p.inv_y_scale = a.inv_y_scale;
-    p.batch = a.batch; p.L = a.seqlen; p.H = a.nheads; p.G = a.ngroups; p.N = a.dstate;
-    p.nch = ceil_div(a.seqlen, Q);
-    p.total = (long long)a.batch * a.nheads * p.nch;
-    int sms = num_sms();
-    if (sms <= 0) return cudaErrorInvalidDevice;
-    long long nctas = std::min<long long>(std::min(sms, kMaxCtas), p.total);
-    p.nctas = static_cast<int>(nctas);
-    uint8_t* ws = static_cast<uint8_t*>(a.workspace);
-    p.status = reinterpret_cast<unsigned long long*>(ws);
-    p.flags = reinterpret_cast<unsigned long long*>(ws + 256);
-    p.slots = reinterpret_cast<float*>(ws + 256 + kMaxCtas * 8);
-    p.epoch = ++epoch_counter();
-    // at least 120 KB of shared memory per CTA keeps it alone on its SM: the kernel takes all of
-    // the SM's tensor memory and CTAs wait on their predecessor's hand-off
-    const int smem = std::max(Layout<Q>::kAlloc, 120 * 1024);
-    cudaError_t e = cudaFuncSetAttribute(fused_chunk_scan_kernel<Q>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    fused_chunk_scan_kernel<Q><<<p.nctas, kThreads, smem, st>>>(mx, mB, mC, p);
-    return cudaGetLastError();
-}
-
-template <int Q>
 cudaError_t launch_cb_q(const int8_t* C, const int8_t* B, int batch, int seqlen, int G, int N,
                         int32_t* cb, cudaStream_t st) {
     CUtensorMap mB, mC;
@@ -738,8 +876,12 @@ cudaError_t launch_cb_q(const int8_t* C, const int8_t* B, int batch, int seqlen,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     dim3 grid(nch, G, batch);
-    chunk_cb_tc_kernel<Q><<<grid, kThreads, smem, st>>>(mB, mC, nch, G, cb);
+    chunk_cb_tc_kernel<Q><<<grid, kCbThreads, smem, st>>>(mB, mC, nch, G, cb);
     return cudaGetLastError();
+}
+
+long long total_blocks(int batch, int seqlen, int nheads) {
+    return (long long)batch * nheads * ceil_div(seqlen, kBlk);
 }
 
 }  // namespace
@@ -748,18 +890,37 @@ size_t chunk_scan_workspace_bytes(int batch, int seqlen, int nheads, int headdim
                                   int chunk_size) {
     (void)headdim;
     (void)dstate;
-    const long long total = (long long)batch * nheads * ceil_div(seqlen, chunk_size);
-    const long long slots = std::min<long long>(total, kMaxCtas);
+    (void)chunk_size;
+    const long long slots = std::min<long long>(total_blocks(batch, seqlen, nheads), kMaxCtas);
     return 256 + kMaxCtas * 8 + (size_t)slots * 128 * kP * 4;
 }
 
 cudaError_t launch_chunk_scan(const ChunkScanArgs& a, cudaStream_t st) {
-    switch (a.chunk_size) {
-        case 64: return launch_fused_q<64>(a, st);
-        case 128: return launch_fused_q<128>(a, st);
-        case 256: return launch_fused_q<256>(a, st);
-        default: return cudaErrorInvalidValue;
-    }
+    CUtensorMap mx, mB, mC;
+    if (!make_map(&mx, a.x, kP, a.nheads, a.seqlen, a.batch, kP, kBlk, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map(&mB, a.B, a.dstate, a.ngroups, a.seqlen, a.batch, 128, kBlk, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mC, a.C, a.dstate, a.ngroups, a.seqlen, a.batch, 128, kBlk, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    FusedParams p{};
+    p.dt = a.dt; p.A = a.A; p.D = a.D; p.x_scale = a.x_scale; p.B_scale = a.B_scale;
+    p.C_scale = a.C_scale; p.init_state = a.init_state; p.final_state = a.final_state;
+    p.y = a.y; p.y_dtype = a.y_dtype; p.inv_y_scale = a.inv_y_scale;
+    p.batch = a.batch; p.L = a.seqlen; p.H = a.nheads; p.G = a.ngroups; p.N = a.dstate;
+    p.nblk = ceil_div(a.seqlen, kBlk);
+    p.total = total_blocks(a.batch, a.seqlen, a.nheads);
+    const int sms = num_sms();
+    if (sms <= 0) return cudaErrorInvalidDevice;
+    p.nctas = static_cast<int>(std::min<long long>(std::min(sms, kMaxCtas), p.total));
+    uint8_t* ws = static_cast<uint8_t*>(a.workspace);
+    p.status = reinterpret_cast<unsigned long long*>(ws);
+    p.flags = reinterpret_cast<unsigned long long*>(ws + 256);
+    p.slots = reinterpret_cast<float*>(ws + 256 + kMaxCtas * 8);
+    p.epoch = ++epoch_counter();
+    cudaError_t e = cudaFuncSetAttribute(fused_chunk_scan_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    fused_chunk_scan_kernel<<<p.nctas, kThreads, kSmemBytes, st>>>(mx, mB, mC, p);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_chunk_cb(const int8_t* C, const int8_t* B, int batch, int seqlen, int G,
