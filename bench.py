@@ -29,6 +29,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 from quantized_mamba_ssd_b200 import workloads as W  # noqa: E402
+from quantized_mamba_ssd_b200.dist_util import aggregate_tokens_per_s, max_over_ranks, rank_seed  # noqa: E402
 
 PREFILL_CFG = 3
 METRIC = "SSD scan tokens/s (int8 in) at 1 B200; achieved fraction of HBM/int8 roofline"
@@ -212,6 +213,9 @@ def main():
                     help="timed passes of the 512-step decode run (0 skips the decode report)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) leg")
+    ap.add_argument("--decode-batch", type=int, default=None,
+                    help="decode batch per rank (default: the workload's 128); smaller batches "
+                         "of the same shape serve profiling captures")
     ap.add_argument("--batch", type=int, default=None,
                     help="sequences per rank (default: the workload's batch of 2); a smaller "
                          "batch of the same shape serves profiling captures")
@@ -246,7 +250,7 @@ def main():
 
     # ---- prefill workload: this rank's own batch (seeded per rank) ----
     overrides = {} if args.batch is None else {"batch": args.batch}
-    case = W.make_prefill_config(PREFILL_CFG, seed=1000 + PREFILL_CFG + 97 * rank, **overrides)
+    case = W.make_prefill_config(PREFILL_CFG, seed=rank_seed(1000 + PREFILL_CFG, rank), **overrides)
     x, B, C = (torch.from_numpy(a).to(dev) for a in (case.x, case.B, case.C))
     dt = torch.from_numpy(case.dt).to(dev)
     A, Dp, sx, sb, sc = (torch.from_numpy(a).to(dev) for a in
@@ -285,12 +289,9 @@ def main():
         torch.cuda.synchronize()
     barrier()
     ms = ev0.elapsed_time(ev1) / args.steps
-    t = torch.tensor([ms], device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, dev)
     tokens_all = bsz * L * world
-    value = tokens_all / (ms_max * 1e-3)
+    value = aggregate_tokens_per_s(bsz * L, world, ms_max)
 
     # ---- end to end: pinned host inputs in, int8 output back, every step ----
     hx, hB, hC, hdt = (torch.from_numpy(a).pin_memory() for a in (case.x, case.B, case.C, case.dt))
@@ -319,10 +320,8 @@ def main():
         ev1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        t = torch.tensor([ev0.elapsed_time(ev1) / e2e_steps], device=dev)
-        if world > 1:
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e = {"value": tokens_all / (float(t.item()) * 1e-3), "unit": UNIT,
+        e2e_ms = max_over_ranks(ev0.elapsed_time(ev1) / e2e_steps, dev)
+        e2e = {"value": aggregate_tokens_per_s(bsz * L, world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     # ---- roofline of the timed call ----
@@ -344,7 +343,8 @@ def main():
     # ---- decode state update, 512 steps of batch 128 (CUDA graph replay) ----
     decode = None
     if args.decode_passes > 0:
-        d = W.make_decode_config(seed=1004 + 97 * rank)
+        dover = {} if args.decode_batch is None else {"batch": args.decode_batch}
+        d = W.make_decode_config(seed=rank_seed(1004, rank), **dover)
         st = torch.from_numpy(d.state).to(dev)
         dx, dB, dC, ddt = (torch.from_numpy(a).to(dev) for a in (d.x, d.B, d.C, d.dt))
         dA, dD, dsx, dsb, dsc = (torch.from_numpy(a).to(dev) for a in
@@ -375,10 +375,7 @@ def main():
         ev1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        t = torch.tensor([ev0.elapsed_time(ev1) / args.decode_passes], device=dev)
-        if world > 1:
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        dms = float(t.item())
+        dms = max_over_ranks(ev0.elapsed_time(ev1) / args.decode_passes, dev)
         dbytes = decode_alg_bytes(d, 2) * d.steps
         dgbs = dbytes / (dms * 1e-3) / 1e9
         decode = {

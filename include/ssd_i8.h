@@ -105,6 +105,16 @@ SSD_API ssd_status ssd_i8_chunk_scan(const int8_t *x, const int8_t *B, const int
 SSD_API ssd_status ssd_i8_chunk_scan_status(const void *workspace, void *stream);
 
 /*
+ * Test hook for failure detection (not for production use).  Arms a one-shot fault for the next
+ * ssd_i8_chunk_scan launch in this process: the CTA with index `drop_publish_cta` skips publishing
+ * its state hand-off (so its successor's bounded wait runs out), and every device-side wait of
+ * that launch is bounded by `wait_cycles` SM clocks (<= 0 keeps the default of about one second).
+ * The launch still terminates; ssd_i8_chunk_scan_status then reports SSD_ERR_TIMEOUT and later
+ * calls run normally.  drop_publish_cta = -1 only shortens the waits.
+ */
+SSD_API ssd_status ssd_i8_debug_inject(int drop_publish_cta, long long wait_cycles);
+
+/*
  * Allocation-free variant of ssd_i8_chunk_scan.  The pages have no counterpart: this entry point
  * exists for callers that cannot allocate device memory when they run the scan -- code working
  * inside a memory pool reserved in full up front, code that must not risk the device

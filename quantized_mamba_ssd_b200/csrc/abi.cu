@@ -135,6 +135,12 @@ ssd_status ssd_i8_chunk_cb(const int8_t* C, const int8_t* B, int batch, int seql
                : SSD_ERR_CUDA;
 }
 
+ssd_status ssd_i8_debug_inject(int drop_publish_cta, long long wait_cycles) {
+    if (drop_publish_cta < -1) return SSD_ERR_INVALID_ARG;
+    ssd::arm_fault_injection(drop_publish_cta, wait_cycles);
+    return SSD_OK;
+}
+
 ssd_status ssd_i8_chunk_scan_status(const void* workspace, void* stream) {
     if (!workspace) return SSD_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);

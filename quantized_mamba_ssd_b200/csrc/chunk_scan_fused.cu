@@ -114,6 +114,8 @@ struct FusedParams {
     unsigned long long* flags;   // [nctas] epoch of the published slot
     unsigned long long* status;  // [3]: epoch and code of a device-side failure, last epoch
     unsigned long long epoch;
+    long long wait_limit;        // bound of every device-side wait, SM clocks
+    int drop_publish;            // test hook: this CTA never publishes its hand-off (-1: none)
 };
 
 // the pieces of this CTA's range, in processing order (last piece first, first piece last)
@@ -209,7 +211,7 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity,
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
         if (*abort_flag) return false;
-        if (clock64() - t0 > kWaitCycles) {
+        if (clock64() - t0 > p.wait_limit) {
             *abort_flag = 1;
             report_failure(p, 1);
             return false;
@@ -262,6 +264,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
     Range rg;
     rg.init(p);
     const int nb_total = static_cast<int>(rg.we - rg.ws);
+    int n_ch = 0;  // kBarCh commits issued by the MMA thread (for the final drain)
 
     if (warp == kWarpTma) {
         // ============================== TMA producer ==============================
@@ -270,13 +273,14 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             tma_prefetch_map(&map_B);
             tma_prefetch_map(&map_C);
             int kb = 0;
-            for (int k = 0; k < rg.nseg; ++k) {
+            for (int k = 0; k < rg.nseg && !*abort_flag; ++k) {
                 int b, h, cb, ce;
                 rg.seg(k, b, h, cb, ce);
                 const int g = h / (p.H / p.G);
                 for (int c = cb; c < ce; ++c, ++kb) {
                     const int s = kb & 1;
                     if (kb >= 2) wait_phase(bars + kBarEmpty0 + s, ((kb >> 1) - 1) & 1, abort_flag, p);
+                    if (*abort_flag) break;  // after a failure no new load is started
                     uint8_t* stage = smem + s * kStageBytes;
                     uint64_t* bar = bars + kBarFull0 + s;
                     mbar_arrive_expect_tx(bar, kStageBytes);
@@ -286,7 +290,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 }
             }
             // drain: both stages' last loads must have landed before the CTA exits
-            for (int kb2 = nb_total > 2 ? nb_total - 2 : 0; kb2 < nb_total; ++kb2)
+            for (int kb2 = kb > 2 ? kb - 2 : 0; kb2 < kb; ++kb2)
                 mbar_wait(bars + kBarFull0 + (kb2 & 1), (kb2 >> 1) & 1, kWaitCycles);
         }
     } else if (warp == kWarpMma) {
@@ -306,7 +310,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 tc_commit(bars + kBarEmpty0 + j);
             };
             issue_cb_block(0);
-            for (int kb = 0; kb < nb_total; ++kb) {
+            for (int kb = 0; kb < nb_total && !*abort_flag; ++kb) {  // no new MMA after a failure
                 const int j = kb & 1;
                 const uint32_t xf = smem_u32(smem + kOffXf + j * 16384);
                 const uint32_t bp = smem_u32(smem + kOffBp + j * 32768);
@@ -327,6 +331,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                     mma_f16_ts(tmem + kColAcc + 64 * j, tmem + kColC + 8 * kk,
                                smem_desc(hp + 2048 * kk, 16, 1024, kSwizzle128B), id_y, kk > 0);
                 tc_commit(bars + kBarCh);
+                ++n_ch;
                 // acc += M' x   (A = M' from TMEM, K = 128 s)
                 wait_phase(bars + kBarMp0 + j, (kb >> 1) & 1, abort_flag, p);
                 tc_fence_after();
@@ -372,7 +377,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                                          pv_out * __uint_as_float(hv[(4 * q + 3) / 32][(4 * q + 3) % 32]));
                 __threadfence();
                 wg_sync(1);
-                if (row == 0) {
+                if (row == 0 && p.drop_publish != static_cast<int>(blockIdx.x)) {
                     unsigned long long* f = p.flags + blockIdx.x;
                     asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(f), "l"(p.epoch) : "memory");
                 }
@@ -418,7 +423,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                             for (;;) {
                                 asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(f) : "memory");
                                 if (v == p.epoch || *abort_flag) break;
-                                if (clock64() - t0 > kWaitCycles) {
+                                if (clock64() - t0 > p.wait_limit) {
                                     *abort_flag = 1;
                                     report_failure(p, 2);
                                     break;
@@ -735,9 +740,10 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
     __syncthreads();
     if (warp == kWarpMma) {
         if (lane == 0 && nb_total > 0) {
-            tc_commit(bars + kBarCh);  // completes once every MMA issued above is done
-            // the commit count of kBarCh so far is nb_total; wait for one more phase
-            mbar_wait(bars + kBarCh, nb_total & 1, kWaitCycles);
+            // every warp is past its waits: one more commit on kBarCh completes its phase n_ch
+            // once all MMAs issued above are done
+            tc_commit(bars + kBarCh);
+            mbar_wait(bars + kBarCh, n_ch & 1, kWaitCycles);
         }
         __syncwarp();
         tc_fence_after();
@@ -880,6 +886,13 @@ cudaError_t launch_cb_q(const int8_t* C, const int8_t* B, int batch, int seqlen,
     return cudaGetLastError();
 }
 
+// test hook (ssd_i8_debug_inject): the next launch gets a short wait bound and one CTA that
+// never publishes its hand-off, so that a waiting CTA gives up and reports it
+std::mutex g_inject_mutex;
+bool g_inject_armed = false;
+int g_inject_cta = -1;
+long long g_inject_wait = kWaitCycles;
+
 long long total_blocks(int batch, int seqlen, int nheads) {
     return (long long)batch * nheads * ceil_div(seqlen, kBlk);
 }
@@ -916,11 +929,28 @@ cudaError_t launch_chunk_scan(const ChunkScanArgs& a, cudaStream_t st) {
     p.flags = reinterpret_cast<unsigned long long*>(ws + 256);
     p.slots = reinterpret_cast<float*>(ws + 256 + kMaxCtas * 8);
     p.epoch = ++epoch_counter();
+    p.wait_limit = kWaitCycles;
+    p.drop_publish = -1;
+    {
+        std::lock_guard<std::mutex> lock(g_inject_mutex);
+        if (g_inject_armed) {  // one-shot fault injection for the failure-detection test
+            p.wait_limit = g_inject_wait;
+            p.drop_publish = g_inject_cta;
+            g_inject_armed = false;
+        }
+    }
     cudaError_t e = cudaFuncSetAttribute(fused_chunk_scan_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     fused_chunk_scan_kernel<<<p.nctas, kThreads, kSmemBytes, st>>>(mx, mB, mC, p);
     return cudaGetLastError();
+}
+
+void arm_fault_injection(int drop_publish_cta, long long wait_cycles) {
+    std::lock_guard<std::mutex> lock(g_inject_mutex);
+    g_inject_armed = true;
+    g_inject_cta = drop_publish_cta;
+    g_inject_wait = wait_cycles > 0 ? wait_cycles : kWaitCycles;
 }
 
 cudaError_t launch_chunk_cb(const int8_t* C, const int8_t* B, int batch, int seqlen, int G,

@@ -49,5 +49,6 @@ cudaError_t launch_chunk_scan(const ChunkScanArgs& a, cudaStream_t stream);
 cudaError_t launch_chunk_cb(const int8_t* C, const int8_t* B, int batch, int seqlen, int ngroups,
                             int dstate, int chunk_size, int32_t* cb, cudaStream_t stream);
 cudaError_t launch_state_update(const StateUpdateArgs& a, cudaStream_t stream);
+void arm_fault_injection(int drop_publish_cta, long long wait_cycles);
 
 }  // namespace ssd

@@ -25,7 +25,7 @@ OUT_DTYPES = {"f32": (0, torch.float32), "f16": (1, torch.float16), "i8": (2, to
 # names of every extern "C" symbol include/ssd_i8.h declares
 EXPORTED = ("ssd_i8_abi_version", "ssd_status_string", "ssd_i8_chunk_scan_workspace_size",
             "ssd_i8_chunk_scan", "ssd_i8_state_update", "ssd_i8_chunk_cb",
-            "ssd_i8_chunk_scan_noalloc", "ssd_i8_chunk_scan_status")
+            "ssd_i8_chunk_scan_noalloc", "ssd_i8_chunk_scan_status", "ssd_i8_debug_inject")
 
 # built-in scratch of ssd_i8_chunk_scan_noalloc (bytes); larger problems are refused
 NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -70,6 +70,8 @@ def library() -> ctypes.CDLL:
         lib.ssd_i8_state_update.argtypes = [vp] * 10 + [ci] * 5 + [vp, ci, cf, vp]
         lib.ssd_i8_chunk_cb.restype = ci
         lib.ssd_i8_chunk_cb.argtypes = [vp, vp] + [ci] * 5 + [vp, vp]
+        lib.ssd_i8_debug_inject.restype = ci
+        lib.ssd_i8_debug_inject.argtypes = [ci, ctypes.c_longlong]
         lib.ssd_i8_chunk_scan_status.restype = ci
         lib.ssd_i8_chunk_scan_status.argtypes = [vp, vp]
         lib.ssd_i8_chunk_scan_noalloc.restype = ci
@@ -212,6 +214,11 @@ def ssd_i8_chunk_cb(C: torch.Tensor, B: torch.Tensor, chunk_size: int, *,
     ]
     _check("ssd_i8_chunk_cb", library().ssd_i8_chunk_cb(*args))
     return cb
+
+
+def ssd_i8_debug_inject(drop_publish_cta: int, wait_cycles: int) -> None:
+    """Test hook: arm a one-shot hand-off fault for the next chunk scan (see include/ssd_i8.h)."""
+    _check("ssd_i8_debug_inject", library().ssd_i8_debug_inject(int(drop_publish_cta), int(wait_cycles)))
 
 
 def ssd_i8_chunk_scan_status(workspace: torch.Tensor, stream=None) -> None:
