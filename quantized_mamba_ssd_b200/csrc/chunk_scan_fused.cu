@@ -12,24 +12,26 @@
 // The chunked scan is evaluated in blocks of 128 tokens (SSDi8 page: ChunkState, state path,
 // ChunkScan, ChunkBMM of Table 5; X_scaled of Figure 3(a)).  This is the same recurrence for
 // any chunk length, so the result depends on the caller's chunk size only through rounding.
-// Per block and head, with Acum_t = sum_{k<=t} dt_k A_h inside the block:
+// Per block and head, with a_t = log2(e) * sum_{k<=t} dt_k A_h inside the block:
 //   CB    = Cq Bq^T                                   tcgen05 kind::i8, exact int32 in TMEM
-//   M'    = CB * exp(Acum_t - Acum_s) * dt_s / kappa   (s <= t), plus D s_x / rho on the
-//           diagonal; f16, written over CB in TMEM
-//   acc   = C' H'^T + M' x                             tcgen05 kind::f16, A from TMEM
-//           C'[t,n] = Cq[t,n] exp(Acum_t),  H' = (H / s_x s_B) / kappa
+//   M'    = CB * 2^(a_t - a_s) * dt_s / kappa  (s <= t), f16, written over CB in TMEM; off the
+//           32 x 32 diagonal sub-blocks as a product of a row and a column factor (both <= 1)
+//   acc   = C' H'^T + x (D s_x / rho) + M' x          tcgen05 kind::f16
+//           C'[t,n] = Cq[t,n] 2^a_t,  H' = (H / s_x s_B) / kappa
 //   y     = rho * acc,  rho = s_C s_x s_B kappa (a power of two)
-//   H    <- exp(Acum_end) H + B'^T x,  B'[t,n] = Bq[t,n] dt_t exp(Acum_end - Acum_t) / U
+//   H    <- 2^a_end H + B'^T x,  B'[t,n] = Bq[t,n] dt_t 2^(a_end - a_t) / U
 // H lives in TMEM in units of s_x s_B U, U a per-block power of two that keeps B' inside f16
 // range; kappa comes from a running bound on |H| so that no reduction over the state is
-// needed.  Only the non-int8 operands (M', C', B', H') are rounded, once each, to f16.
+// needed.  Only the non-int8 operands (M', C', B', H', D s_x / rho) are rounded, once each,
+// to f16.
 //
 // Warp roles, coupled only through mbarriers (buffers alternate with the block parity j):
-//   warp 8      TMA: x, B, C tiles of block k into stage j            (waits: stage free)
-//   warp 9      MMA issue: CB(k); state(k), C'H(k); M'x(k)            (waits: tiles, operands)
-//   warps 0-3   prep: block scan of dt*A, state hand-over (H', decay), x / B' / C' conversions,
-//               piece start / end (initial state, hand-off slot, final state)
-//   warps 4-7   M' from CB(k); output of block k-1 while the tensor core runs block k
+//   warp 8      TMA: x, B, C tiles of block k into stage j
+//   warp 9      MMA issue: state(k); C'H'(k) + x D(k); CB(k+1); M'x(k)
+//   warps 0-3   prep: block scan of dt*A, block factors, B' and C' conversions (before the
+//               state of the previous block is needed), then the state hand-over (H', decay)
+//               and piece start / end (initial state, hand-off slot, final state)
+//   warps 4-7   x -> f16, M' from CB(k), output of block k-1 while the tensor core runs block k
 // Every wait is bounded; a timeout sets a status word and turns the remaining waits into
 // no-ops so that the kernel still ends (its outputs are then undefined).
 #include <algorithm>
@@ -53,6 +55,9 @@ constexpr int kBlk = 128;       // tokens per block (MMA M)
 constexpr long long kWaitCycles = 1ll << 31;  // bound of every device-side wait (~1 s)
 constexpr int kMaxCtas = 256;   // workspace slots
 constexpr float kF16Range = 16384.f;  // target magnitude of the f16 operands (2^14)
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRound = 12582912.f;      // 1.5 * 2^23: adding it rounds to an integer
+constexpr uint32_t kRoundBits = 0x4B400000u;  // bit pattern of kRound
 
 // tensor memory columns (512 allocated)
 constexpr uint32_t kColCB = 0;     // 2 x 128: CB int32 per buffer; M' f16 pairs over cols 0..63
@@ -64,36 +69,41 @@ constexpr uint32_t kTmemCols = 512;
 // shared memory (offsets from a 1024-byte aligned base)
 constexpr int kStageBytes = 40960;  // C [128][128 B], B [128][128 B] (128B swizzle), X [128][64 B]
 constexpr int kStC = 0, kStB = 16384, kStX = 32768;
-constexpr int kOffXf = 2 * kStageBytes;         // x f16 [128 t][64 p] MN-major, 2 buffers
+constexpr int kOffXf = 2 * kStageBytes;         // x f16 [128 t][64 p], 128B swizzle, 2 buffers
 constexpr int kOffBp = kOffXf + 2 * 16384;      // B' f16 2 x [128 t][64 n] MN-major, 2 buffers
 constexpr int kOffHp = kOffBp + 2 * 32768;      // H' f16 [128 n][64 p] MN-major, 2 buffers
-constexpr int kOffColf = kOffHp + 2 * 16384;    // column factors [2][4][128] f32
-constexpr int kOffDt = kOffColf + 2 * 2048;     // dt [2][128]
-constexpr int kOffAcum = kOffDt + 2 * 512;      // Acum [2][128]
-constexpr int kOffInfo = kOffAcum + 2 * 512;    // per-block info [2]
-constexpr int kOffRed = kOffInfo + 2 * 64;      // prep scratch [32] f32
-constexpr int kOffBar = kOffRed + 128;          // mbarriers [16]
-constexpr int kOffMisc = kOffBar + 16 * 8;      // TMEM base, abort flag
+constexpr int kOffDm = kOffHp + 2 * 16384;      // D s_x / rho on the diagonal of [64][64] f16
+constexpr int kOffColf = kOffDm + 8192;         // off-diagonal column factors [2][192] f32
+constexpr int kOffNb = kOffColf + 2 * 768;      // -beta_s = log2(dt_s / kappa) - a_s [2][128]
+constexpr int kOffA2 = kOffNb + 2 * 512;        // a_t [2][128]
+constexpr int kOffInfo = kOffA2 + 2 * 512;      // per-block info [2]
+constexpr int kOffRed = kOffInfo + 2 * 32;      // prep scratch [32] f32
+constexpr int kOffBar = kOffRed + 128;          // mbarriers [24]
+constexpr int kOffMisc = kOffBar + 24 * 8;      // TMEM base, abort flag
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
-static_assert(kOffXf % 1024 == 0 && kOffBp % 1024 == 0 && kOffHp % 1024 == 0, "alignment");
+static_assert(kOffXf % 1024 == 0 && kOffBp % 1024 == 0 && kOffHp % 1024 == 0 &&
+                  kOffDm % 1024 == 0, "alignment");
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 enum {
     kBarFull0 = 0, kBarFull1,      // tiles of stage j landed (TMA transaction count)
-    kBarEmpty0, kBarEmpty1,        // stage j consumed: prep arrival + ChunkBMM commit
+    kBarEmpty0, kBarEmpty1,        // stage j consumed: prep + x conversion + ChunkBMM commit
     kBarCb0, kBarCb1,              // CB(k) in TMEM buffer j
-    kBarPrep0, kBarPrep1,          // operands of block k ready (prep warpgroup)
+    kBarPa0, kBarPa1,              // block tables, B', C', D of block k ready (prep)
+    kBarPb0, kBarPb1,              // H' written and H decayed for block k (prep)
+    kBarXf0, kBarXf1,              // x f16 of block k ready
     kBarMp0, kBarMp1,              // M'(k) in TMEM buffer j
     kBarAcc0, kBarAcc1,            // accumulator j complete (M'x(k) done)
     kBarAccFree0, kBarAccFree1,    // accumulator j read out
     kBarState,                     // state update of the last issued block done
-    kBarCh,                        // C'.H' of the last issued block done (C' columns free)
+    kBarCh,                        // C'H' + xD of the last issued block done (C', D free)
     kNumBars
 };
+static_assert(kNumBars <= 24, "barrier space");
 
 struct BlockInfo {  // handed from the prep warpgroup to the M' / output warpgroup
-    float rho, inv_kappa, dterm, pad;
-    int b, h, c, valid;
+    float rho, inv_kappa;
+    int b, h, c, valid, pad0, pad1;
 };
 
 struct FusedParams {
@@ -106,7 +116,6 @@ struct FusedParams {
     const float* init_state;
     float* final_state;
     void* y;
-    int y_dtype;
     float inv_y_scale;
     int batch, L, H, G, N, nblk, nctas;
     long long total;             // batch * H * nblk
@@ -141,6 +150,45 @@ struct Range {
     }
 };
 
+// ---------------------------------------------------------------------------------------
+// arithmetic helpers
+// ---------------------------------------------------------------------------------------
+struct f2 {
+    float x, y;
+};
+
+// packed fp32 pairs (one instruction for two lanes of work on sm_100)
+__device__ __forceinline__ f2 fmul2(f2 a, f2 b) {
+    f2 r;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+
+__device__ __forceinline__ f2 fadd2(f2 a, f2 b) {
+    f2 r;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+
+// hardware base-2 exponential and logarithm (MUFU; subnormal results flush to zero)
+__device__ __forceinline__ float ex2f(float v) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
+    return r;
+}
+
+__device__ __forceinline__ float lg2f(float v) {
+    float r;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
+    return r;
+}
+
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
     const __half2 h = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<const uint32_t*>(&h);
@@ -165,15 +213,18 @@ __device__ __forceinline__ void i8x4_to_h2x2(uint32_t w, uint32_t& lo, uint32_t&
     hi = *reinterpret_cast<uint32_t*>(&hb);
 }
 
-// exact int32 -> float for |v| < 2^22 (ChunkBMM entries: |CB| <= 127^2 * 128)
-__device__ __forceinline__ float i32_to_f32_small(uint32_t v) {
-    return __int_as_float(static_cast<int>(v) + 0x4B400000) - 12582912.0f;
+// two ChunkBMM entries (int32, |v| < 2^22) -> exact fp32 pair
+__device__ __forceinline__ f2 cb_pair(uint32_t v0, uint32_t v1) {
+    const f2 biased = {__uint_as_float(v0 + kRoundBits), __uint_as_float(v1 + kRoundBits)};
+    return fadd2(biased, f2{-kRound, -kRound});
 }
 
-// fp32 -> int8 code: round half to even, clamp to [-127, 127]
-__device__ __forceinline__ uint32_t q8(float v) {
-    v = fminf(fmaxf(v, -127.f), 127.f);
-    return __float_as_uint(v + 12582912.0f) & 0xffu;
+// bit pattern of kRound + q (q an integer after the rounding add) clamped to q in [-127, 127];
+// its low byte is then the int8 code
+__device__ __forceinline__ uint32_t clamp_code(float biased) {
+    int v = static_cast<int>(__float_as_uint(biased));
+    v = min(max(v, static_cast<int>(kRoundBits) - 127), static_cast<int>(kRoundBits) + 127);
+    return static_cast<uint32_t>(v);
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
@@ -191,11 +242,11 @@ __device__ __forceinline__ void wg_sync(int id) {
     asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
 }
 
-// smallest power of two >= v (v > 0, finite)
+// smallest power of two >= v (v > 0); exact for normal and subnormal v
 __device__ __forceinline__ float pow2_ceil(float v) {
-    int e;
-    const float m = frexpf(v, &e);  // v = m * 2^e, m in [0.5, 1)
-    return ldexpf(1.f, m == 0.5f ? e - 1 : e);
+    const uint32_t b = __float_as_uint(v);
+    if ((b & 0x007FFFFFu) == 0u && b >= 0x00800000u) return v;
+    return __uint_as_float((b & 0x7F800000u) + 0x00800000u);
 }
 
 __device__ void report_failure(const FusedParams& p, unsigned long long code) {
@@ -223,14 +274,16 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity,
 // ChunkBMM MMAs: D[tmem] = C rows [t0, t0+128) x B rows [0, ncols), K = 128 (int8).
 __device__ __forceinline__ void issue_cb(uint32_t d, uint32_t sC, uint32_t sB, int t0, int ncols) {
     const uint32_t id = idesc_i8(kBlk, ncols, false, false);
+    const uint64_t a0 = smem_desc(sC + t0 * 128, 16, 1024, kSwizzle128B);
+    const uint64_t b0 = smem_desc(sB, 16, 1024, kSwizzle128B);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const uint64_t a = smem_desc(sC + t0 * 128 + 32 * k, 16, 1024, kSwizzle128B);
-        const uint64_t b = smem_desc(sB + 32 * k, 16, 1024, kSwizzle128B);
-        mma_i8_ss(d, a, b, id, k > 0);
-    }
+    for (int k = 0; k < 4; ++k) mma_i8_ss(d, a0 + 2 * k, b0 + 2 * k, id, k > 0);
 }
 
+// start column of quad q's off-diagonal column factors (q = 1, 2, 3 hold 32 q entries)
+__host__ __device__ constexpr int colf_off(int q) { return 16 * q * (q - 1); }
+
+template <int YT>
 __global__ void __launch_bounds__(kThreads, 1)
 fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                         const __grid_constant__ CUtensorMap map_B,
@@ -248,11 +301,15 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
 
     if (tid == 0) {
         for (int i = 0; i < kNumBars; ++i)
-            mbar_init(bars + i, (i == kBarEmpty0 || i == kBarEmpty1) ? 2 : 1);
+            mbar_init(bars + i, (i == kBarEmpty0 || i == kBarEmpty1) ? 3 : 1);
         fence_mbar_init();
         *abort_flag = 0;
         if (blockIdx.x == 0) p.status[2] = p.epoch;  // the call the status word refers to
     }
+    // the D matrix is zero off its diagonal
+    for (int i = tid; i < 8192 / 16; i += kThreads)
+        reinterpret_cast<uint4*>(smem + kOffDm)[i] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
     if (warp == kWarpMma) {
         tmem_alloc(misc, kTmemCols);
         tmem_relinquish();
@@ -296,11 +353,18 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
     } else if (warp == kWarpMma) {
         // ============================== MMA issue ==============================
         if (lane == 0 && nb_total > 0) {
-            const uint32_t id_st = idesc_f16(kBlk, kP, true, true);
-            const uint32_t id_y = idesc_f16(kBlk, kP, false, true);
+            const uint32_t id_st = idesc_f16(kBlk, kP, true, true);   // B'^T (MN) x xf (MN)
+            const uint32_t id_y = idesc_f16(kBlk, kP, false, true);   // C' / M' (TMEM) x hp / xf
+            const uint32_t id_d = idesc_f16(kBlk, kP, false, false);  // xf (K-major) x D (K-major)
+            const uint32_t sbase = smem_u32(smem);
+            const uint64_t d_bp = smem_desc(sbase + kOffBp, 16384, 1024, kSwizzle128B);
+            const uint64_t d_xf = smem_desc(sbase + kOffXf, 16, 1024, kSwizzle128B);
+            const uint64_t d_hp = smem_desc(sbase + kOffHp, 16, 1024, kSwizzle128B);
+            const uint64_t d_dm = smem_desc(sbase + kOffDm, 16, 1024, kSwizzle128B);
             auto issue_cb_block = [&](int kb) {
                 const int j = kb & 1;
                 wait_phase(bars + kBarFull0 + j, (kb >> 1) & 1, abort_flag, p);
+                // CB buffer j held M'(kb - 2), read by M'x(kb - 2)
                 if (kb >= 2) wait_phase(bars + kBarAcc0 + j, ((kb >> 1) - 1) & 1, abort_flag, p);
                 tc_fence_after();
                 uint8_t* stage = smem + j * kStageBytes;
@@ -312,35 +376,35 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             issue_cb_block(0);
             for (int kb = 0; kb < nb_total && !*abort_flag; ++kb) {  // no new MMA after a failure
                 const int j = kb & 1;
-                const uint32_t xf = smem_u32(smem + kOffXf + j * 16384);
-                const uint32_t bp = smem_u32(smem + kOffBp + j * 32768);
-                const uint32_t hp = smem_u32(smem + kOffHp + j * 16384);
-                wait_phase(bars + kBarPrep0 + j, (kb >> 1) & 1, abort_flag, p);
+                const uint64_t bp = d_bp + static_cast<uint64_t>((j * 32768) >> 4);
+                const uint64_t xf = d_xf + static_cast<uint64_t>((j * 16384) >> 4);
+                const uint64_t hp = d_hp + static_cast<uint64_t>((j * 16384) >> 4);
+                const uint32_t acc = tmem + kColAcc + 64u * j;
+                wait_phase(bars + kBarPb0 + j, (kb >> 1) & 1, abort_flag, p);
+                wait_phase(bars + kBarXf0 + j, (kb >> 1) & 1, abort_flag, p);
                 if (kb >= 2) wait_phase(bars + kBarAccFree0 + j, ((kb >> 1) - 1) & 1, abort_flag, p);
                 tc_fence_after();
                 // state: H += B'^T x   (M = 128 n, N = 64 p, K = 128 t)
 #pragma unroll
                 for (int kk = 0; kk < kBlk / 16; ++kk)
-                    mma_f16_ss(tmem + kColH,
-                               smem_desc(bp + 2048 * kk, 16384, 1024, kSwizzle128B),
-                               smem_desc(xf + 2048 * kk, 16, 1024, kSwizzle128B), id_st, 1);
+                    mma_f16_ss(tmem + kColH, bp + 128 * kk, xf + 128 * kk, id_st, 1);
                 tc_commit(bars + kBarState);
-                // acc = C' H'^T   (A = C' from TMEM, K = 128 n)
+                // acc = C' H'^T (A = C' from TMEM, K = 128 n) + x D (K = 64 p)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_f16_ts(tmem + kColAcc + 64 * j, tmem + kColC + 8 * kk,
-                               smem_desc(hp + 2048 * kk, 16, 1024, kSwizzle128B), id_y, kk > 0);
+                    mma_f16_ts(acc, tmem + kColC + 8 * kk, hp + 128 * kk, id_y, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) mma_f16_ss(acc, xf + 2 * kk, d_dm + 2 * kk, id_d, 1);
                 tc_commit(bars + kBarCh);
                 ++n_ch;
+                if (kb + 1 < nb_total) issue_cb_block(kb + 1);
                 // acc += M' x   (A = M' from TMEM, K = 128 s)
                 wait_phase(bars + kBarMp0 + j, (kb >> 1) & 1, abort_flag, p);
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_f16_ts(tmem + kColAcc + 64 * j, tmem + kColCB + 128u * j + 8 * kk,
-                               smem_desc(xf + 2048 * kk, 16, 1024, kSwizzle128B), id_y, 1);
+                    mma_f16_ts(acc, tmem + kColCB + 128u * j + 8 * kk, xf + 128 * kk, id_y, 1);
                 tc_commit(bars + kBarAcc0 + j);
-                if (kb + 1 < nb_total) issue_cb_block(kb + 1);
             }
         }
         __syncwarp();
@@ -349,7 +413,6 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
         const int row = tid;  // block row t / state row n (TMEM lane)
         const uint32_t lane_base = static_cast<uint32_t>(warp) * 32u;
         float* red = reinterpret_cast<float*>(smem + kOffRed);
-        int kb = 0;
         // previous piece, whose state is stored once its last update is done
         int pv_b = 0, pv_h = 0, pv_cta_end = 0;
         bool pv_valid = false, pv_final = false;
@@ -364,8 +427,8 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                     float* dst = p.final_state + ((size_t)pv_b * p.H + pv_h) * kP * p.N;
                     const float s = pv_out * p.x_scale[pv_h] * p.B_scale[pv_h / (p.H / p.G)];
 #pragma unroll
-                    for (int j = 0; j < 64; ++j)
-                        dst[(size_t)j * p.N + row] = s * __uint_as_float(hv[j / 32][j % 32]);
+                    for (int jj = 0; jj < 64; ++jj)
+                        dst[(size_t)jj * p.N + row] = s * __uint_as_float(hv[jj / 32][jj % 32]);
                 }
             } else if (pv_cta_end) {
                 float4* dst = reinterpret_cast<float4*>(p.slots + ((size_t)blockIdx.x * 128 + row) * kP);
@@ -383,241 +446,276 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 }
             }
         };
-        for (int k = 0; k < rg.nseg; ++k) {
-            int b, h, c_begin, c_end;
-            rg.seg(k, b, h, c_begin, c_end);
+        // cursor over this CTA's blocks, and the per-piece constants
+        int seg = 0, b = 0, h = 0, c_begin = 0, c_end = 0;
+        if (rg.nseg > 0) rg.seg(0, b, h, c_begin, c_end);
+        int c = c_begin;
+        float sx = 1.f, sBg = 1.f, sCg = 1.f, A2h = 0.f, D_h = 0.f;
+        auto load_piece = [&]() {
             const int g = h / (p.H / p.G);
-            const float sx = p.x_scale[h], sBg = p.B_scale[g], sCg = p.C_scale[g];
+            sx = p.x_scale[h];
+            sBg = p.B_scale[g];
+            sCg = p.C_scale[g];
+            A2h = p.A[h] * kLog2e;
+            D_h = p.D[h];
+        };
+        auto dt_at = [&](int bb, int hh, int cc) -> float {
+            const int t = cc * kBlk + row;
+            return t < p.L ? p.dt[((size_t)bb * p.L + t) * p.H + hh] : 0.f;
+        };
+        if (nb_total > 0) load_piece();
+        float d = nb_total > 0 ? dt_at(b, h, c) : 0.f;  // dt of this token, this block
+        float U = 1.f;   // H_true / sigma = U * H_tmem
+        float hb = 0.f;  // running bound on max |H_true| / sigma
+        for (int kb = 0; kb < nb_total; ++kb) {
+            const int j = kb & 1;
+            uint8_t* stage = smem + j * kStageBytes;
+            uint8_t* bp = smem + kOffBp + j * 32768;
+            uint8_t* hp = smem + kOffHp + j * 16384;
+            float* colf = reinterpret_cast<float*>(smem + kOffColf) + j * 192;
+            float* nbeta = reinterpret_cast<float*>(smem + kOffNb) + j * 128;
+            float* a2s = reinterpret_cast<float*>(smem + kOffA2) + j * 128;
             const float sigma = sx * sBg;
-            const float A_h = p.A[h], D_h = p.D[h];
-            const float* dt_bh = p.dt + (size_t)b * p.L * p.H + h;
-            float U = 1.f;   // H_true / sigma = U * H_tmem
-            float hb = 0.f;  // running bound on max |H_true| / sigma
-            for (int c = c_begin; c < c_end; ++c, ++kb) {
-                const int j = kb & 1;
-                uint8_t* stage = smem + j * kStageBytes;
-                uint8_t* xf = smem + kOffXf + j * 16384;
-                uint8_t* bp = smem + kOffBp + j * 32768;
-                uint8_t* hp = smem + kOffHp + j * 16384;
-                float* colf = reinterpret_cast<float*>(smem + kOffColf) + j * 512;
-                float* dts = reinterpret_cast<float*>(smem + kOffDt) + j * 128;
-                float* acum = reinterpret_cast<float*>(smem + kOffAcum) + j * 128;
-                const int valid = min(kBlk, p.L - c * kBlk);
-                // dt of this token (in flight during the waits below)
-                const float d = row < valid ? dt_bh[(size_t)(c * kBlk + row) * p.H] : 0.f;
-                // (a) the previous block's state update is done: H, hp[j], xf[j], bp[j] free
+            const int valid = min(kBlk, p.L - c * kBlk);
+            // the next block of this CTA; its dt is in flight during this block
+            int n_seg = seg, n_b = b, n_h = h, n_cb = c_begin, n_ce = c_end, n_c = c + 1;
+            if (n_c >= c_end && seg + 1 < rg.nseg) {
+                n_seg = seg + 1;
+                rg.seg(n_seg, n_b, n_h, n_cb, n_ce);
+                n_c = n_cb;
+            }
+            const float d_next = kb + 1 < nb_total ? dt_at(n_b, n_h, n_c) : 0.f;
+            // (a) the block tables of buffer j are free once M'(k-2) is built
+            if (kb >= 2) wait_phase(bars + kBarMp0 + j, ((kb >> 1) - 1) & 1, abort_flag, p);
+            // (b) piece start: store the previous piece's state, load this piece's
+            bool state_ready = (kb == 0);
+            if (c == c_begin) {
                 if (kb >= 1) wait_phase(bars + kBarState, (kb - 1) & 1, abort_flag, p);
                 tc_fence_after();
-                // (b) piece start: store the previous piece's state, load this piece's
-                if (c == c_begin) {
-                    if (pv_valid) store_piece();
-                    const float* src = nullptr;
-                    bool from_slot = false;
-                    if (c_begin == 0) {
-                        if (p.init_state) src = p.init_state + ((size_t)b * p.H + h) * kP * p.N;
-                    } else {
-                        if (row == 0) {
-                            const unsigned long long* f = p.flags + (blockIdx.x - 1);
-                            const long long t0 = clock64();
-                            unsigned long long v;
-                            for (;;) {
-                                asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(f) : "memory");
-                                if (v == p.epoch || *abort_flag) break;
-                                if (clock64() - t0 > p.wait_limit) {
-                                    *abort_flag = 1;
-                                    report_failure(p, 2);
-                                    break;
-                                }
-                                __nanosleep(256);
+                state_ready = true;
+                if (pv_valid) store_piece();
+                const float* src = nullptr;
+                bool from_slot = false;
+                if (c_begin == 0) {
+                    if (p.init_state) src = p.init_state + ((size_t)b * p.H + h) * kP * p.N;
+                } else {
+                    if (row == 0) {
+                        const unsigned long long* f = p.flags + (blockIdx.x - 1);
+                        const long long t0 = clock64();
+                        unsigned long long v;
+                        for (;;) {
+                            asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(f) : "memory");
+                            if (v == p.epoch || *abort_flag) break;
+                            if (clock64() - t0 > p.wait_limit) {
+                                *abort_flag = 1;
+                                report_failure(p, 2);
+                                break;
                             }
+                            __nanosleep(256);
                         }
-                        wg_sync(1);
-                        src = p.slots + (size_t)(blockIdx.x - 1) * 128 * kP;
-                        from_slot = true;
-                    }
-                    uint32_t r[2][32];
-                    float m = 0.f;
-#pragma unroll
-                    for (int jj = 0; jj < 64; ++jj) {
-                        float v = 0.f;
-                        if (src != nullptr && row < p.N)
-                            v = from_slot ? __ldcg(src + row * kP + jj) : src[(size_t)jj * p.N + row] / sigma;
-                        m = fmaxf(m, fabsf(v));
-                        r[jj / 32][jj % 32] = __float_as_uint(v);
-                    }
-                    tmem_st32(tmem_addr(tmem, lane_base, kColH), r[0]);
-                    tmem_st32(tmem_addr(tmem, lane_base, kColH + 32), r[1]);
-                    tmem_st_wait();
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                    if (lane == 0) red[16 + warp] = m;
-                    wg_sync(1);
-                    hb = fmaxf(fmaxf(red[16], red[17]), fmaxf(red[18], red[19]));
-                    U = 1.f;
-                }
-                // (c) block scan of dt * A, with the block's max dt and sum dt
-                float incl, dmax, dsum;
-                {
-                    const float a = d * A_h;
-                    float v = a, mx = d, sm = d;
-#pragma unroll
-                    for (int o = 1; o < 32; o <<= 1) {
-                        const float u = __shfl_up_sync(0xffffffffu, v, o);
-                        if (lane >= o) v += u;
-                    }
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) {
-                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                        sm += __shfl_xor_sync(0xffffffffu, sm, o);
-                    }
-                    if (lane == 31) red[warp] = v;
-                    if (lane == 0) {
-                        red[4 + warp] = mx;
-                        red[8 + warp] = sm;
                     }
                     wg_sync(1);
-                    float pre = 0.f;
-                    for (int w = 0; w < warp; ++w) pre += red[w];
-                    incl = v + pre;
-                    dmax = fmaxf(fmaxf(red[4], red[5]), fmaxf(red[6], red[7]));
-                    dsum = (red[8] + red[9]) + (red[10] + red[11]);
-                    dts[row] = d;
-                    acum[row] = incl;
+                    src = p.slots + (size_t)(blockIdx.x - 1) * 128 * kP;
+                    from_slot = true;
                 }
-                wg_sync(1);  // acum complete; red[] free again
-                const float a_end = acum[kBlk - 1];
-                // (d) scales of this block
-                float need = fmaxf(fmaxf(hb, 16129.f * static_cast<float>(p.N) * dmax),
-                                   fabsf(D_h) / (sCg * sBg)) * (1.f / kF16Range);
-                if (!(need > 1e-30f) || !isfinite(need)) need = 1.f;
-                const float rho = pow2_ceil(sCg * sigma * need);
-                const float kappa = rho / (sCg * sigma);
-                const float U_new = dmax > 0.f ? pow2_ceil(127.f * dmax * (1.f / kF16Range)) : U;
-                const float e_end = __expf(a_end);
-                // (e) state hand-over: H' = H / kappa (f16) for C'.H', then decay + rescale
-                {
-                    const float to_hp = U / kappa;
-                    const float to_h = e_end * (U / U_new);
+                uint32_t r[2][32];
+                float m = 0.f;
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        uint32_t hv[32];
-                        tmem_ld32(tmem_addr(tmem, lane_base, kColH + 32 * hh), hv);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint4 v;
-                            v.x = pack_f16x2(__uint_as_float(hv[8 * q + 0]) * to_hp, __uint_as_float(hv[8 * q + 1]) * to_hp);
-                            v.y = pack_f16x2(__uint_as_float(hv[8 * q + 2]) * to_hp, __uint_as_float(hv[8 * q + 3]) * to_hp);
-                            v.z = pack_f16x2(__uint_as_float(hv[8 * q + 4]) * to_hp, __uint_as_float(hv[8 * q + 5]) * to_hp);
-                            v.w = pack_f16x2(__uint_as_float(hv[8 * q + 6]) * to_hp, __uint_as_float(hv[8 * q + 7]) * to_hp);
-                            *reinterpret_cast<uint4*>(hp + sw128(row, 64 * hh + 16 * q)) = v;
-                        }
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) hv[i] = __float_as_uint(__uint_as_float(hv[i]) * to_h);
-                        tmem_st32(tmem_addr(tmem, lane_base, kColH + 32 * hh), hv);
-                    }
-                    U = U_new;
-                    hb = hb * e_end + 16129.f * dsum;  // bound after this block's update
+                for (int jj = 0; jj < 64; ++jj) {
+                    float v = 0.f;
+                    if (src != nullptr && row < p.N)
+                        v = from_slot ? __ldcg(src + row * kP + jj) : src[(size_t)jj * p.N + row] / sigma;
+                    m = fmaxf(m, fabsf(v));
+                    r[jj / 32][jj % 32] = __float_as_uint(v);
                 }
-                // (f) conversions of the block's tiles
+                tmem_st32(tmem_addr(tmem, lane_base, kColH), r[0]);
+                tmem_st32(tmem_addr(tmem, lane_base, kColH + 32), r[1]);
+                tmem_st_wait();
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                if (lane == 0) red[16 + warp] = m;
+                wg_sync(1);
+                hb = fmaxf(fmaxf(red[16], red[17]), fmaxf(red[18], red[19]));
+                U = 1.f;
+            }
+            // (c) block scan of a = log2(e) dt A, with the block's max dt and sum dt
+            float incl, tot, dmax, dsum;
+            {
+                float v = d * A2h, mx = d, sm = d;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float u = __shfl_up_sync(0xffffffffu, v, o);
+                    if (lane >= o) v += u;
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                    sm += __shfl_xor_sync(0xffffffffu, sm, o);
+                }
+                if (lane == 31) red[warp] = v;
+                if (lane == 0) {
+                    red[4 + warp] = mx;
+                    red[8 + warp] = sm;
+                }
+                wg_sync(1);
+                float pre = 0.f;
+                for (int w = 0; w < warp; ++w) pre += red[w];
+                incl = v + pre;
+                tot = ((red[0] + red[1]) + red[2]) + red[3];
+                dmax = fmaxf(fmaxf(red[4], red[5]), fmaxf(red[6], red[7]));
+                dsum = (red[8] + red[9]) + (red[10] + red[11]);
+                a2s[row] = incl;
+            }
+            wg_sync(1);  // a2s complete; red[] free again
+            // (d) scales of this block
+            float need = fmaxf(fmaxf(hb, 16129.f * static_cast<float>(p.N) * dmax),
+                               fabsf(D_h) / (sCg * sBg)) * (1.f / kF16Range);
+            if (!(need > 1e-30f) || !isfinite(need)) need = 1.f;
+            const float rho = pow2_ceil(sCg * sigma * need);
+            const float kappa = rho / (sCg * sigma);
+            const float invk = 1.f / kappa;
+            const float U_new = dmax > 0.f ? pow2_ceil(127.f * dmax * (1.f / kF16Range)) : U;
+            const float e_end = ex2f(tot);
+            // (f) block tables, B', C' and D (independent of the previous block's state)
+            {
+                const float base = d * invk;
+                nbeta[row] = lg2f(base) - incl;  // dt = 0 gives -inf: no contribution
+                if (row < 96) {
+                    colf[colf_off(3) + row] = ex2f(a2s[96] - incl) * base;
+                    if (row < 64) colf[colf_off(2) + row] = ex2f(a2s[64] - incl) * base;
+                    if (row < 32) colf[colf_off(1) + row] = ex2f(a2s[32] - incl) * base;
+                }
+                // B row scaled by w_t / U -> B' (two MN blocks of 64 n)
                 wait_phase(bars + kBarFull0 + j, (kb >> 1) & 1, abort_flag, p);
-                {
-                    // x row -> f16 (64 values)
-                    const uint4* xs = reinterpret_cast<const uint4*>(stage + kStX + row * 64);
+                const __half2 w2 = __float2half2_rn(d * ex2f(tot - incl) * (1.f / U_new));
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const uint4 w = *reinterpret_cast<const uint4*>(stage + kStB + sw128(row, 16 * q));
+                    uint4 o0, o1;
+                    i8x4_to_h2x2(w.x, o0.x, o0.y);
+                    i8x4_to_h2x2(w.y, o0.z, o0.w);
+                    i8x4_to_h2x2(w.z, o1.x, o1.y);
+                    i8x4_to_h2x2(w.w, o1.z, o1.w);
+                    o0.x = hmul2_u32(o0.x, w2); o0.y = hmul2_u32(o0.y, w2);
+                    o0.z = hmul2_u32(o0.z, w2); o0.w = hmul2_u32(o0.w, w2);
+                    o1.x = hmul2_u32(o1.x, w2); o1.y = hmul2_u32(o1.y, w2);
+                    o1.z = hmul2_u32(o1.z, w2); o1.w = hmul2_u32(o1.w, w2);
+                    uint8_t* blk = bp + (q / 4) * 16384;
+                    *reinterpret_cast<uint4*>(blk + sw128(row, 32 * (q % 4))) = o0;
+                    *reinterpret_cast<uint4*>(blk + sw128(row, 32 * (q % 4) + 16)) = o1;
+                }
+                // C row scaled by 2^a_t -> C' in TMEM, and D, once the previous C'H' is done
+                if (kb >= 1) wait_phase(bars + kBarCh, (kb - 1) & 1, abort_flag, p);
+                tc_fence_after();
+                const __half2 f2h = __float2half2_rn(ex2f(incl));
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t r[32];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const uint4 w = xs[q];
-                        uint4 o0, o1;
-                        i8x4_to_h2x2(w.x, o0.x, o0.y);
-                        i8x4_to_h2x2(w.y, o0.z, o0.w);
-                        i8x4_to_h2x2(w.z, o1.x, o1.y);
-                        i8x4_to_h2x2(w.w, o1.z, o1.w);
-                        *reinterpret_cast<uint4*>(xf + sw128(row, 32 * q)) = o0;
-                        *reinterpret_cast<uint4*>(xf + sw128(row, 32 * q + 16)) = o1;
-                    }
-                    // B row scaled by w_t / U -> B' (two MN blocks of 64 n)
-                    const float wt = row < valid ? d * __expf(a_end - incl) / U : 0.f;
-                    const __half2 w2 = __float2half2_rn(wt);
+                        const uint4 w = *reinterpret_cast<const uint4*>(stage + kStC + sw128(row, 16 * (4 * hh + q)));
+                        i8x4_to_h2x2(w.x, r[8 * q + 0], r[8 * q + 1]);
+                        i8x4_to_h2x2(w.y, r[8 * q + 2], r[8 * q + 3]);
+                        i8x4_to_h2x2(w.z, r[8 * q + 4], r[8 * q + 5]);
+                        i8x4_to_h2x2(w.w, r[8 * q + 6], r[8 * q + 7]);
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const uint4 w = *reinterpret_cast<const uint4*>(stage + kStB + sw128(row, 16 * q));
-                        uint4 o0, o1;
-                        i8x4_to_h2x2(w.x, o0.x, o0.y);
-                        i8x4_to_h2x2(w.y, o0.z, o0.w);
-                        i8x4_to_h2x2(w.z, o1.x, o1.y);
-                        i8x4_to_h2x2(w.w, o1.z, o1.w);
-                        o0.x = hmul2_u32(o0.x, w2); o0.y = hmul2_u32(o0.y, w2);
-                        o0.z = hmul2_u32(o0.z, w2); o0.w = hmul2_u32(o0.w, w2);
-                        o1.x = hmul2_u32(o1.x, w2); o1.y = hmul2_u32(o1.y, w2);
-                        o1.z = hmul2_u32(o1.z, w2); o1.w = hmul2_u32(o1.w, w2);
-                        uint8_t* blk = bp + (q / 4) * 16384;
-                        *reinterpret_cast<uint4*>(blk + sw128(row, 32 * (q % 4))) = o0;
-                        *reinterpret_cast<uint4*>(blk + sw128(row, 32 * (q % 4) + 16)) = o1;
+                        for (int i = 0; i < 8; ++i) r[8 * q + i] = hmul2_u32(r[8 * q + i], f2h);
                     }
-                    // C row scaled by exp(Acum_t) -> C' in TMEM, once the previous C'.H' is done
-                    if (kb >= 1) wait_phase(bars + kBarCh, (kb - 1) & 1, abort_flag, p);
-                    tc_fence_after();
-                    const __half2 f2 = __float2half2_rn(__expf(incl));
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        uint32_t r[32];
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const uint4 w = *reinterpret_cast<const uint4*>(stage + kStC + sw128(row, 16 * (4 * hh + q)));
-                            i8x4_to_h2x2(w.x, r[8 * q + 0], r[8 * q + 1]);
-                            i8x4_to_h2x2(w.y, r[8 * q + 2], r[8 * q + 3]);
-                            i8x4_to_h2x2(w.z, r[8 * q + 4], r[8 * q + 5]);
-                            i8x4_to_h2x2(w.w, r[8 * q + 6], r[8 * q + 7]);
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) r[8 * q + i] = hmul2_u32(r[8 * q + i], f2);
-                        }
-                        tmem_st32(tmem_addr(tmem, lane_base, kColC + 32 * hh), r);
-                    }
-                    // column factors exp(Acum_{32 q} - Acum_s) dt_s / kappa for s < 32 q
-                    for (int idx = row; idx < 192; idx += kBlk) {
-                        const int q = idx < 32 ? 1 : (idx < 96 ? 2 : 3);
-                        const int s = idx - (q == 1 ? 0 : (q == 2 ? 32 : 96));
-                        colf[q * 128 + s] = __expf(acum[32 * q] - acum[s]) * dts[s] / kappa;
-                    }
-                    if (row == 0) {
-                        BlockInfo bi;
-                        bi.rho = rho;
-                        bi.inv_kappa = 1.f / kappa;
-                        bi.dterm = D_h * sx / rho;
-                        bi.pad = 0.f;
-                        bi.b = b;
-                        bi.h = h;
-                        bi.c = c;
-                        bi.valid = valid;
-                        info[j] = bi;
-                    }
+                    tmem_st32(tmem_addr(tmem, lane_base, kColC + 32 * hh), r);
                 }
-                fence_proxy_async_smem();
-                tmem_st_wait();
-                tc_fence_before();
-                wg_sync(1);
+                if (row < kP)
+                    *reinterpret_cast<__half*>(smem + kOffDm + sw128(row, 2 * row)) =
+                        __float2half_rn(D_h * sx / rho);
                 if (row == 0) {
-                    mbar_arrive(bars + kBarEmpty0 + j);
-                    mbar_arrive(bars + kBarPrep0 + j);
+                    BlockInfo bi;
+                    bi.rho = rho;
+                    bi.inv_kappa = invk;
+                    bi.b = b;
+                    bi.h = h;
+                    bi.c = c;
+                    bi.valid = valid;
+                    bi.pad0 = bi.pad1 = 0;
+                    info[j] = bi;
                 }
             }
-            // this piece's state is stored when the next piece starts (or below)
-            pv_valid = true;
-            pv_b = b;
-            pv_h = h;
-            pv_final = (c_end == p.nblk);
-            pv_cta_end = (c_end != p.nblk);
-            pv_out = U;
+            fence_proxy_async_smem();
+            tmem_st_wait();
+            tc_fence_before();
+            wg_sync(1);
+            if (row == 0) {
+                mbar_arrive(bars + kBarEmpty0 + j);
+                mbar_arrive(bars + kBarPa0 + j);
+            }
+            // (e) state hand-over: H' = H U / kappa (f16) for C'H', then decay + rescale
+            if (!state_ready) wait_phase(bars + kBarState, (kb - 1) & 1, abort_flag, p);
+            tc_fence_after();
+            {
+                const f2 to_hp = {U * invk, U * invk};
+                const float th = e_end * (U / U_new);
+                const f2 to_h = {th, th};
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t hv[32];
+                    tmem_ld32(tmem_addr(tmem, lane_base, kColH + 32 * hh), hv);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const f2 v = fmul2(f2{__uint_as_float(hv[8 * q + 2 * i]),
+                                                  __uint_as_float(hv[8 * q + 2 * i + 1])}, to_hp);
+                            w[i] = pack_f16x2(v.x, v.y);
+                        }
+                        *reinterpret_cast<uint4*>(hp + sw128(row, 64 * hh + 16 * q)) =
+                            make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const f2 v = fmul2(f2{__uint_as_float(hv[2 * i]), __uint_as_float(hv[2 * i + 1])}, to_h);
+                        hv[2 * i] = __float_as_uint(v.x);
+                        hv[2 * i + 1] = __float_as_uint(v.y);
+                    }
+                    tmem_st32(tmem_addr(tmem, lane_base, kColH + 32 * hh), hv);
+                }
+                U = U_new;
+                hb = hb * e_end + 16129.f * dsum;  // bound after this block's update
+            }
+            fence_proxy_async_smem();
+            tmem_st_wait();
+            tc_fence_before();
+            wg_sync(1);
+            if (row == 0) mbar_arrive(bars + kBarPb0 + j);
+            // piece end: its state is stored when the next piece starts (or below)
+            if (c + 1 == c_end) {
+                pv_valid = true;
+                pv_b = b;
+                pv_h = h;
+                pv_final = (c_end == p.nblk);
+                pv_cta_end = (c_end != p.nblk);
+                pv_out = U;
+            }
+            if (n_seg != seg) {
+                seg = n_seg;
+                b = n_b;
+                h = n_h;
+                c_begin = n_cb;
+                c_end = n_ce;
+                load_piece();
+            }
+            c = n_c;
+            d = d_next;
         }
         if (pv_valid) {
-            wait_phase(bars + kBarState, (kb - 1) & 1, abort_flag, p);
+            wait_phase(bars + kBarState, (nb_total - 1) & 1, abort_flag, p);
             tc_fence_after();
             store_piece();
         }
     } else {
-        // ============================== M' and output warpgroup ==============================
+        // ============================== x, M' and output warpgroup ==============================
         const int quad = warp & 3;
         const int row = quad * 32 + lane;
+        const int lt = tid - 128;
         const uint32_t lane_base = static_cast<uint32_t>(quad) * 32u;
         // output of the previous block
         int pv_j = 0, pv_b = 0, pv_h = 0, pv_c = 0, pv_valid = 0;
@@ -631,87 +729,120 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             tmem_ld_wait();
             tc_fence_before();
             wg_sync(2);
-            if (row == 0 + 0 && quad == 0 && lane == 0) mbar_arrive(bars + kBarAccFree0 + pv_j);
+            if (lt == 0) mbar_arrive(bars + kBarAccFree0 + pv_j);
             if (row < pv_valid) {
                 const size_t ybase = (((size_t)pv_b * p.L + (size_t)pv_c * kBlk + row) * p.H + pv_h) * kP;
-                if (p.y_dtype == SSD_OUT_I8) {
-                    const float sc = pv_rho * p.inv_y_scale;
+                if constexpr (YT == SSD_OUT_I8) {
+                    // q = clamp(rint(fp32(acc * rho / s_y))): the same rounding as the fp32 output
+                    const float s = pv_rho * p.inv_y_scale;
+                    const f2 s2 = {s, s}, rnd = {kRound, kRound};
                     uint32_t wv[16];
 #pragma unroll
                     for (int q = 0; q < 16; ++q) {
                         const uint32_t* rr = &r[q / 8][(q % 8) * 4];
-                        wv[q] = q8(__uint_as_float(rr[0]) * sc) | (q8(__uint_as_float(rr[1]) * sc) << 8) |
-                                (q8(__uint_as_float(rr[2]) * sc) << 16) | (q8(__uint_as_float(rr[3]) * sc) << 24);
+                        const f2 v0 = fadd2(fmul2(f2{__uint_as_float(rr[0]), __uint_as_float(rr[1])}, s2), rnd);
+                        const f2 v1 = fadd2(fmul2(f2{__uint_as_float(rr[2]), __uint_as_float(rr[3])}, s2), rnd);
+                        const uint32_t lo = __byte_perm(clamp_code(v0.x), clamp_code(v0.y), 0x0040);
+                        const uint32_t hi = __byte_perm(clamp_code(v1.x), clamp_code(v1.y), 0x0040);
+                        wv[q] = __byte_perm(lo, hi, 0x5410);
                     }
                     uint4* yo = reinterpret_cast<uint4*>(static_cast<int8_t*>(p.y) + ybase);
 #pragma unroll
                     for (int q = 0; q < 4; ++q) yo[q] = make_uint4(wv[4 * q], wv[4 * q + 1], wv[4 * q + 2], wv[4 * q + 3]);
-                } else if (p.y_dtype == SSD_OUT_F16) {
+                } else if constexpr (YT == SSD_OUT_F16) {
+                    const f2 s2 = {pv_rho, pv_rho};
                     uint4* yo = reinterpret_cast<uint4*>(static_cast<__half*>(p.y) + ybase);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         const uint32_t* rr = &r[q / 4][(q % 4) * 8];
-                        yo[q] = make_uint4(pack_f16x2(__uint_as_float(rr[0]) * pv_rho, __uint_as_float(rr[1]) * pv_rho),
-                                           pack_f16x2(__uint_as_float(rr[2]) * pv_rho, __uint_as_float(rr[3]) * pv_rho),
-                                           pack_f16x2(__uint_as_float(rr[4]) * pv_rho, __uint_as_float(rr[5]) * pv_rho),
-                                           pack_f16x2(__uint_as_float(rr[6]) * pv_rho, __uint_as_float(rr[7]) * pv_rho));
+                        uint32_t w[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const f2 v = fmul2(f2{__uint_as_float(rr[2 * i]), __uint_as_float(rr[2 * i + 1])}, s2);
+                            w[i] = pack_f16x2(v.x, v.y);
+                        }
+                        yo[q] = make_uint4(w[0], w[1], w[2], w[3]);
                     }
                 } else {
+                    const f2 s2 = {pv_rho, pv_rho};
                     float4* yo = reinterpret_cast<float4*>(static_cast<float*>(p.y) + ybase);
 #pragma unroll
                     for (int q = 0; q < 16; ++q) {
                         const uint32_t* rr = &r[q / 8][(q % 8) * 4];
-                        yo[q] = make_float4(__uint_as_float(rr[0]) * pv_rho, __uint_as_float(rr[1]) * pv_rho,
-                                            __uint_as_float(rr[2]) * pv_rho, __uint_as_float(rr[3]) * pv_rho);
+                        const f2 v0 = fmul2(f2{__uint_as_float(rr[0]), __uint_as_float(rr[1])}, s2);
+                        const f2 v1 = fmul2(f2{__uint_as_float(rr[2]), __uint_as_float(rr[3])}, s2);
+                        yo[q] = make_float4(v0.x, v0.y, v1.x, v1.y);
                     }
                 }
             }
         };
         for (int kb = 0; kb < nb_total; ++kb) {
             const int j = kb & 1;
-            const float* colf = reinterpret_cast<const float*>(smem + kOffColf) + j * 512;
-            const float* dts = reinterpret_cast<const float*>(smem + kOffDt) + j * 128;
-            const float* acum = reinterpret_cast<const float*>(smem + kOffAcum) + j * 128;
+            const uint8_t* stage = smem + j * kStageBytes;
+            uint8_t* xf = smem + kOffXf + j * 16384;
+            const float* colf = reinterpret_cast<const float*>(smem + kOffColf) + j * 192;
+            const float* nbeta = reinterpret_cast<const float*>(smem + kOffNb) + j * 128;
+            const float* a2s = reinterpret_cast<const float*>(smem + kOffA2) + j * 128;
             const uint32_t col_cb = kColCB + 128u * j;
-            wait_phase(bars + kBarPrep0 + j, (kb >> 1) & 1, abort_flag, p);
+            // ---- x -> f16: a quarter row (16 tokens' bytes) per thread and step ----
+            wait_phase(bars + kBarFull0 + j, (kb >> 1) & 1, abort_flag, p);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int idx = lt + 128 * i;
+                const int r = idx >> 2, c4 = idx & 3;
+                const uint4 w = *reinterpret_cast<const uint4*>(stage + kStX + r * 64 + 16 * c4);
+                uint4 o0, o1;
+                i8x4_to_h2x2(w.x, o0.x, o0.y);
+                i8x4_to_h2x2(w.y, o0.z, o0.w);
+                i8x4_to_h2x2(w.z, o1.x, o1.y);
+                i8x4_to_h2x2(w.w, o1.z, o1.w);
+                *reinterpret_cast<uint4*>(xf + sw128(r, 32 * c4)) = o0;
+                *reinterpret_cast<uint4*>(xf + sw128(r, 32 * c4 + 16)) = o1;
+            }
+            fence_proxy_async_smem();
+            wg_sync(2);
+            if (lt == 0) {
+                mbar_arrive(bars + kBarXf0 + j);
+                mbar_arrive(bars + kBarEmpty0 + j);
+            }
+            // ---- M' in place over CB, one 32-column chunk at a time (increasing order) ----
+            wait_phase(bars + kBarPa0 + j, (kb >> 1) & 1, abort_flag, p);
             const BlockInfo bi = info[j];
             wait_phase(bars + kBarCb0 + j, (kb >> 1) & 1, abort_flag, p);
             tc_fence_after();
-            // ---- M' in place over CB, one 32-column chunk at a time (increasing order) ----
             {
-                const bool row_ok = row < bi.valid;
-                const float at = acum[row];
-                const float rowf = row_ok ? __expf(at - acum[32 * quad]) : 0.f;
+                const float a2t = a2s[row];
+                const int tl = row & 31;
+                const f2 a2t2 = {a2t, a2t};
+                const float rowf = quad > 0 ? ex2f(a2t - a2s[32 * quad]) : 0.f;
+                const f2 rowf2 = {rowf, rowf};
+                const float* cfq = colf + colf_off(quad);
                 for (int sc = 0; sc < 4; ++sc) {
                     uint32_t o[16];
-                    if (sc <= quad) {
+                    if (sc < quad) {
+                        // 2^(a_t - a_s) = 2^(a_t - a_32q) * 2^(a_32q - a_s), both factors <= 1
                         uint32_t cbv[32];
                         tmem_ld32(tmem_addr(tmem, lane_base, col_cb + 32 * sc), cbv);
                         tmem_ld_wait();
-                        if (sc < quad) {
-                            const float* cf = colf + quad * 128 + 32 * sc;
+                        const float2* cf = reinterpret_cast<const float2*>(cfq + 32 * sc);
 #pragma unroll
-                            for (int e = 0; e < 16; ++e) {
-                                const float2 f = *reinterpret_cast<const float2*>(cf + 2 * e);
-                                o[e] = pack_f16x2(i32_to_f32_small(cbv[2 * e]) * f.x * rowf,
-                                                  i32_to_f32_small(cbv[2 * e + 1]) * f.y * rowf);
-                            }
-                        } else {
+                        for (int e = 0; e < 16; ++e) {
+                            const float2 c2 = cf[e];
+                            const f2 v = fmul2(fmul2(cb_pair(cbv[2 * e], cbv[2 * e + 1]), f2{c2.x, c2.y}), rowf2);
+                            o[e] = pack_f16x2(v.x, v.y);
+                        }
+                    } else if (sc == quad) {
+                        // diagonal sub-block: one exponential per entry, s > t masked
+                        uint32_t cbv[32];
+                        tmem_ld32(tmem_addr(tmem, lane_base, col_cb + 32 * sc), cbv);
+                        tmem_ld_wait();
+                        const float2* nb = reinterpret_cast<const float2*>(nbeta + 32 * sc);
 #pragma unroll
-                            for (int e = 0; e < 16; ++e) {
-                                float mv[2];
-#pragma unroll
-                                for (int z = 0; z < 2; ++z) {
-                                    const int s = 32 * sc + 2 * e + z;
-                                    float v = 0.f;
-                                    if (row_ok && s <= row)
-                                        v = i32_to_f32_small(cbv[2 * e + z]) * __expf(at - acum[s]) *
-                                            dts[s] * bi.inv_kappa;
-                                    if (row_ok && s == row) v += bi.dterm;
-                                    mv[z] = v;
-                                }
-                                o[e] = pack_f16x2(mv[0], mv[1]);
-                            }
+                        for (int e = 0; e < 16; ++e) {
+                            const float2 n2 = nb[e];
+                            const f2 arg = fadd2(a2t2, f2{n2.x, n2.y});
+                            const f2 v = fmul2(cb_pair(cbv[2 * e], cbv[2 * e + 1]), f2{ex2f(arg.x), ex2f(arg.y)});
+                            o[e] = pack_f16x2(2 * e <= tl ? v.x : 0.f, 2 * e + 1 <= tl ? v.y : 0.f);
                         }
                     } else {
 #pragma unroll
@@ -723,7 +854,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             }
             tc_fence_before();
             wg_sync(2);
-            if (tid == 128) mbar_arrive(bars + kBarMp0 + j);
+            if (lt == 0) mbar_arrive(bars + kBarMp0 + j);
             // ---- output of the previous block while the tensor core runs this one ----
             if (kb >= 1) output(kb - 1);
             pv_j = j;
@@ -897,6 +1028,16 @@ long long total_blocks(int batch, int seqlen, int nheads) {
     return (long long)batch * nheads * ceil_div(seqlen, kBlk);
 }
 
+template <int YT>
+cudaError_t launch_fused(const CUtensorMap& mx, const CUtensorMap& mB, const CUtensorMap& mC,
+                         const FusedParams& p, cudaStream_t st) {
+    cudaError_t e = cudaFuncSetAttribute(fused_chunk_scan_kernel<YT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    fused_chunk_scan_kernel<YT><<<p.nctas, kThreads, kSmemBytes, st>>>(mx, mB, mC, p);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 size_t chunk_scan_workspace_bytes(int batch, int seqlen, int nheads, int headdim, int dstate,
@@ -917,7 +1058,7 @@ cudaError_t launch_chunk_scan(const ChunkScanArgs& a, cudaStream_t st) {
     FusedParams p{};
     p.dt = a.dt; p.A = a.A; p.D = a.D; p.x_scale = a.x_scale; p.B_scale = a.B_scale;
     p.C_scale = a.C_scale; p.init_state = a.init_state; p.final_state = a.final_state;
-    p.y = a.y; p.y_dtype = a.y_dtype; p.inv_y_scale = a.inv_y_scale;
+    p.y = a.y; p.inv_y_scale = a.inv_y_scale;
     p.batch = a.batch; p.L = a.seqlen; p.H = a.nheads; p.G = a.ngroups; p.N = a.dstate;
     p.nblk = ceil_div(a.seqlen, kBlk);
     p.total = total_blocks(a.batch, a.seqlen, a.nheads);
@@ -939,11 +1080,12 @@ cudaError_t launch_chunk_scan(const ChunkScanArgs& a, cudaStream_t st) {
             g_inject_armed = false;
         }
     }
-    cudaError_t e = cudaFuncSetAttribute(fused_chunk_scan_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    fused_chunk_scan_kernel<<<p.nctas, kThreads, kSmemBytes, st>>>(mx, mB, mC, p);
-    return cudaGetLastError();
+    switch (a.y_dtype) {
+        case SSD_OUT_F32: return launch_fused<SSD_OUT_F32>(mx, mB, mC, p, st);
+        case SSD_OUT_F16: return launch_fused<SSD_OUT_F16>(mx, mB, mC, p, st);
+        case SSD_OUT_I8: return launch_fused<SSD_OUT_I8>(mx, mB, mC, p, st);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 void arm_fault_injection(int drop_publish_cta, long long wait_cycles) {
