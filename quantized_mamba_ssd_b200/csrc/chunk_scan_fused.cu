@@ -249,16 +249,21 @@ __device__ __forceinline__ float pow2_ceil(float v) {
     return __uint_as_float((b & 0x7F800000u) + 0x00800000u);
 }
 
+// 1 / v for v a power of two in [2^-126, 2^126] (exact)
+__device__ __forceinline__ float inv_pow2(float v) {
+    return __uint_as_float(0x7F000000u - __float_as_uint(v));
+}
+
 __device__ void report_failure(const FusedParams& p, unsigned long long code) {
     p.status[1] = code;
     __threadfence();
     atomicExch(p.status, p.epoch);
 }
 
-// Bounded wait that gives up at once after any failure of the CTA.
-__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity,
-                                           volatile uint32_t* abort_flag, const FusedParams& p) {
-    if (mbar_try_wait(bar, parity)) return true;
+// Bounded wait that gives up at once after any failure of the CTA: an inline test, and the
+// polling loop out of line (it keeps the hot loops small).
+__device__ __noinline__ bool wait_phase_slow(uint64_t* bar, uint32_t parity,
+                                             volatile uint32_t* abort_flag, const FusedParams& p) {
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
         if (*abort_flag) return false;
@@ -271,6 +276,11 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity,
     return true;
 }
 
+__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity,
+                                           volatile uint32_t* abort_flag, const FusedParams& p) {
+    return mbar_try_wait(bar, parity) || wait_phase_slow(bar, parity, abort_flag, p);
+}
+
 // ChunkBMM MMAs: D[tmem] = C rows [t0, t0+128) x B rows [0, ncols), K = 128 (int8).
 __device__ __forceinline__ void issue_cb(uint32_t d, uint32_t sC, uint32_t sB, int t0, int ncols) {
     const uint32_t id = idesc_i8(kBlk, ncols, false, false);
@@ -280,6 +290,99 @@ __device__ __forceinline__ void issue_cb(uint32_t d, uint32_t sC, uint32_t sB, i
     for (int k = 0; k < 4; ++k) mma_i8_ss(d, a0 + 2 * k, b0 + 2 * k, id, k > 0);
 }
 
+// Piece end (prep warpgroup, thread = state row n): writes the state of the finished piece,
+// either as the caller's final state or into this CTA's hand-off slot (then publishes the slot).
+// `out_scale` converts TMEM units to units of s_x s_B.  Kept out of line: it runs once or twice
+// per CTA.
+__device__ __noinline__ void store_piece_state(const FusedParams& p, uint32_t tmem, int row,
+                                               bool final_piece, bool cta_end, int b, int h,
+                                               float out_scale) {
+    const uint32_t lane_base = static_cast<uint32_t>(row & ~31);
+    uint32_t hv[2][32];
+    tmem_ld32(tmem_addr(tmem, lane_base, kColH), hv[0]);
+    tmem_ld32(tmem_addr(tmem, lane_base, kColH + 32), hv[1]);
+    tmem_ld_wait();
+    if (final_piece) {
+        if (p.final_state != nullptr && row < p.N) {
+            float* dst = p.final_state + ((size_t)b * p.H + h) * kP * p.N;
+            const float s = out_scale * p.x_scale[h] * p.B_scale[h / (p.H / p.G)];
+#pragma unroll
+            for (int jj = 0; jj < 64; ++jj)
+                dst[(size_t)jj * p.N + row] = s * __uint_as_float(hv[jj / 32][jj % 32]);
+        }
+    } else if (cta_end) {
+        float4* dst = reinterpret_cast<float4*>(p.slots + ((size_t)blockIdx.x * 128 + row) * kP);
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+            dst[q] = make_float4(out_scale * __uint_as_float(hv[(4 * q) / 32][(4 * q) % 32]),
+                                 out_scale * __uint_as_float(hv[(4 * q + 1) / 32][(4 * q + 1) % 32]),
+                                 out_scale * __uint_as_float(hv[(4 * q + 2) / 32][(4 * q + 2) % 32]),
+                                 out_scale * __uint_as_float(hv[(4 * q + 3) / 32][(4 * q + 3) % 32]));
+        __threadfence();
+        wg_sync(1);
+        if (row == 0 && p.drop_publish != static_cast<int>(blockIdx.x)) {
+            unsigned long long* f = p.flags + blockIdx.x;
+            asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(f), "l"(p.epoch) : "memory");
+        }
+    }
+}
+
+// Piece start (prep warpgroup): loads the piece's initial state into TMEM in units of s_x s_B:
+// the caller's initial state (or zero) at sequence start, else the predecessor CTA's hand-off
+// slot after a bounded wait for its flag.  Returns max |state| over the piece's state.
+__device__ __noinline__ float load_piece_state(const FusedParams& p, uint32_t tmem, int row,
+                                               float* red, volatile uint32_t* abort_flag, int b,
+                                               int h, int c_begin, float sigma) {
+    const int warp = row >> 5, lane = row & 31;
+    const uint32_t lane_base = static_cast<uint32_t>(row & ~31);
+    const float* src = nullptr;
+    bool from_slot = false;
+    if (c_begin == 0) {
+        if (p.init_state) src = p.init_state + ((size_t)b * p.H + h) * kP * p.N;
+    } else {
+        if (row == 0) {
+            const unsigned long long* f = p.flags + (blockIdx.x - 1);
+            const long long t0 = clock64();
+            unsigned long long v;
+            for (;;) {
+                asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(f) : "memory");
+                if (v == p.epoch || *abort_flag) break;
+                if (clock64() - t0 > p.wait_limit) {
+                    *abort_flag = 1;
+                    report_failure(p, 2);
+                    break;
+                }
+                __nanosleep(256);
+            }
+        }
+        wg_sync(1);
+        src = p.slots + (size_t)(blockIdx.x - 1) * 128 * kP;
+        from_slot = true;
+    }
+    const float inv_sigma = 1.f / sigma;
+    float m = 0.f;
+#pragma unroll 1
+    for (int half = 0; half < 2; ++half) {
+        uint32_t r[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int jj = 32 * half + i;
+            float v = 0.f;
+            if (src != nullptr && row < p.N)
+                v = from_slot ? __ldcg(src + row * kP + jj) : src[(size_t)jj * p.N + row] * inv_sigma;
+            m = fmaxf(m, fabsf(v));
+            r[i] = __float_as_uint(v);
+        }
+        tmem_st32(tmem_addr(tmem, lane_base, kColH + 32 * half), r);
+    }
+    tmem_st_wait();
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) red[16 + warp] = m;
+    wg_sync(1);
+    return fmaxf(fmaxf(red[16], red[17]), fmaxf(red[18], red[19]));
+}
+
 // start column of quad q's off-diagonal column factors (q = 1, 2, 3 hold 32 q entries)
 __host__ __device__ constexpr int colf_off(int q) { return 16 * q * (q - 1); }
 
@@ -287,10 +390,12 @@ template <int YT>
 __global__ void __launch_bounds__(kThreads, 1)
 fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                         const __grid_constant__ CUtensorMap map_B,
-                        const __grid_constant__ CUtensorMap map_C, const FusedParams p) {
+                        const __grid_constant__ CUtensorMap map_C,
+                        const __grid_constant__ FusedParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    // 1024-byte aligned base; offsetting the shared array (not an integer round trip) keeps
+    // every access below in the shared state space
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
     uint32_t* misc = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile uint32_t* abort_flag = misc + 1;
@@ -414,43 +519,14 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
         const uint32_t lane_base = static_cast<uint32_t>(warp) * 32u;
         float* red = reinterpret_cast<float*>(smem + kOffRed);
         // previous piece, whose state is stored once its last update is done
-        int pv_b = 0, pv_h = 0, pv_cta_end = 0;
-        bool pv_valid = false, pv_final = false;
+        int pv_b = 0, pv_h = 0;
+        bool pv_valid = false, pv_final = false, pv_cta_end = false;
         float pv_out = 1.f;  // H_true / s_x s_B = pv_out * H_tmem
-        auto store_piece = [&]() {
-            uint32_t hv[2][32];
-            tmem_ld32(tmem_addr(tmem, lane_base, kColH), hv[0]);
-            tmem_ld32(tmem_addr(tmem, lane_base, kColH + 32), hv[1]);
-            tmem_ld_wait();
-            if (pv_final) {
-                if (p.final_state != nullptr && row < p.N) {
-                    float* dst = p.final_state + ((size_t)pv_b * p.H + pv_h) * kP * p.N;
-                    const float s = pv_out * p.x_scale[pv_h] * p.B_scale[pv_h / (p.H / p.G)];
-#pragma unroll
-                    for (int jj = 0; jj < 64; ++jj)
-                        dst[(size_t)jj * p.N + row] = s * __uint_as_float(hv[jj / 32][jj % 32]);
-                }
-            } else if (pv_cta_end) {
-                float4* dst = reinterpret_cast<float4*>(p.slots + ((size_t)blockIdx.x * 128 + row) * kP);
-#pragma unroll
-                for (int q = 0; q < 16; ++q)
-                    dst[q] = make_float4(pv_out * __uint_as_float(hv[(4 * q) / 32][(4 * q) % 32]),
-                                         pv_out * __uint_as_float(hv[(4 * q + 1) / 32][(4 * q + 1) % 32]),
-                                         pv_out * __uint_as_float(hv[(4 * q + 2) / 32][(4 * q + 2) % 32]),
-                                         pv_out * __uint_as_float(hv[(4 * q + 3) / 32][(4 * q + 3) % 32]));
-                __threadfence();
-                wg_sync(1);
-                if (row == 0 && p.drop_publish != static_cast<int>(blockIdx.x)) {
-                    unsigned long long* f = p.flags + blockIdx.x;
-                    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(f), "l"(p.epoch) : "memory");
-                }
-            }
-        };
         // cursor over this CTA's blocks, and the per-piece constants
         int seg = 0, b = 0, h = 0, c_begin = 0, c_end = 0;
         if (rg.nseg > 0) rg.seg(0, b, h, c_begin, c_end);
         int c = c_begin;
-        float sx = 1.f, sBg = 1.f, sCg = 1.f, A2h = 0.f, D_h = 0.f;
+        float sx = 1.f, sBg = 1.f, sCg = 1.f, A2h = 0.f, D_h = 0.f, d_bound = 0.f;
         auto load_piece = [&]() {
             const int g = h / (p.H / p.G);
             sx = p.x_scale[h];
@@ -458,6 +534,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             sCg = p.C_scale[g];
             A2h = p.A[h] * kLog2e;
             D_h = p.D[h];
+            d_bound = fabsf(D_h) / (sCg * sBg);  // |D s_x / rho| <= 2^14 needs kappa >= this / 2^14
         };
         auto dt_at = [&](int bb, int hh, int cc) -> float {
             const int t = cc * kBlk + row;
@@ -493,49 +570,8 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 if (kb >= 1) wait_phase(bars + kBarState, (kb - 1) & 1, abort_flag, p);
                 tc_fence_after();
                 state_ready = true;
-                if (pv_valid) store_piece();
-                const float* src = nullptr;
-                bool from_slot = false;
-                if (c_begin == 0) {
-                    if (p.init_state) src = p.init_state + ((size_t)b * p.H + h) * kP * p.N;
-                } else {
-                    if (row == 0) {
-                        const unsigned long long* f = p.flags + (blockIdx.x - 1);
-                        const long long t0 = clock64();
-                        unsigned long long v;
-                        for (;;) {
-                            asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(f) : "memory");
-                            if (v == p.epoch || *abort_flag) break;
-                            if (clock64() - t0 > p.wait_limit) {
-                                *abort_flag = 1;
-                                report_failure(p, 2);
-                                break;
-                            }
-                            __nanosleep(256);
-                        }
-                    }
-                    wg_sync(1);
-                    src = p.slots + (size_t)(blockIdx.x - 1) * 128 * kP;
-                    from_slot = true;
-                }
-                uint32_t r[2][32];
-                float m = 0.f;
-#pragma unroll
-                for (int jj = 0; jj < 64; ++jj) {
-                    float v = 0.f;
-                    if (src != nullptr && row < p.N)
-                        v = from_slot ? __ldcg(src + row * kP + jj) : src[(size_t)jj * p.N + row] / sigma;
-                    m = fmaxf(m, fabsf(v));
-                    r[jj / 32][jj % 32] = __float_as_uint(v);
-                }
-                tmem_st32(tmem_addr(tmem, lane_base, kColH), r[0]);
-                tmem_st32(tmem_addr(tmem, lane_base, kColH + 32), r[1]);
-                tmem_st_wait();
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                if (lane == 0) red[16 + warp] = m;
-                wg_sync(1);
-                hb = fmaxf(fmaxf(red[16], red[17]), fmaxf(red[18], red[19]));
+                if (pv_valid) store_piece_state(p, tmem, row, pv_final, pv_cta_end, pv_b, pv_h, pv_out);
+                hb = load_piece_state(p, tmem, row, red, abort_flag, b, h, c_begin, sigma);
                 U = 1.f;
             }
             // (c) block scan of a = log2(e) dt A, with the block's max dt and sum dt
@@ -568,13 +604,14 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             }
             wg_sync(1);  // a2s complete; red[] free again
             // (d) scales of this block
-            float need = fmaxf(fmaxf(hb, 16129.f * static_cast<float>(p.N) * dmax),
-                               fabsf(D_h) / (sCg * sBg)) * (1.f / kF16Range);
+            float need = fmaxf(fmaxf(hb, 16129.f * static_cast<float>(p.N) * dmax), d_bound) *
+                         (1.f / kF16Range);
             if (!(need > 1e-30f) || !isfinite(need)) need = 1.f;
             const float rho = pow2_ceil(sCg * sigma * need);
-            const float kappa = rho / (sCg * sigma);
-            const float invk = 1.f / kappa;
+            const float inv_rho = inv_pow2(rho);
+            const float invk = sCg * sigma * inv_rho;  // 1 / kappa
             const float U_new = dmax > 0.f ? pow2_ceil(127.f * dmax * (1.f / kF16Range)) : U;
+            const float inv_U_new = inv_pow2(U_new);
             const float e_end = ex2f(tot);
             // (f) block tables, B', C' and D (independent of the previous block's state)
             {
@@ -587,10 +624,15 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 }
                 // B row scaled by w_t / U -> B' (two MN blocks of 64 n)
                 wait_phase(bars + kBarFull0 + j, (kb >> 1) & 1, abort_flag, p);
-                const __half2 w2 = __float2half2_rn(d * ex2f(tot - incl) * (1.f / U_new));
+                const __half2 w2 = __float2half2_rn(d * ex2f(tot - incl) * inv_U_new);
+                // all loads ahead of the stores (the compiler cannot reorder them across stores
+                // into the same shared array)
+                uint4 wb[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) wb[q] = *reinterpret_cast<const uint4*>(stage + kStB + sw128(row, 16 * q));
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
-                    const uint4 w = *reinterpret_cast<const uint4*>(stage + kStB + sw128(row, 16 * q));
+                    const uint4 w = wb[q];
                     uint4 o0, o1;
                     i8x4_to_h2x2(w.x, o0.x, o0.y);
                     i8x4_to_h2x2(w.y, o0.z, o0.w);
@@ -608,12 +650,15 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 if (kb >= 1) wait_phase(bars + kBarCh, (kb - 1) & 1, abort_flag, p);
                 tc_fence_after();
                 const __half2 f2h = __float2half2_rn(ex2f(incl));
+                uint4 wc[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) wc[q] = *reinterpret_cast<const uint4*>(stage + kStC + sw128(row, 16 * q));
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     uint32_t r[32];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const uint4 w = *reinterpret_cast<const uint4*>(stage + kStC + sw128(row, 16 * (4 * hh + q)));
+                        const uint4 w = wc[4 * hh + q];
                         i8x4_to_h2x2(w.x, r[8 * q + 0], r[8 * q + 1]);
                         i8x4_to_h2x2(w.y, r[8 * q + 2], r[8 * q + 3]);
                         i8x4_to_h2x2(w.z, r[8 * q + 4], r[8 * q + 5]);
@@ -625,7 +670,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 }
                 if (row < kP)
                     *reinterpret_cast<__half*>(smem + kOffDm + sw128(row, 2 * row)) =
-                        __float2half_rn(D_h * sx / rho);
+                        __float2half_rn(D_h * sx * inv_rho);
                 if (row == 0) {
                     BlockInfo bi;
                     bi.rho = rho;
@@ -651,13 +696,15 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             tc_fence_after();
             {
                 const f2 to_hp = {U * invk, U * invk};
-                const float th = e_end * (U / U_new);
+                const float th = e_end * (U * inv_U_new);
                 const f2 to_h = {th, th};
+                uint32_t hv2[2][32];
+                tmem_ld32(tmem_addr(tmem, lane_base, kColH), hv2[0]);
+                tmem_ld32(tmem_addr(tmem, lane_base, kColH + 32), hv2[1]);
+                tmem_ld_wait();
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t hv[32];
-                    tmem_ld32(tmem_addr(tmem, lane_base, kColH + 32 * hh), hv);
-                    tmem_ld_wait();
+                    uint32_t (&hv)[32] = hv2[hh];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         uint32_t w[4];
@@ -709,7 +756,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
         if (pv_valid) {
             wait_phase(bars + kBarState, (nb_total - 1) & 1, abort_flag, p);
             tc_fence_after();
-            store_piece();
+            store_piece_state(p, tmem, row, pv_final, pv_cta_end, pv_b, pv_h, pv_out);
         }
     } else {
         // ============================== x, M' and output warpgroup ==============================
@@ -786,11 +833,17 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             const uint32_t col_cb = kColCB + 128u * j;
             // ---- x -> f16: a quarter row (16 tokens' bytes) per thread and step ----
             wait_phase(bars + kBarFull0 + j, (kb >> 1) & 1, abort_flag, p);
+            uint4 wx[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int idx = lt + 128 * i;
+                wx[i] = *reinterpret_cast<const uint4*>(stage + kStX + (idx >> 2) * 64 + 16 * (idx & 3));
+            }
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int idx = lt + 128 * i;
                 const int r = idx >> 2, c4 = idx & 3;
-                const uint4 w = *reinterpret_cast<const uint4*>(stage + kStX + r * 64 + 16 * c4);
+                const uint4 w = wx[i];
                 uint4 o0, o1;
                 i8x4_to_h2x2(w.x, o0.x, o0.y);
                 i8x4_to_h2x2(w.y, o0.z, o0.w);
@@ -817,38 +870,43 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 const float rowf = quad > 0 ? ex2f(a2t - a2s[32 * quad]) : 0.f;
                 const f2 rowf2 = {rowf, rowf};
                 const float* cfq = colf + colf_off(quad);
-                for (int sc = 0; sc < 4; ++sc) {
-                    uint32_t o[16];
-                    if (sc < quad) {
-                        // 2^(a_t - a_s) = 2^(a_t - a_32q) * 2^(a_32q - a_s), both factors <= 1
-                        uint32_t cbv[32];
-                        tmem_ld32(tmem_addr(tmem, lane_base, col_cb + 32 * sc), cbv);
-                        tmem_ld_wait();
-                        const float2* cf = reinterpret_cast<const float2*>(cfq + 32 * sc);
+                // off the diagonal: 2^(a_t - a_s) = 2^(a_t - a_32q) * 2^(a_32q - a_s), both <= 1
+#pragma unroll 1
+                for (int sc = 0; sc < quad; ++sc) {
+                    uint32_t cbv[32], o[16];
+                    tmem_ld32(tmem_addr(tmem, lane_base, col_cb + 32 * sc), cbv);
+                    tmem_ld_wait();
+                    const float2* cf = reinterpret_cast<const float2*>(cfq + 32 * sc);
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const float2 c2 = cf[e];
-                            const f2 v = fmul2(fmul2(cb_pair(cbv[2 * e], cbv[2 * e + 1]), f2{c2.x, c2.y}), rowf2);
-                            o[e] = pack_f16x2(v.x, v.y);
-                        }
-                    } else if (sc == quad) {
-                        // diagonal sub-block: one exponential per entry, s > t masked
-                        uint32_t cbv[32];
-                        tmem_ld32(tmem_addr(tmem, lane_base, col_cb + 32 * sc), cbv);
-                        tmem_ld_wait();
-                        const float2* nb = reinterpret_cast<const float2*>(nbeta + 32 * sc);
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const float2 n2 = nb[e];
-                            const f2 arg = fadd2(a2t2, f2{n2.x, n2.y});
-                            const f2 v = fmul2(cb_pair(cbv[2 * e], cbv[2 * e + 1]), f2{ex2f(arg.x), ex2f(arg.y)});
-                            o[e] = pack_f16x2(2 * e <= tl ? v.x : 0.f, 2 * e + 1 <= tl ? v.y : 0.f);
-                        }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) o[e] = 0u;
+                    for (int e = 0; e < 16; ++e) {
+                        const float2 c2 = cf[e];
+                        const f2 v = fmul2(fmul2(cb_pair(cbv[2 * e], cbv[2 * e + 1]), f2{c2.x, c2.y}), rowf2);
+                        o[e] = pack_f16x2(v.x, v.y);
                     }
                     tmem_st16(tmem_addr(tmem, lane_base, col_cb + 16 * sc), o);
+                }
+                // diagonal sub-block: one exponential per entry, s > t masked
+                {
+                    uint32_t cbv[32], o[16];
+                    tmem_ld32(tmem_addr(tmem, lane_base, col_cb + 32 * quad), cbv);
+                    tmem_ld_wait();
+                    const float2* nb = reinterpret_cast<const float2*>(nbeta + 32 * quad);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float2 n2 = nb[e];
+                        const f2 arg = fadd2(a2t2, f2{n2.x, n2.y});
+                        const f2 v = fmul2(cb_pair(cbv[2 * e], cbv[2 * e + 1]), f2{ex2f(arg.x), ex2f(arg.y)});
+                        o[e] = pack_f16x2(2 * e <= tl ? v.x : 0.f, 2 * e + 1 <= tl ? v.y : 0.f);
+                    }
+                    tmem_st16(tmem_addr(tmem, lane_base, col_cb + 16 * quad), o);
+                }
+                // above the diagonal: zero
+                {
+                    uint32_t o[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) o[e] = 0u;
+#pragma unroll 1
+                    for (int sc = quad + 1; sc < 4; ++sc) tmem_st16(tmem_addr(tmem, lane_base, col_cb + 16 * sc), o);
                 }
                 tmem_st_wait();
             }
@@ -892,8 +950,7 @@ chunk_cb_tc_kernel(const __grid_constant__ CUtensorMap map_B, const __grid_const
                    int nch, int G, int32_t* __restrict__ cb) {
     constexpr int NTB = Q > kBlk ? Q / kBlk : 1;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* sC = smem;
     uint8_t* sB = smem + Q * 128;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * Q * 128);
