@@ -28,10 +28,11 @@
 // Warp roles, coupled only through mbarriers (buffers alternate with the block parity j):
 //   warp 8      TMA: x, B, C tiles of block k into stage j
 //   warp 9      MMA issue: state(k); C'H'(k) + x D(k); CB(k+1); M'x(k)
-//   warps 0-3   prep: block scan of dt*A, block factors, B' and C' conversions (before the
-//               state of the previous block is needed), then the state hand-over (H', decay)
-//               and piece start / end (initial state, hand-off slot, final state)
-//   warps 4-7   x -> f16, M' from CB(k), output of block k-1 while the tensor core runs block k
+//   warps 0-3   prep: block scan of dt*A, block tables, C' conversion (before the state of
+//               the previous block is needed), then the state hand-over (H', decay) and
+//               piece start / end (initial state, hand-off slot, final state)
+//   warps 4-7   x -> f16 and B' conversions, M' from CB(k), output of block k-1 while the
+//               tensor core runs block k
 // Every wait is bounded; a timeout sets a status word and turns the remaining waits into
 // no-ops so that the kernel still ends (its outputs are then undefined).
 #include <algorithm>
@@ -76,7 +77,8 @@ constexpr int kOffDm = kOffHp + 2 * 16384;      // D s_x / rho on the diagonal o
 constexpr int kOffColf = kOffDm + 8192;         // off-diagonal column factors [2][192] f32
 constexpr int kOffNb = kOffColf + 2 * 768;      // -beta_s = log2(dt_s / kappa) - a_s [2][128]
 constexpr int kOffA2 = kOffNb + 2 * 512;        // a_t [2][128]
-constexpr int kOffInfo = kOffA2 + 2 * 512;      // per-block info [2]
+constexpr int kOffW = kOffA2 + 2 * 512;         // w_t / U = dt_t 2^(a_end - a_t) / U [2][128]
+constexpr int kOffInfo = kOffW + 2 * 512;       // per-block info [2]
 constexpr int kOffRed = kOffInfo + 2 * 32;      // prep scratch [32] f32
 constexpr int kOffBar = kOffRed + 128;          // mbarriers [24]
 constexpr int kOffMisc = kOffBar + 24 * 8;      // TMEM base, abort flag
@@ -87,11 +89,11 @@ static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 enum {
     kBarFull0 = 0, kBarFull1,      // tiles of stage j landed (TMA transaction count)
-    kBarEmpty0, kBarEmpty1,        // stage j consumed: prep + x conversion + ChunkBMM commit
+    kBarEmpty0, kBarEmpty1,        // stage j consumed: C' (prep), x and B' conversion, ChunkBMM
     kBarCb0, kBarCb1,              // CB(k) in TMEM buffer j
-    kBarPa0, kBarPa1,              // block tables, B', C', D of block k ready (prep)
-    kBarPb0, kBarPb1,              // H' written and H decayed for block k (prep)
-    kBarXf0, kBarXf1,              // x f16 of block k ready
+    kBarPa0, kBarPa1,              // block tables of block k ready (prep)
+    kBarPb0, kBarPb1,              // C', D, H' written and H decayed for block k (prep)
+    kBarXb0, kBarXb1,              // x f16 and B' of block k ready
     kBarMp0, kBarMp1,              // M'(k) in TMEM buffer j
     kBarAcc0, kBarAcc1,            // accumulator j complete (M'x(k) done)
     kBarAccFree0, kBarAccFree1,    // accumulator j read out
@@ -247,6 +249,18 @@ __device__ __forceinline__ float pow2_ceil(float v) {
     const uint32_t b = __float_as_uint(v);
     if ((b & 0x007FFFFFu) == 0u && b >= 0x00800000u) return v;
     return __uint_as_float((b & 0x7F800000u) + 0x00800000u);
+}
+
+// Predicated global load issued where it stands (the compiler may not sink it towards its
+// first use): the next block's dt is requested a whole block ahead.
+__device__ __forceinline__ float ldg_early(const float* ptr, bool pred) {
+    float v;
+    asm volatile(
+        "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %2, 0;\n\tmov.b32 %0, 0;\n\t"
+        "@q ld.global.nc.f32 %0, [%1];\n\t}"
+        : "=f"(v)
+        : "l"(ptr), "r"(static_cast<int>(pred)));
+    return v;
 }
 
 // 1 / v for v a power of two in [2^-126, 2^126] (exact)
@@ -486,7 +500,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 const uint64_t hp = d_hp + static_cast<uint64_t>((j * 16384) >> 4);
                 const uint32_t acc = tmem + kColAcc + 64u * j;
                 wait_phase(bars + kBarPb0 + j, (kb >> 1) & 1, abort_flag, p);
-                wait_phase(bars + kBarXf0 + j, (kb >> 1) & 1, abort_flag, p);
+                wait_phase(bars + kBarXb0 + j, (kb >> 1) & 1, abort_flag, p);
                 if (kb >= 2) wait_phase(bars + kBarAccFree0 + j, ((kb >> 1) - 1) & 1, abort_flag, p);
                 tc_fence_after();
                 // state: H += B'^T x   (M = 128 n, N = 64 p, K = 128 t)
@@ -538,7 +552,8 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
         };
         auto dt_at = [&](int bb, int hh, int cc) -> float {
             const int t = cc * kBlk + row;
-            return t < p.L ? p.dt[((size_t)bb * p.L + t) * p.H + hh] : 0.f;
+            const bool in = t < p.L;
+            return ldg_early(p.dt + (in ? ((size_t)bb * p.L + t) * p.H + hh : 0), in);
         };
         if (nb_total > 0) load_piece();
         float d = nb_total > 0 ? dt_at(b, h, c) : 0.f;  // dt of this token, this block
@@ -547,11 +562,11 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
         for (int kb = 0; kb < nb_total; ++kb) {
             const int j = kb & 1;
             uint8_t* stage = smem + j * kStageBytes;
-            uint8_t* bp = smem + kOffBp + j * 32768;
             uint8_t* hp = smem + kOffHp + j * 16384;
             float* colf = reinterpret_cast<float*>(smem + kOffColf) + j * 192;
             float* nbeta = reinterpret_cast<float*>(smem + kOffNb) + j * 128;
             float* a2s = reinterpret_cast<float*>(smem + kOffA2) + j * 128;
+            float* wts = reinterpret_cast<float*>(smem + kOffW) + j * 128;
             const float sigma = sx * sBg;
             const int valid = min(kBlk, p.L - c * kBlk);
             // the next block of this CTA; its dt is in flight during this block
@@ -613,7 +628,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             const float U_new = dmax > 0.f ? pow2_ceil(127.f * dmax * (1.f / kF16Range)) : U;
             const float inv_U_new = inv_pow2(U_new);
             const float e_end = ex2f(tot);
-            // (f) block tables, B', C' and D (independent of the previous block's state)
+            // (f) block tables and C', D (independent of the previous block's state)
             {
                 const float base = d * invk;
                 nbeta[row] = lg2f(base) - incl;  // dt = 0 gives -inf: no contribution
@@ -622,30 +637,23 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                     if (row < 64) colf[colf_off(2) + row] = ex2f(a2s[64] - incl) * base;
                     if (row < 32) colf[colf_off(1) + row] = ex2f(a2s[32] - incl) * base;
                 }
-                // B row scaled by w_t / U -> B' (two MN blocks of 64 n)
-                wait_phase(bars + kBarFull0 + j, (kb >> 1) & 1, abort_flag, p);
-                const __half2 w2 = __float2half2_rn(d * ex2f(tot - incl) * inv_U_new);
-                // all loads ahead of the stores (the compiler cannot reorder them across stores
-                // into the same shared array)
-                uint4 wb[8];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) wb[q] = *reinterpret_cast<const uint4*>(stage + kStB + sw128(row, 16 * q));
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const uint4 w = wb[q];
-                    uint4 o0, o1;
-                    i8x4_to_h2x2(w.x, o0.x, o0.y);
-                    i8x4_to_h2x2(w.y, o0.z, o0.w);
-                    i8x4_to_h2x2(w.z, o1.x, o1.y);
-                    i8x4_to_h2x2(w.w, o1.z, o1.w);
-                    o0.x = hmul2_u32(o0.x, w2); o0.y = hmul2_u32(o0.y, w2);
-                    o0.z = hmul2_u32(o0.z, w2); o0.w = hmul2_u32(o0.w, w2);
-                    o1.x = hmul2_u32(o1.x, w2); o1.y = hmul2_u32(o1.y, w2);
-                    o1.z = hmul2_u32(o1.z, w2); o1.w = hmul2_u32(o1.w, w2);
-                    uint8_t* blk = bp + (q / 4) * 16384;
-                    *reinterpret_cast<uint4*>(blk + sw128(row, 32 * (q % 4))) = o0;
-                    *reinterpret_cast<uint4*>(blk + sw128(row, 32 * (q % 4) + 16)) = o1;
+                wts[row] = d * ex2f(tot - incl) * inv_U_new;
+                if (row == 0) {
+                    BlockInfo bi;
+                    bi.rho = rho;
+                    bi.inv_kappa = invk;
+                    bi.b = b;
+                    bi.h = h;
+                    bi.c = c;
+                    bi.valid = valid;
+                    bi.pad0 = bi.pad1 = 0;
+                    info[j] = bi;
                 }
+            }
+            wg_sync(1);
+            if (row == 0) mbar_arrive(bars + kBarPa0 + j);
+            {
+                wait_phase(bars + kBarFull0 + j, (kb >> 1) & 1, abort_flag, p);
                 // C row scaled by 2^a_t -> C' in TMEM, and D, once the previous C'H' is done
                 if (kb >= 1) wait_phase(bars + kBarCh, (kb - 1) & 1, abort_flag, p);
                 tc_fence_after();
@@ -671,26 +679,9 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 if (row < kP)
                     *reinterpret_cast<__half*>(smem + kOffDm + sw128(row, 2 * row)) =
                         __float2half_rn(D_h * sx * inv_rho);
-                if (row == 0) {
-                    BlockInfo bi;
-                    bi.rho = rho;
-                    bi.inv_kappa = invk;
-                    bi.b = b;
-                    bi.h = h;
-                    bi.c = c;
-                    bi.valid = valid;
-                    bi.pad0 = bi.pad1 = 0;
-                    info[j] = bi;
-                }
             }
-            fence_proxy_async_smem();
-            tmem_st_wait();
-            tc_fence_before();
-            wg_sync(1);
-            if (row == 0) {
-                mbar_arrive(bars + kBarEmpty0 + j);
-                mbar_arrive(bars + kBarPa0 + j);
-            }
+            wg_sync(1);  // every prep thread is done with the stage
+            if (row == 0) mbar_arrive(bars + kBarEmpty0 + j);
             // (e) state hand-over: H' = H U / kappa (f16) for C'H', then decay + rescale
             if (!state_ready) wait_phase(bars + kBarState, (kb - 1) & 1, abort_flag, p);
             tc_fence_after();
@@ -852,15 +843,42 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 *reinterpret_cast<uint4*>(xf + sw128(r, 32 * c4)) = o0;
                 *reinterpret_cast<uint4*>(xf + sw128(r, 32 * c4 + 16)) = o1;
             }
+            // ---- B row scaled by w_t / U -> B' (two MN blocks of 64 n), once the tables exist ----
+            wait_phase(bars + kBarPa0 + j, (kb >> 1) & 1, abort_flag, p);
+            const BlockInfo bi = info[j];
+            {
+                uint8_t* bp = smem + kOffBp + j * 32768;
+                const float* wts = reinterpret_cast<const float*>(smem + kOffW) + j * 128;
+                // all loads ahead of the stores (the compiler cannot reorder them across stores
+                // into the same shared array)
+                uint4 wb[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) wb[q] = *reinterpret_cast<const uint4*>(stage + kStB + sw128(row, 16 * q));
+                const __half2 w2 = __float2half2_rn(wts[row]);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const uint4 w = wb[q];
+                    uint4 o0, o1;
+                    i8x4_to_h2x2(w.x, o0.x, o0.y);
+                    i8x4_to_h2x2(w.y, o0.z, o0.w);
+                    i8x4_to_h2x2(w.z, o1.x, o1.y);
+                    i8x4_to_h2x2(w.w, o1.z, o1.w);
+                    o0.x = hmul2_u32(o0.x, w2); o0.y = hmul2_u32(o0.y, w2);
+                    o0.z = hmul2_u32(o0.z, w2); o0.w = hmul2_u32(o0.w, w2);
+                    o1.x = hmul2_u32(o1.x, w2); o1.y = hmul2_u32(o1.y, w2);
+                    o1.z = hmul2_u32(o1.z, w2); o1.w = hmul2_u32(o1.w, w2);
+                    uint8_t* blk = bp + (q / 4) * 16384;
+                    *reinterpret_cast<uint4*>(blk + sw128(row, 32 * (q % 4))) = o0;
+                    *reinterpret_cast<uint4*>(blk + sw128(row, 32 * (q % 4) + 16)) = o1;
+                }
+            }
             fence_proxy_async_smem();
             wg_sync(2);
             if (lt == 0) {
-                mbar_arrive(bars + kBarXf0 + j);
+                mbar_arrive(bars + kBarXb0 + j);
                 mbar_arrive(bars + kBarEmpty0 + j);
             }
             // ---- M' in place over CB, one 32-column chunk at a time (increasing order) ----
-            wait_phase(bars + kBarPa0 + j, (kb >> 1) & 1, abort_flag, p);
-            const BlockInfo bi = info[j];
             wait_phase(bars + kBarCb0 + j, (kb >> 1) & 1, abort_flag, p);
             tc_fence_after();
             {
