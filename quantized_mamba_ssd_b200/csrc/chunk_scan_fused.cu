@@ -215,6 +215,22 @@ __device__ __forceinline__ void i8x4_to_h2x2(uint32_t w, uint32_t& lo, uint32_t&
     hi = *reinterpret_cast<uint32_t*>(&hb);
 }
 
+// 16 int8 (one 16-byte chunk) -> 16 f16, optionally times a common f16 factor
+__device__ __forceinline__ void cvt16(const uint4 w, uint4& o0, uint4& o1) {
+    i8x4_to_h2x2(w.x, o0.x, o0.y);
+    i8x4_to_h2x2(w.y, o0.z, o0.w);
+    i8x4_to_h2x2(w.z, o1.x, o1.y);
+    i8x4_to_h2x2(w.w, o1.z, o1.w);
+}
+
+__device__ __forceinline__ void cvt16_scaled(const uint4 w, __half2 s, uint4& o0, uint4& o1) {
+    cvt16(w, o0, o1);
+    o0.x = hmul2_u32(o0.x, s); o0.y = hmul2_u32(o0.y, s);
+    o0.z = hmul2_u32(o0.z, s); o0.w = hmul2_u32(o0.w, s);
+    o1.x = hmul2_u32(o1.x, s); o1.y = hmul2_u32(o1.y, s);
+    o1.z = hmul2_u32(o1.z, s); o1.w = hmul2_u32(o1.w, s);
+}
+
 // two ChunkBMM entries (int32, |v| < 2^22) -> exact fp32 pair
 __device__ __forceinline__ f2 cb_pair(uint32_t v0, uint32_t v1) {
     const f2 biased = {__uint_as_float(v0 + kRoundBits), __uint_as_float(v1 + kRoundBits)};
@@ -237,6 +253,12 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
         "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
         "r"(r[15])
         : "memory");
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint4& a, const uint4& b) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+                 "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+                 : "memory");
 }
 
 // barrier among the 128 threads of one warpgroup (id 1: prep, id 2: M' / output)
@@ -658,23 +680,17 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 if (kb >= 1) wait_phase(bars + kBarCh, (kb - 1) & 1, abort_flag, p);
                 tc_fence_after();
                 const __half2 f2h = __float2half2_rn(ex2f(incl));
-                uint4 wc[8];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) wc[q] = *reinterpret_cast<const uint4*>(stage + kStC + sw128(row, 16 * q));
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t r[32];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint4 w = wc[4 * hh + q];
-                        i8x4_to_h2x2(w.x, r[8 * q + 0], r[8 * q + 1]);
-                        i8x4_to_h2x2(w.y, r[8 * q + 2], r[8 * q + 3]);
-                        i8x4_to_h2x2(w.z, r[8 * q + 4], r[8 * q + 5]);
-                        i8x4_to_h2x2(w.w, r[8 * q + 6], r[8 * q + 7]);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) r[8 * q + i] = hmul2_u32(r[8 * q + i], f2h);
-                    }
-                    tmem_st32(tmem_addr(tmem, lane_base, kColC + 32 * hh), r);
+                // compact loop (the kernel is limited by instruction fetch): one 16-byte chunk
+                // per step, the next one already loading
+                uint4 w = *reinterpret_cast<const uint4*>(stage + kStC + sw128(row, 0));
+#pragma unroll 1
+                for (int q = 0; q < 8; ++q) {
+                    uint4 nw = w;
+                    if (q < 7) nw = *reinterpret_cast<const uint4*>(stage + kStC + sw128(row, 16 * (q + 1)));
+                    uint4 o0, o1;
+                    cvt16_scaled(w, f2h, o0, o1);
+                    tmem_st8(tmem_addr(tmem, lane_base, kColC + 8 * q), o0, o1);
+                    w = nw;
                 }
                 if (row < kP)
                     *reinterpret_cast<__half*>(smem + kOffDm + sw128(row, 2 * row)) =
@@ -689,13 +705,11 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 const f2 to_hp = {U * invk, U * invk};
                 const float th = e_end * (U * inv_U_new);
                 const f2 to_h = {th, th};
-                uint32_t hv2[2][32];
-                tmem_ld32(tmem_addr(tmem, lane_base, kColH), hv2[0]);
-                tmem_ld32(tmem_addr(tmem, lane_base, kColH + 32), hv2[1]);
-                tmem_ld_wait();
-#pragma unroll
+#pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t (&hv)[32] = hv2[hh];
+                    uint32_t hv[32];
+                    tmem_ld32(tmem_addr(tmem, lane_base, kColH + 32 * hh), hv);
+                    tmem_ld_wait();
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         uint32_t w[4];
@@ -761,58 +775,58 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
         auto output = [&](int kb) {
             wait_phase(bars + kBarAcc0 + pv_j, (kb >> 1) & 1, abort_flag, p);
             tc_fence_after();
-            uint32_t r[2][32];
-            tmem_ld32(tmem_addr(tmem, lane_base, kColAcc + 64 * pv_j), r[0]);
-            tmem_ld32(tmem_addr(tmem, lane_base, kColAcc + 64 * pv_j + 32), r[1]);
-            tmem_ld_wait();
-            tc_fence_before();
-            wg_sync(2);
-            if (lt == 0) mbar_arrive(bars + kBarAccFree0 + pv_j);
-            if (row < pv_valid) {
-                const size_t ybase = (((size_t)pv_b * p.L + (size_t)pv_c * kBlk + row) * p.H + pv_h) * kP;
+            const size_t ybase = (((size_t)pv_b * p.L + (size_t)pv_c * kBlk + row) * p.H + pv_h) * kP;
+            const bool store = row < pv_valid;
+            // two halves of 32 columns: a compact loop (the kernel is instruction-fetch bound)
+#pragma unroll 1
+            for (int hq = 0; hq < 2; ++hq) {
+                uint32_t r[32];
+                tmem_ld32(tmem_addr(tmem, lane_base, kColAcc + 64 * pv_j + 32 * hq), r);
+                tmem_ld_wait();
+                if (!store) continue;
                 if constexpr (YT == SSD_OUT_I8) {
                     // q = clamp(rint(fp32(acc * rho / s_y))): the same rounding as the fp32 output
-                    const float s = pv_rho * p.inv_y_scale;
-                    const f2 s2 = {s, s}, rnd = {kRound, kRound};
-                    uint32_t wv[16];
+                    const float sc = pv_rho * p.inv_y_scale;
+                    const f2 s2 = {sc, sc}, rnd = {kRound, kRound};
+                    uint32_t wv[8];
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const uint32_t* rr = &r[q / 8][(q % 8) * 4];
-                        const f2 v0 = fadd2(fmul2(f2{__uint_as_float(rr[0]), __uint_as_float(rr[1])}, s2), rnd);
-                        const f2 v1 = fadd2(fmul2(f2{__uint_as_float(rr[2]), __uint_as_float(rr[3])}, s2), rnd);
+                    for (int q = 0; q < 8; ++q) {
+                        const f2 v0 = fadd2(fmul2(f2{__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1])}, s2), rnd);
+                        const f2 v1 = fadd2(fmul2(f2{__uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])}, s2), rnd);
                         const uint32_t lo = __byte_perm(clamp_code(v0.x), clamp_code(v0.y), 0x0040);
                         const uint32_t hi = __byte_perm(clamp_code(v1.x), clamp_code(v1.y), 0x0040);
                         wv[q] = __byte_perm(lo, hi, 0x5410);
                     }
-                    uint4* yo = reinterpret_cast<uint4*>(static_cast<int8_t*>(p.y) + ybase);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) yo[q] = make_uint4(wv[4 * q], wv[4 * q + 1], wv[4 * q + 2], wv[4 * q + 3]);
+                    uint4* yo = reinterpret_cast<uint4*>(static_cast<int8_t*>(p.y) + ybase) + 2 * hq;
+                    yo[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                    yo[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
                 } else if constexpr (YT == SSD_OUT_F16) {
                     const f2 s2 = {pv_rho, pv_rho};
-                    uint4* yo = reinterpret_cast<uint4*>(static_cast<__half*>(p.y) + ybase);
+                    uint4* yo = reinterpret_cast<uint4*>(static_cast<__half*>(p.y) + ybase) + 4 * hq;
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const uint32_t* rr = &r[q / 4][(q % 4) * 8];
+                    for (int q = 0; q < 4; ++q) {
                         uint32_t w[4];
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
-                            const f2 v = fmul2(f2{__uint_as_float(rr[2 * i]), __uint_as_float(rr[2 * i + 1])}, s2);
+                            const f2 v = fmul2(f2{__uint_as_float(r[8 * q + 2 * i]), __uint_as_float(r[8 * q + 2 * i + 1])}, s2);
                             w[i] = pack_f16x2(v.x, v.y);
                         }
                         yo[q] = make_uint4(w[0], w[1], w[2], w[3]);
                     }
                 } else {
                     const f2 s2 = {pv_rho, pv_rho};
-                    float4* yo = reinterpret_cast<float4*>(static_cast<float*>(p.y) + ybase);
+                    float4* yo = reinterpret_cast<float4*>(static_cast<float*>(p.y) + ybase) + 8 * hq;
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const uint32_t* rr = &r[q / 8][(q % 8) * 4];
-                        const f2 v0 = fmul2(f2{__uint_as_float(rr[0]), __uint_as_float(rr[1])}, s2);
-                        const f2 v1 = fmul2(f2{__uint_as_float(rr[2]), __uint_as_float(rr[3])}, s2);
+                    for (int q = 0; q < 8; ++q) {
+                        const f2 v0 = fmul2(f2{__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1])}, s2);
+                        const f2 v1 = fmul2(f2{__uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])}, s2);
                         yo[q] = make_float4(v0.x, v0.y, v1.x, v1.y);
                     }
                 }
             }
+            tc_fence_before();
+            wg_sync(2);
+            if (lt == 0) mbar_arrive(bars + kBarAccFree0 + pv_j);
         };
         for (int kb = 0; kb < nb_total; ++kb) {
             const int j = kb & 1;
@@ -824,24 +838,23 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             const uint32_t col_cb = kColCB + 128u * j;
             // ---- x -> f16: a quarter row (16 tokens' bytes) per thread and step ----
             wait_phase(bars + kBarFull0 + j, (kb >> 1) & 1, abort_flag, p);
-            uint4 wx[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int idx = lt + 128 * i;
-                wx[i] = *reinterpret_cast<const uint4*>(stage + kStX + (idx >> 2) * 64 + 16 * (idx & 3));
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int idx = lt + 128 * i;
-                const int r = idx >> 2, c4 = idx & 3;
-                const uint4 w = wx[i];
-                uint4 o0, o1;
-                i8x4_to_h2x2(w.x, o0.x, o0.y);
-                i8x4_to_h2x2(w.y, o0.z, o0.w);
-                i8x4_to_h2x2(w.z, o1.x, o1.y);
-                i8x4_to_h2x2(w.w, o1.z, o1.w);
-                *reinterpret_cast<uint4*>(xf + sw128(r, 32 * c4)) = o0;
-                *reinterpret_cast<uint4*>(xf + sw128(r, 32 * c4 + 16)) = o1;
+            {
+                uint4 w = *reinterpret_cast<const uint4*>(stage + kStX + (lt >> 2) * 64 + 16 * (lt & 3));
+#pragma unroll 1
+                for (int i = 0; i < 4; ++i) {
+                    const int idx = lt + 128 * i;
+                    uint4 nw = w;
+                    if (i < 3) {
+                        const int n = idx + 128;
+                        nw = *reinterpret_cast<const uint4*>(stage + kStX + (n >> 2) * 64 + 16 * (n & 3));
+                    }
+                    uint4 o0, o1;
+                    cvt16(w, o0, o1);
+                    const int r = idx >> 2, c4 = idx & 3;
+                    *reinterpret_cast<uint4*>(xf + sw128(r, 32 * c4)) = o0;
+                    *reinterpret_cast<uint4*>(xf + sw128(r, 32 * c4 + 16)) = o1;
+                    w = nw;
+                }
             }
             // ---- B row scaled by w_t / U -> B' (two MN blocks of 64 n), once the tables exist ----
             wait_phase(bars + kBarPa0 + j, (kb >> 1) & 1, abort_flag, p);
@@ -849,27 +862,18 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             {
                 uint8_t* bp = smem + kOffBp + j * 32768;
                 const float* wts = reinterpret_cast<const float*>(smem + kOffW) + j * 128;
-                // all loads ahead of the stores (the compiler cannot reorder them across stores
-                // into the same shared array)
-                uint4 wb[8];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) wb[q] = *reinterpret_cast<const uint4*>(stage + kStB + sw128(row, 16 * q));
                 const __half2 w2 = __float2half2_rn(wts[row]);
-#pragma unroll
+                uint4 w = *reinterpret_cast<const uint4*>(stage + kStB + sw128(row, 0));
+#pragma unroll 1
                 for (int q = 0; q < 8; ++q) {
-                    const uint4 w = wb[q];
+                    uint4 nw = w;
+                    if (q < 7) nw = *reinterpret_cast<const uint4*>(stage + kStB + sw128(row, 16 * (q + 1)));
                     uint4 o0, o1;
-                    i8x4_to_h2x2(w.x, o0.x, o0.y);
-                    i8x4_to_h2x2(w.y, o0.z, o0.w);
-                    i8x4_to_h2x2(w.z, o1.x, o1.y);
-                    i8x4_to_h2x2(w.w, o1.z, o1.w);
-                    o0.x = hmul2_u32(o0.x, w2); o0.y = hmul2_u32(o0.y, w2);
-                    o0.z = hmul2_u32(o0.z, w2); o0.w = hmul2_u32(o0.w, w2);
-                    o1.x = hmul2_u32(o1.x, w2); o1.y = hmul2_u32(o1.y, w2);
-                    o1.z = hmul2_u32(o1.z, w2); o1.w = hmul2_u32(o1.w, w2);
-                    uint8_t* blk = bp + (q / 4) * 16384;
-                    *reinterpret_cast<uint4*>(blk + sw128(row, 32 * (q % 4))) = o0;
-                    *reinterpret_cast<uint4*>(blk + sw128(row, 32 * (q % 4) + 16)) = o1;
+                    cvt16_scaled(w, w2, o0, o1);
+                    uint8_t* blk = bp + (q >> 2) * 16384;
+                    *reinterpret_cast<uint4*>(blk + sw128(row, 32 * (q & 3))) = o0;
+                    *reinterpret_cast<uint4*>(blk + sw128(row, 32 * (q & 3) + 16)) = o1;
+                    w = nw;
                 }
             }
             fence_proxy_async_smem();
