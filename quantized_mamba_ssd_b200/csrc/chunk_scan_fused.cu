@@ -266,11 +266,10 @@ __device__ __forceinline__ void wg_sync(int id) {
     asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
 }
 
-// smallest power of two >= v (v > 0); exact for normal and subnormal v
+// smallest power of two >= v, for v a positive normal float (rounds the bits up to a whole
+// exponent)
 __device__ __forceinline__ float pow2_ceil(float v) {
-    const uint32_t b = __float_as_uint(v);
-    if ((b & 0x007FFFFFu) == 0u && b >= 0x00800000u) return v;
-    return __uint_as_float((b & 0x7F800000u) + 0x00800000u);
+    return __uint_as_float((__float_as_uint(v) + 0x007FFFFFu) & 0xFF800000u);
 }
 
 // Predicated global load issued where it stands (the compiler may not sink it towards its
@@ -611,40 +610,37 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 hb = load_piece_state(p, tmem, row, red, abort_flag, b, h, c_begin, sigma);
                 U = 1.f;
             }
-            // (c) block scan of a = log2(e) dt A, with the block's max dt and sum dt
+            // (c) block scan of dt (a_t = log2(e) A cumsum(dt)), with the block's max and sum
             float incl, tot, dmax, dsum;
             {
-                float v = d * A2h, mx = d, sm = d;
+                float v = d, mx = d;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
                     const float u = __shfl_up_sync(0xffffffffu, v, o);
                     if (lane >= o) v += u;
                 }
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                    sm += __shfl_xor_sync(0xffffffffu, sm, o);
-                }
+                for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
                 if (lane == 31) red[warp] = v;
-                if (lane == 0) {
-                    red[4 + warp] = mx;
-                    red[8 + warp] = sm;
-                }
+                if (lane == 0) red[4 + warp] = mx;
                 wg_sync(1);
-                float pre = 0.f;
-                for (int w = 0; w < warp; ++w) pre += red[w];
-                incl = v + pre;
-                tot = ((red[0] + red[1]) + red[2]) + red[3];
-                dmax = fmaxf(fmaxf(red[4], red[5]), fmaxf(red[6], red[7]));
-                dsum = (red[8] + red[9]) + (red[10] + red[11]);
+                const float4 ws = *reinterpret_cast<const float4*>(red);
+                const float4 wm = *reinterpret_cast<const float4*>(red + 4);
+                // prefix over warps in a fixed order, so that row 127 carries exactly dsum
+                const float p1 = ws.x, p2 = p1 + ws.y, p3 = p2 + ws.z;
+                const float pre = warp == 0 ? 0.f : (warp == 1 ? p1 : (warp == 2 ? p2 : p3));
+                dsum = p3 + ws.w;
+                dmax = fmaxf(fmaxf(wm.x, wm.y), fmaxf(wm.z, wm.w));
+                incl = A2h * (v + pre);
+                tot = A2h * dsum;
                 a2s[row] = incl;
             }
             wg_sync(1);  // a2s complete; red[] free again
             // (d) scales of this block
             float need = fmaxf(fmaxf(hb, 16129.f * static_cast<float>(p.N) * dmax), d_bound) *
                          (1.f / kF16Range);
-            if (!(need > 1e-30f) || !isfinite(need)) need = 1.f;
-            const float rho = pow2_ceil(sCg * sigma * need);
+            need = (need > 1e-30f && need < 1e30f) ? need : 1.f;  // also catches NaN / inf
+            const float rho = pow2_ceil(fmaxf(sCg * sigma * need, 1e-30f));
             const float inv_rho = inv_pow2(rho);
             const float invk = sCg * sigma * inv_rho;  // 1 / kappa
             const float U_new = dmax > 0.f ? pow2_ceil(127.f * dmax * (1.f / kF16Range)) : U;
