@@ -27,12 +27,13 @@
 //
 // Warp roles, coupled only through mbarriers (buffers alternate with the block parity j):
 //   warp 8      TMA: x, B, C tiles of block k into stage j
-//   warp 9      MMA issue: state(k); C'H'(k) + x D(k); CB(k+1); M'x(k)
-//   warps 0-3   prep: block scan of dt*A, block tables, C' conversion (before the state of
-//               the previous block is needed), then the state hand-over (H', decay) and
-//               piece start / end (initial state, hand-off slot, final state)
-//   warps 4-7   x -> f16 and B' conversions, M' from CB(k), output of block k-1 while the
-//               tensor core runs block k
+//   warp 9      MMA issue: CB(k+1); M'x(k); state(k); C'H'(k) + x D(k)
+//   warps 0-3   block worker for even blocks, warps 4-7 for odd blocks: both run the same
+//               compact loop (the kernel is limited by instruction fetch, and two warps on an
+//               SM sub-partition that run the same code share it): output of the worker's
+//               previous block, block scan of dt, block statistics chained through the
+//               workers (bound on |H|, state unit), x and B' conversions, M' from CB(k), then
+//               the serial part, the state hand-over (H', decay) and C', D.
 // Every wait is bounded; a timeout sets a status word and turns the remaining waits into
 // no-ops so that the kernel still ends (its outputs are then undefined).
 #include <algorithm>
@@ -77,11 +78,10 @@ constexpr int kOffDm = kOffHp + 2 * 16384;      // D s_x / rho on the diagonal o
 constexpr int kOffColf = kOffDm + 8192;         // off-diagonal column factors [2][192] f32
 constexpr int kOffNb = kOffColf + 2 * 768;      // -beta_s = log2(dt_s / kappa) - a_s [2][128]
 constexpr int kOffA2 = kOffNb + 2 * 512;        // a_t [2][128]
-constexpr int kOffW = kOffA2 + 2 * 512;         // w_t / U = dt_t 2^(a_end - a_t) / U [2][128]
-constexpr int kOffInfo = kOffW + 2 * 512;       // per-block info [2]
-constexpr int kOffRed = kOffInfo + 2 * 32;      // prep scratch [32] f32
-constexpr int kOffBar = kOffRed + 128;          // mbarriers [24]
-constexpr int kOffMisc = kOffBar + 24 * 8;      // TMEM base, abort flag
+constexpr int kOffStats = kOffA2 + 2 * 512;     // per-block statistics handed between workers [2]
+constexpr int kOffRed = kOffStats + 2 * 16;     // worker scratch [2][16] f32
+constexpr int kOffBar = kOffRed + 2 * 64;       // mbarriers [32]
+constexpr int kOffMisc = kOffBar + 32 * 8;      // TMEM base, abort flag
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
 static_assert(kOffXf % 1024 == 0 && kOffBp % 1024 == 0 && kOffHp % 1024 == 0 &&
                   kOffDm % 1024 == 0, "alignment");
@@ -89,24 +89,22 @@ static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 enum {
     kBarFull0 = 0, kBarFull1,      // tiles of stage j landed (TMA transaction count)
-    kBarEmpty0, kBarEmpty1,        // stage j consumed: C' (prep), x and B' conversion, ChunkBMM
+    kBarEmpty0, kBarEmpty1,        // stage j consumed: worker conversions + ChunkBMM commit
     kBarCb0, kBarCb1,              // CB(k) in TMEM buffer j
-    kBarPa0, kBarPa1,              // block tables of block k ready (prep)
-    kBarPb0, kBarPb1,              // C', D, H' written and H decayed for block k (prep)
+    kBarSt0, kBarSt1,              // statistics of block k published (worker j)
     kBarXb0, kBarXb1,              // x f16 and B' of block k ready
     kBarMp0, kBarMp1,              // M'(k) in TMEM buffer j
-    kBarAcc0, kBarAcc1,            // accumulator j complete (M'x(k) done)
+    kBarPh0, kBarPh1,              // H' written and H decayed for block k
+    kBarPc0, kBarPc1,              // C' and D of block k written
+    kBarMx0, kBarMx1,              // M'x(k) done (CB buffer j free)
+    kBarAcc0, kBarAcc1,            // accumulator j complete
     kBarAccFree0, kBarAccFree1,    // accumulator j read out
     kBarState,                     // state update of the last issued block done
     kBarCh,                        // C'H' + xD of the last issued block done (C', D free)
     kNumBars
 };
-static_assert(kNumBars <= 24, "barrier space");
+static_assert(kNumBars <= 32, "barrier space");
 
-struct BlockInfo {  // handed from the prep warpgroup to the M' / output warpgroup
-    float rho, inv_kappa;
-    int b, h, c, valid, pad0, pad1;
-};
 
 struct FusedParams {
     const float* dt;
@@ -149,6 +147,26 @@ struct Range {
         c_end = static_cast<int>(u == u_last ? we - u * nblk : nblk);
         b = static_cast<int>(u / H);
         h = static_cast<int>(u % H);
+    }
+};
+
+// position of a block in this CTA's processing order
+struct Cursor {
+    int seg, b, h, cb, ce, c;
+    __device__ void init(const Range& rg) {
+        seg = 0;
+        b = h = cb = ce = c = 0;
+        if (rg.nseg > 0) {
+            rg.seg(0, b, h, cb, ce);
+            c = cb;
+        }
+    }
+    __device__ void advance(const Range& rg) {
+        if (++c >= ce && seg + 1 < rg.nseg) {
+            ++seg;
+            rg.seg(seg, b, h, cb, ce);
+            c = cb;
+        }
     }
 };
 
@@ -261,7 +279,7 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint4& a, const u
                  : "memory");
 }
 
-// barrier among the 128 threads of one warpgroup (id 1: prep, id 2: M' / output)
+// barrier among the 128 threads of one worker warpgroup (id 1: even blocks, id 2: odd blocks)
 __device__ __forceinline__ void wg_sync(int id) {
     asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
 }
@@ -325,13 +343,13 @@ __device__ __forceinline__ void issue_cb(uint32_t d, uint32_t sC, uint32_t sB, i
     for (int k = 0; k < 4; ++k) mma_i8_ss(d, a0 + 2 * k, b0 + 2 * k, id, k > 0);
 }
 
-// Piece end (prep warpgroup, thread = state row n): writes the state of the finished piece,
+// Piece end (worker warpgroup, thread = state row n): writes the state of the finished piece,
 // either as the caller's final state or into this CTA's hand-off slot (then publishes the slot).
 // `out_scale` converts TMEM units to units of s_x s_B.  Kept out of line: it runs once or twice
 // per CTA.
 __device__ __noinline__ void store_piece_state(const FusedParams& p, uint32_t tmem, int row,
                                                bool final_piece, bool cta_end, int b, int h,
-                                               float out_scale) {
+                                               float out_scale, int bar_id) {
     const uint32_t lane_base = static_cast<uint32_t>(row & ~31);
     uint32_t hv[2][32];
     tmem_ld32(tmem_addr(tmem, lane_base, kColH), hv[0]);
@@ -354,7 +372,7 @@ __device__ __noinline__ void store_piece_state(const FusedParams& p, uint32_t tm
                                  out_scale * __uint_as_float(hv[(4 * q + 2) / 32][(4 * q + 2) % 32]),
                                  out_scale * __uint_as_float(hv[(4 * q + 3) / 32][(4 * q + 3) % 32]));
         __threadfence();
-        wg_sync(1);
+        wg_sync(bar_id);
         if (row == 0 && p.drop_publish != static_cast<int>(blockIdx.x)) {
             unsigned long long* f = p.flags + blockIdx.x;
             asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(f), "l"(p.epoch) : "memory");
@@ -362,13 +380,13 @@ __device__ __noinline__ void store_piece_state(const FusedParams& p, uint32_t tm
     }
 }
 
-// Piece start (prep warpgroup): loads the piece's initial state into TMEM in units of s_x s_B:
+// Piece start (worker warpgroup): loads the piece's initial state into TMEM in units of s_x s_B:
 // the caller's initial state (or zero) at sequence start, else the predecessor CTA's hand-off
 // slot after a bounded wait for its flag.  Returns max |state| over the piece's state.
 __device__ __noinline__ float load_piece_state(const FusedParams& p, uint32_t tmem, int row,
                                                float* red, volatile uint32_t* abort_flag, int b,
-                                               int h, int c_begin, float sigma) {
-    const int warp = row >> 5, lane = row & 31;
+                                               int h, int c_begin, float sigma, int bar_id) {
+    const int warp = row >> 5, lane = row & 31;  // warp within the worker warpgroup
     const uint32_t lane_base = static_cast<uint32_t>(row & ~31);
     const float* src = nullptr;
     bool from_slot = false;
@@ -390,7 +408,7 @@ __device__ __noinline__ float load_piece_state(const FusedParams& p, uint32_t tm
                 __nanosleep(256);
             }
         }
-        wg_sync(1);
+        wg_sync(bar_id);
         src = p.slots + (size_t)(blockIdx.x - 1) * 128 * kP;
         from_slot = true;
     }
@@ -413,9 +431,9 @@ __device__ __noinline__ float load_piece_state(const FusedParams& p, uint32_t tm
     tmem_st_wait();
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (lane == 0) red[16 + warp] = m;
-    wg_sync(1);
-    return fmaxf(fmaxf(red[16], red[17]), fmaxf(red[18], red[19]));
+    if (lane == 0) red[8 + warp] = m;
+    wg_sync(bar_id);
+    return fmaxf(fmaxf(red[8], red[9]), fmaxf(red[10], red[11]));
 }
 
 // start column of quad q's off-diagonal column factors (q = 1, 2, 3 hold 32 q entries)
@@ -434,14 +452,13 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
     uint32_t* misc = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile uint32_t* abort_flag = misc + 1;
-    BlockInfo* info = reinterpret_cast<BlockInfo*>(smem + kOffInfo);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
 
     if (tid == 0) {
         for (int i = 0; i < kNumBars; ++i)
-            mbar_init(bars + i, (i == kBarEmpty0 || i == kBarEmpty1) ? 3 : 1);
+            mbar_init(bars + i, (i == kBarEmpty0 || i == kBarEmpty1) ? 2 : 1);
         fence_mbar_init();
         *abort_flag = 0;
         if (blockIdx.x == 0) p.status[2] = p.epoch;  // the call the status word refers to
@@ -505,7 +522,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 const int j = kb & 1;
                 wait_phase(bars + kBarFull0 + j, (kb >> 1) & 1, abort_flag, p);
                 // CB buffer j held M'(kb - 2), read by M'x(kb - 2)
-                if (kb >= 2) wait_phase(bars + kBarAcc0 + j, ((kb >> 1) - 1) & 1, abort_flag, p);
+                if (kb >= 2) wait_phase(bars + kBarMx0 + j, ((kb >> 1) - 1) & 1, abort_flag, p);
                 tc_fence_after();
                 uint8_t* stage = smem + j * kStageBytes;
                 issue_cb(tmem + kColCB + 128u * j, smem_u32(stage + kStC), smem_u32(stage + kStB),
@@ -516,268 +533,90 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             issue_cb_block(0);
             for (int kb = 0; kb < nb_total && !*abort_flag; ++kb) {  // no new MMA after a failure
                 const int j = kb & 1;
+                const uint32_t ph = (kb >> 1) & 1;
                 const uint64_t bp = d_bp + static_cast<uint64_t>((j * 32768) >> 4);
                 const uint64_t xf = d_xf + static_cast<uint64_t>((j * 16384) >> 4);
                 const uint64_t hp = d_hp + static_cast<uint64_t>((j * 16384) >> 4);
                 const uint32_t acc = tmem + kColAcc + 64u * j;
-                wait_phase(bars + kBarPb0 + j, (kb >> 1) & 1, abort_flag, p);
-                wait_phase(bars + kBarXb0 + j, (kb >> 1) & 1, abort_flag, p);
-                if (kb >= 2) wait_phase(bars + kBarAccFree0 + j, ((kb >> 1) - 1) & 1, abort_flag, p);
+                if (kb + 1 < nb_total) issue_cb_block(kb + 1);
+                // acc = M' x   (A = M' from TMEM, K = 128 s): opens the accumulator
+                wait_phase(bars + kBarMp0 + j, ph, abort_flag, p);
+                wait_phase(bars + kBarXb0 + j, ph, abort_flag, p);
+                if (kb >= 2) wait_phase(bars + kBarAccFree0 + j, ph ^ 1u, abort_flag, p);
                 tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_f16_ts(acc, tmem + kColCB + 128u * j + 8 * kk, xf + 128 * kk, id_y, kk > 0);
+                tc_commit(bars + kBarMx0 + j);
                 // state: H += B'^T x   (M = 128 n, N = 64 p, K = 128 t)
+                wait_phase(bars + kBarPh0 + j, ph, abort_flag, p);
+                tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kBlk / 16; ++kk)
                     mma_f16_ss(tmem + kColH, bp + 128 * kk, xf + 128 * kk, id_st, 1);
                 tc_commit(bars + kBarState);
-                // acc = C' H'^T (A = C' from TMEM, K = 128 n) + x D (K = 64 p)
+                // acc += C' H'^T (A = C' from TMEM, K = 128 n) + x D (K = 64 p)
+                wait_phase(bars + kBarPc0 + j, ph, abort_flag, p);
+                tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_f16_ts(acc, tmem + kColC + 8 * kk, hp + 128 * kk, id_y, kk > 0);
+                    mma_f16_ts(acc, tmem + kColC + 8 * kk, hp + 128 * kk, id_y, 1);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) mma_f16_ss(acc, xf + 2 * kk, d_dm + 2 * kk, id_d, 1);
                 tc_commit(bars + kBarCh);
                 ++n_ch;
-                if (kb + 1 < nb_total) issue_cb_block(kb + 1);
-                // acc += M' x   (A = M' from TMEM, K = 128 s)
-                wait_phase(bars + kBarMp0 + j, (kb >> 1) & 1, abort_flag, p);
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_f16_ts(acc, tmem + kColCB + 128u * j + 8 * kk, xf + 128 * kk, id_y, 1);
                 tc_commit(bars + kBarAcc0 + j);
             }
         }
         __syncwarp();
-    } else if (warp < 4) {
-        // ============================== prep warpgroup ==============================
-        const int row = tid;  // block row t / state row n (TMEM lane)
-        const uint32_t lane_base = static_cast<uint32_t>(warp) * 32u;
-        float* red = reinterpret_cast<float*>(smem + kOffRed);
-        // previous piece, whose state is stored once its last update is done
-        int pv_b = 0, pv_h = 0;
-        bool pv_valid = false, pv_final = false, pv_cta_end = false;
-        float pv_out = 1.f;  // H_true / s_x s_B = pv_out * H_tmem
-        // cursor over this CTA's blocks, and the per-piece constants
-        int seg = 0, b = 0, h = 0, c_begin = 0, c_end = 0;
-        if (rg.nseg > 0) rg.seg(0, b, h, c_begin, c_end);
-        int c = c_begin;
-        float sx = 1.f, sBg = 1.f, sCg = 1.f, A2h = 0.f, D_h = 0.f, d_bound = 0.f;
-        auto load_piece = [&]() {
-            const int g = h / (p.H / p.G);
-            sx = p.x_scale[h];
-            sBg = p.B_scale[g];
-            sCg = p.C_scale[g];
-            A2h = p.A[h] * kLog2e;
-            D_h = p.D[h];
-            d_bound = fabsf(D_h) / (sCg * sBg);  // |D s_x / rho| <= 2^14 needs kappa >= this / 2^14
-        };
-        auto dt_at = [&](int bb, int hh, int cc) -> float {
-            const int t = cc * kBlk + row;
-            const bool in = t < p.L;
-            return ldg_early(p.dt + (in ? ((size_t)bb * p.L + t) * p.H + hh : 0), in);
-        };
-        if (nb_total > 0) load_piece();
-        float d = nb_total > 0 ? dt_at(b, h, c) : 0.f;  // dt of this token, this block
-        float U = 1.f;   // H_true / sigma = U * H_tmem
-        float hb = 0.f;  // running bound on max |H_true| / sigma
-        for (int kb = 0; kb < nb_total; ++kb) {
-            const int j = kb & 1;
-            uint8_t* stage = smem + j * kStageBytes;
-            uint8_t* hp = smem + kOffHp + j * 16384;
-            float* colf = reinterpret_cast<float*>(smem + kOffColf) + j * 192;
-            float* nbeta = reinterpret_cast<float*>(smem + kOffNb) + j * 128;
-            float* a2s = reinterpret_cast<float*>(smem + kOffA2) + j * 128;
-            float* wts = reinterpret_cast<float*>(smem + kOffW) + j * 128;
-            const float sigma = sx * sBg;
-            const int valid = min(kBlk, p.L - c * kBlk);
-            // the next block of this CTA; its dt is in flight during this block
-            int n_seg = seg, n_b = b, n_h = h, n_cb = c_begin, n_ce = c_end, n_c = c + 1;
-            if (n_c >= c_end && seg + 1 < rg.nseg) {
-                n_seg = seg + 1;
-                rg.seg(n_seg, n_b, n_h, n_cb, n_ce);
-                n_c = n_cb;
-            }
-            const float d_next = kb + 1 < nb_total ? dt_at(n_b, n_h, n_c) : 0.f;
-            // (a) the block tables of buffer j are free once M'(k-2) is built
-            if (kb >= 2) wait_phase(bars + kBarMp0 + j, ((kb >> 1) - 1) & 1, abort_flag, p);
-            // (b) piece start: store the previous piece's state, load this piece's
-            bool state_ready = (kb == 0);
-            if (c == c_begin) {
-                if (kb >= 1) wait_phase(bars + kBarState, (kb - 1) & 1, abort_flag, p);
-                tc_fence_after();
-                state_ready = true;
-                if (pv_valid) store_piece_state(p, tmem, row, pv_final, pv_cta_end, pv_b, pv_h, pv_out);
-                hb = load_piece_state(p, tmem, row, red, abort_flag, b, h, c_begin, sigma);
-                U = 1.f;
-            }
-            // (c) block scan of dt (a_t = log2(e) A cumsum(dt)), with the block's max and sum
-            float incl, tot, dmax, dsum;
-            {
-                float v = d, mx = d;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float u = __shfl_up_sync(0xffffffffu, v, o);
-                    if (lane >= o) v += u;
-                }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                if (lane == 31) red[warp] = v;
-                if (lane == 0) red[4 + warp] = mx;
-                wg_sync(1);
-                const float4 ws = *reinterpret_cast<const float4*>(red);
-                const float4 wm = *reinterpret_cast<const float4*>(red + 4);
-                // prefix over warps in a fixed order, so that row 127 carries exactly dsum
-                const float p1 = ws.x, p2 = p1 + ws.y, p3 = p2 + ws.z;
-                const float pre = warp == 0 ? 0.f : (warp == 1 ? p1 : (warp == 2 ? p2 : p3));
-                dsum = p3 + ws.w;
-                dmax = fmaxf(fmaxf(wm.x, wm.y), fmaxf(wm.z, wm.w));
-                incl = A2h * (v + pre);
-                tot = A2h * dsum;
-                a2s[row] = incl;
-            }
-            wg_sync(1);  // a2s complete; red[] free again
-            // (d) scales of this block
-            float need = fmaxf(fmaxf(hb, 16129.f * static_cast<float>(p.N) * dmax), d_bound) *
-                         (1.f / kF16Range);
-            need = (need > 1e-30f && need < 1e30f) ? need : 1.f;  // also catches NaN / inf
-            const float rho = pow2_ceil(fmaxf(sCg * sigma * need, 1e-30f));
-            const float inv_rho = inv_pow2(rho);
-            const float invk = sCg * sigma * inv_rho;  // 1 / kappa
-            const float U_new = dmax > 0.f ? pow2_ceil(127.f * dmax * (1.f / kF16Range)) : U;
-            const float inv_U_new = inv_pow2(U_new);
-            const float e_end = ex2f(tot);
-            // (f) block tables and C', D (independent of the previous block's state)
-            {
-                const float base = d * invk;
-                nbeta[row] = lg2f(base) - incl;  // dt = 0 gives -inf: no contribution
-                if (row < 96) {
-                    colf[colf_off(3) + row] = ex2f(a2s[96] - incl) * base;
-                    if (row < 64) colf[colf_off(2) + row] = ex2f(a2s[64] - incl) * base;
-                    if (row < 32) colf[colf_off(1) + row] = ex2f(a2s[32] - incl) * base;
-                }
-                wts[row] = d * ex2f(tot - incl) * inv_U_new;
-                if (row == 0) {
-                    BlockInfo bi;
-                    bi.rho = rho;
-                    bi.inv_kappa = invk;
-                    bi.b = b;
-                    bi.h = h;
-                    bi.c = c;
-                    bi.valid = valid;
-                    bi.pad0 = bi.pad1 = 0;
-                    info[j] = bi;
-                }
-            }
-            wg_sync(1);
-            if (row == 0) mbar_arrive(bars + kBarPa0 + j);
-            {
-                wait_phase(bars + kBarFull0 + j, (kb >> 1) & 1, abort_flag, p);
-                // C row scaled by 2^a_t -> C' in TMEM, and D, once the previous C'H' is done
-                if (kb >= 1) wait_phase(bars + kBarCh, (kb - 1) & 1, abort_flag, p);
-                tc_fence_after();
-                const __half2 f2h = __float2half2_rn(ex2f(incl));
-                // compact loop (the kernel is limited by instruction fetch): one 16-byte chunk
-                // per step, the next one already loading
-                uint4 w = *reinterpret_cast<const uint4*>(stage + kStC + sw128(row, 0));
-#pragma unroll 1
-                for (int q = 0; q < 8; ++q) {
-                    uint4 nw = w;
-                    if (q < 7) nw = *reinterpret_cast<const uint4*>(stage + kStC + sw128(row, 16 * (q + 1)));
-                    uint4 o0, o1;
-                    cvt16_scaled(w, f2h, o0, o1);
-                    tmem_st8(tmem_addr(tmem, lane_base, kColC + 8 * q), o0, o1);
-                    w = nw;
-                }
-                if (row < kP)
-                    *reinterpret_cast<__half*>(smem + kOffDm + sw128(row, 2 * row)) =
-                        __float2half_rn(D_h * sx * inv_rho);
-            }
-            wg_sync(1);  // every prep thread is done with the stage
-            if (row == 0) mbar_arrive(bars + kBarEmpty0 + j);
-            // (e) state hand-over: H' = H U / kappa (f16) for C'H', then decay + rescale
-            if (!state_ready) wait_phase(bars + kBarState, (kb - 1) & 1, abort_flag, p);
-            tc_fence_after();
-            {
-                const f2 to_hp = {U * invk, U * invk};
-                const float th = e_end * (U * inv_U_new);
-                const f2 to_h = {th, th};
-#pragma unroll 1
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t hv[32];
-                    tmem_ld32(tmem_addr(tmem, lane_base, kColH + 32 * hh), hv);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint32_t w[4];
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const f2 v = fmul2(f2{__uint_as_float(hv[8 * q + 2 * i]),
-                                                  __uint_as_float(hv[8 * q + 2 * i + 1])}, to_hp);
-                            w[i] = pack_f16x2(v.x, v.y);
-                        }
-                        *reinterpret_cast<uint4*>(hp + sw128(row, 64 * hh + 16 * q)) =
-                            make_uint4(w[0], w[1], w[2], w[3]);
-                    }
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const f2 v = fmul2(f2{__uint_as_float(hv[2 * i]), __uint_as_float(hv[2 * i + 1])}, to_h);
-                        hv[2 * i] = __float_as_uint(v.x);
-                        hv[2 * i + 1] = __float_as_uint(v.y);
-                    }
-                    tmem_st32(tmem_addr(tmem, lane_base, kColH + 32 * hh), hv);
-                }
-                U = U_new;
-                hb = hb * e_end + 16129.f * dsum;  // bound after this block's update
-            }
-            fence_proxy_async_smem();
-            tmem_st_wait();
-            tc_fence_before();
-            wg_sync(1);
-            if (row == 0) mbar_arrive(bars + kBarPb0 + j);
-            // piece end: its state is stored when the next piece starts (or below)
-            if (c + 1 == c_end) {
-                pv_valid = true;
-                pv_b = b;
-                pv_h = h;
-                pv_final = (c_end == p.nblk);
-                pv_cta_end = (c_end != p.nblk);
-                pv_out = U;
-            }
-            if (n_seg != seg) {
-                seg = n_seg;
-                b = n_b;
-                h = n_h;
-                c_begin = n_cb;
-                c_end = n_ce;
-                load_piece();
-            }
-            c = n_c;
-            d = d_next;
-        }
-        if (pv_valid) {
-            wait_phase(bars + kBarState, (nb_total - 1) & 1, abort_flag, p);
-            tc_fence_after();
-            store_piece_state(p, tmem, row, pv_final, pv_cta_end, pv_b, pv_h, pv_out);
-        }
     } else {
-        // ============================== x, M' and output warpgroup ==============================
-        const int quad = warp & 3;
-        const int row = quad * 32 + lane;
-        const int lt = tid - 128;
-        const uint32_t lane_base = static_cast<uint32_t>(quad) * 32u;
-        // output of the previous block
-        int pv_j = 0, pv_b = 0, pv_h = 0, pv_c = 0, pv_valid = 0;
-        float pv_rho = 1.f;
+        // ============================== block workers ==============================
+        const int w = warp >> 2;  // this worker runs the blocks kb with kb % 2 == w
+        const int wq = warp & 3;  // TMEM lane quarter of this warp
+        const int row = tid & 127;  // block row t / state row n (TMEM lane)
+        const int tl = row & 31;
+        const uint32_t lane_base = static_cast<uint32_t>(wq) * 32u;
+        const int bar_id = 1 + w;
+        float* red = reinterpret_cast<float*>(smem + kOffRed) + 16 * w;
+        const uint8_t* stage = smem + w * kStageBytes;
+        uint8_t* xf = smem + kOffXf + w * 16384;
+        uint8_t* bp = smem + kOffBp + w * 32768;
+        uint8_t* hp = smem + kOffHp + w * 16384;
+        float* colf = reinterpret_cast<float*>(smem + kOffColf) + w * 192;
+        float* nbeta = reinterpret_cast<float*>(smem + kOffNb) + w * 128;
+        float* a2s = reinterpret_cast<float*>(smem + kOffA2) + w * 128;
+        float4* stats = reinterpret_cast<float4*>(smem + kOffStats);
+        const uint32_t col_cb = kColCB + 128u * w;
+        const uint32_t col_acc = kColAcc + 64u * w;
+
+        Cursor cur, nxt;
+        cur.init(rg);
+        if (w == 1) cur.advance(rg);
+        nxt = cur;
+        nxt.advance(rg);
+        nxt.advance(rg);
+        auto dt_at = [&](const Cursor& q) -> float {
+            const int t = q.c * kBlk + row;
+            const bool in = t < p.L;
+            return ldg_early(p.dt + (in ? ((size_t)q.b * p.L + t) * p.H + q.h : 0), in);
+        };
+        // per-piece constants
+        int const_seg = -1;
+        float sx = 1.f, sBg = 1.f, sCg = 1.f, A2h = 0.f, D_h = 0.f, d_bound = 0.f;
+        float d = w < nb_total ? dt_at(cur) : 0.f;  // dt of this token, this block
+        // this worker's previous block, whose output is pending
+        int pv_b = 0, pv_h = 0, pv_c = 0, pv_valid = 0;
+        float pv_rho = 1.f, last_U = 1.f;
         auto output = [&](int kb) {
-            wait_phase(bars + kBarAcc0 + pv_j, (kb >> 1) & 1, abort_flag, p);
+            wait_phase(bars + kBarAcc0 + w, (kb >> 1) & 1, abort_flag, p);
             tc_fence_after();
             const size_t ybase = (((size_t)pv_b * p.L + (size_t)pv_c * kBlk + row) * p.H + pv_h) * kP;
             const bool store = row < pv_valid;
-            // two halves of 32 columns: a compact loop (the kernel is instruction-fetch bound)
+            // two halves of 32 columns: a compact loop
 #pragma unroll 1
             for (int hq = 0; hq < 2; ++hq) {
                 uint32_t r[32];
-                tmem_ld32(tmem_addr(tmem, lane_base, kColAcc + 64 * pv_j + 32 * hq), r);
+                tmem_ld32(tmem_addr(tmem, lane_base, col_acc + 32 * hq), r);
                 tmem_ld_wait();
                 if (!store) continue;
                 if constexpr (YT == SSD_OUT_I8) {
@@ -801,13 +640,13 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                     uint4* yo = reinterpret_cast<uint4*>(static_cast<__half*>(p.y) + ybase) + 4 * hq;
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        uint32_t w[4];
+                        uint32_t wq4[4];
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
                             const f2 v = fmul2(f2{__uint_as_float(r[8 * q + 2 * i]), __uint_as_float(r[8 * q + 2 * i + 1])}, s2);
-                            w[i] = pack_f16x2(v.x, v.y);
+                            wq4[i] = pack_f16x2(v.x, v.y);
                         }
-                        yo[q] = make_uint4(w[0], w[1], w[2], w[3]);
+                        yo[q] = make_uint4(wq4[0], wq4[1], wq4[2], wq4[3]);
                     }
                 } else {
                     const f2 s2 = {pv_rho, pv_rho};
@@ -821,76 +660,150 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 }
             }
             tc_fence_before();
-            wg_sync(2);
-            if (lt == 0) mbar_arrive(bars + kBarAccFree0 + pv_j);
+            wg_sync(bar_id);
+            if (row == 0) mbar_arrive(bars + kBarAccFree0 + w);
         };
-        for (int kb = 0; kb < nb_total; ++kb) {
-            const int j = kb & 1;
-            const uint8_t* stage = smem + j * kStageBytes;
-            uint8_t* xf = smem + kOffXf + j * 16384;
-            const float* colf = reinterpret_cast<const float*>(smem + kOffColf) + j * 192;
-            const float* nbeta = reinterpret_cast<const float*>(smem + kOffNb) + j * 128;
-            const float* a2s = reinterpret_cast<const float*>(smem + kOffA2) + j * 128;
-            const uint32_t col_cb = kColCB + 128u * j;
-            // ---- x -> f16: a quarter row (16 tokens' bytes) per thread and step ----
-            wait_phase(bars + kBarFull0 + j, (kb >> 1) & 1, abort_flag, p);
+        int kb_last = -1;
+        for (int kb = w; kb < nb_total; kb += 2) {
+            const uint32_t ph = (kb >> 1) & 1;  // phase parity of this worker's barriers
+            if (cur.seg != const_seg) {
+                const_seg = cur.seg;
+                const int g = cur.h / (p.H / p.G);
+                sx = p.x_scale[cur.h];
+                sBg = p.B_scale[g];
+                sCg = p.C_scale[g];
+                A2h = p.A[cur.h] * kLog2e;
+                D_h = p.D[cur.h];
+                d_bound = fabsf(D_h) / (sCg * sBg);  // |D s_x / rho| <= 2^14 needs kappa >= this / 2^14
+            }
+            const float sigma = sx * sBg;
+            const int valid = min(kBlk, p.L - cur.c * kBlk);
+            // dt of this worker's next block, in flight during this block
+            const float d_next = kb + 2 < nb_total ? dt_at(nxt) : 0.f;
+            // (a) output of this worker's previous block
+            if (kb >= 2) output(kb - 2);
+            // (b) block scan of dt (a_t = log2(e) A cumsum(dt)), with the block's max and sum
+            float incl, tot, dmax, dsum;
             {
-                uint4 w = *reinterpret_cast<const uint4*>(stage + kStX + (lt >> 2) * 64 + 16 * (lt & 3));
+                float v = d, mx = d;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float u = __shfl_up_sync(0xffffffffu, v, o);
+                    if (lane >= o) v += u;
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                if (lane == 31) red[wq] = v;
+                if (lane == 0) red[4 + wq] = mx;
+                wg_sync(bar_id);
+                const float4 ws = *reinterpret_cast<const float4*>(red);
+                const float4 wm = *reinterpret_cast<const float4*>(red + 4);
+                // prefix over warps in a fixed order, so that row 127 carries exactly dsum
+                const float p1 = ws.x, p2 = p1 + ws.y, p3 = p2 + ws.z;
+                const float pre = wq == 0 ? 0.f : (wq == 1 ? p1 : (wq == 2 ? p2 : p3));
+                dsum = p3 + ws.w;
+                dmax = fmaxf(fmaxf(wm.x, wm.y), fmaxf(wm.z, wm.w));
+                incl = A2h * (v + pre);
+                tot = A2h * dsum;
+                a2s[row] = incl;
+            }
+            wg_sync(bar_id);  // a_t of every row written (read by the M' tables below)
+            // (c) statistics chained through the workers: the bound hb on |H| / s_x s_B entering
+            //     this block and the state unit U of the previous block
+            const bool pstart = cur.c == cur.cb;
+            if (kb >= 1) wait_phase(bars + kBarSt0 + (w ^ 1), ((kb - 1) >> 1) & 1, abort_flag, p);
+            const float4 sp = kb >= 1 ? stats[w ^ 1] : make_float4(1.f, 0.f, 1.f, 0.f);
+            float hb, U_prev;
+            if (pstart) {
+                // piece start: the previous piece (this CTA's previous segment) ends with block
+                // kb - 1; store its state, then load this piece's
+                if (kb >= 1) {
+                    wait_phase(bars + kBarState, (kb - 1) & 1, abort_flag, p);
+                    tc_fence_after();
+                    int pb, phh, pcb, pce;
+                    rg.seg(cur.seg - 1, pb, phh, pcb, pce);
+                    store_piece_state(p, tmem, row, pce == p.nblk, pce != p.nblk, pb, phh, sp.z, bar_id);
+                }
+                hb = load_piece_state(p, tmem, row, red, abort_flag, cur.b, cur.h, cur.cb, sigma, bar_id);
+                U_prev = 1.f;
+            } else {
+                hb = sp.w * sp.x + 16129.f * sp.y;  // bound after block kb - 1's update
+                U_prev = sp.z;
+            }
+            const float U_new = dmax > 0.f ? pow2_ceil(127.f * dmax * (1.f / kF16Range)) : 1.f;
+            const float inv_U_new = inv_pow2(U_new);
+            const float e_end = ex2f(tot);
+            if (row == 0) {
+                stats[w] = make_float4(e_end, dsum, U_new, hb);
+                mbar_arrive(bars + kBarSt0 + w);
+            }
+            // (d) x -> f16 and B row scaled by w_t / U -> B'
+            wait_phase(bars + kBarFull0 + w, ph, abort_flag, p);
+            {
+                const int lt = row;
+                uint4 wv = *reinterpret_cast<const uint4*>(stage + kStX + (lt >> 2) * 64 + 16 * (lt & 3));
 #pragma unroll 1
                 for (int i = 0; i < 4; ++i) {
                     const int idx = lt + 128 * i;
-                    uint4 nw = w;
+                    uint4 nw = wv;
                     if (i < 3) {
                         const int n = idx + 128;
                         nw = *reinterpret_cast<const uint4*>(stage + kStX + (n >> 2) * 64 + 16 * (n & 3));
                     }
                     uint4 o0, o1;
-                    cvt16(w, o0, o1);
+                    cvt16(wv, o0, o1);
                     const int r = idx >> 2, c4 = idx & 3;
                     *reinterpret_cast<uint4*>(xf + sw128(r, 32 * c4)) = o0;
                     *reinterpret_cast<uint4*>(xf + sw128(r, 32 * c4 + 16)) = o1;
-                    w = nw;
+                    wv = nw;
                 }
             }
-            // ---- B row scaled by w_t / U -> B' (two MN blocks of 64 n), once the tables exist ----
-            wait_phase(bars + kBarPa0 + j, (kb >> 1) & 1, abort_flag, p);
-            const BlockInfo bi = info[j];
             {
-                uint8_t* bp = smem + kOffBp + j * 32768;
-                const float* wts = reinterpret_cast<const float*>(smem + kOffW) + j * 128;
-                const __half2 w2 = __float2half2_rn(wts[row]);
-                uint4 w = *reinterpret_cast<const uint4*>(stage + kStB + sw128(row, 0));
+                const __half2 w2 = __float2half2_rn(d * ex2f(tot - incl) * inv_U_new);
+                uint4 wv = *reinterpret_cast<const uint4*>(stage + kStB + sw128(row, 0));
 #pragma unroll 1
                 for (int q = 0; q < 8; ++q) {
-                    uint4 nw = w;
+                    uint4 nw = wv;
                     if (q < 7) nw = *reinterpret_cast<const uint4*>(stage + kStB + sw128(row, 16 * (q + 1)));
                     uint4 o0, o1;
-                    cvt16_scaled(w, w2, o0, o1);
+                    cvt16_scaled(wv, w2, o0, o1);
                     uint8_t* blk = bp + (q >> 2) * 16384;
                     *reinterpret_cast<uint4*>(blk + sw128(row, 32 * (q & 3))) = o0;
                     *reinterpret_cast<uint4*>(blk + sw128(row, 32 * (q & 3) + 16)) = o1;
-                    w = nw;
+                    wv = nw;
                 }
             }
             fence_proxy_async_smem();
-            wg_sync(2);
-            if (lt == 0) {
-                mbar_arrive(bars + kBarXb0 + j);
-                mbar_arrive(bars + kBarEmpty0 + j);
+            // (e) scales and M' tables of this block
+            float need = fmaxf(fmaxf(hb, 16129.f * static_cast<float>(p.N) * dmax), d_bound) *
+                         (1.f / kF16Range);
+            need = (need > 1e-30f && need < 1e30f) ? need : 1.f;  // also catches NaN / inf
+            const float rho = pow2_ceil(fmaxf(sCg * sigma * need, 1e-30f));
+            const float inv_rho = inv_pow2(rho);
+            const float invk = sCg * sigma * inv_rho;  // 1 / kappa
+            {
+                const float base = d * invk;
+                nbeta[row] = lg2f(base) - incl;  // dt = 0 gives -inf: no contribution
+                if (row < 96) {
+                    colf[colf_off(3) + row] = ex2f(a2s[96] - incl) * base;
+                    if (row < 64) colf[colf_off(2) + row] = ex2f(a2s[64] - incl) * base;
+                    if (row < 32) colf[colf_off(1) + row] = ex2f(a2s[32] - incl) * base;
+                }
             }
-            // ---- M' in place over CB, one 32-column chunk at a time (increasing order) ----
-            wait_phase(bars + kBarCb0 + j, (kb >> 1) & 1, abort_flag, p);
+            wg_sync(bar_id);  // x, B' (for the MMA) and the M' tables complete
+            if (row == 0) mbar_arrive(bars + kBarXb0 + w);
+            // (f) M' in place over CB, one 32-column chunk at a time (increasing order)
+            wait_phase(bars + kBarCb0 + w, ph, abort_flag, p);
             tc_fence_after();
             {
-                const float a2t = a2s[row];
-                const int tl = row & 31;
+                const float a2t = incl;
                 const f2 a2t2 = {a2t, a2t};
-                const float rowf = quad > 0 ? ex2f(a2t - a2s[32 * quad]) : 0.f;
+                const float rowf = wq > 0 ? ex2f(a2t - a2s[32 * wq]) : 0.f;
                 const f2 rowf2 = {rowf, rowf};
-                const float* cfq = colf + colf_off(quad);
+                const float* cfq = colf + colf_off(wq);
                 // off the diagonal: 2^(a_t - a_s) = 2^(a_t - a_32q) * 2^(a_32q - a_s), both <= 1
 #pragma unroll 1
-                for (int sc = 0; sc < quad; ++sc) {
+                for (int sc = 0; sc < wq; ++sc) {
                     uint32_t cbv[32], o[16];
                     tmem_ld32(tmem_addr(tmem, lane_base, col_cb + 32 * sc), cbv);
                     tmem_ld_wait();
@@ -906,9 +819,9 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 // diagonal sub-block: one exponential per entry, s > t masked
                 {
                     uint32_t cbv[32], o[16];
-                    tmem_ld32(tmem_addr(tmem, lane_base, col_cb + 32 * quad), cbv);
+                    tmem_ld32(tmem_addr(tmem, lane_base, col_cb + 32 * wq), cbv);
                     tmem_ld_wait();
-                    const float2* nb = reinterpret_cast<const float2*>(nbeta + 32 * quad);
+                    const float2* nb = reinterpret_cast<const float2*>(nbeta + 32 * wq);
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
                         const float2 n2 = nb[e];
@@ -916,7 +829,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                         const f2 v = fmul2(cb_pair(cbv[2 * e], cbv[2 * e + 1]), f2{ex2f(arg.x), ex2f(arg.y)});
                         o[e] = pack_f16x2(2 * e <= tl ? v.x : 0.f, 2 * e + 1 <= tl ? v.y : 0.f);
                     }
-                    tmem_st16(tmem_addr(tmem, lane_base, col_cb + 16 * quad), o);
+                    tmem_st16(tmem_addr(tmem, lane_base, col_cb + 16 * wq), o);
                 }
                 // above the diagonal: zero
                 {
@@ -924,23 +837,101 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
 #pragma unroll
                     for (int e = 0; e < 16; ++e) o[e] = 0u;
 #pragma unroll 1
-                    for (int sc = quad + 1; sc < 4; ++sc) tmem_st16(tmem_addr(tmem, lane_base, col_cb + 16 * sc), o);
+                    for (int sc = wq + 1; sc < 4; ++sc) tmem_st16(tmem_addr(tmem, lane_base, col_cb + 16 * sc), o);
                 }
                 tmem_st_wait();
             }
             tc_fence_before();
-            wg_sync(2);
-            if (lt == 0) mbar_arrive(bars + kBarMp0 + j);
-            // ---- output of the previous block while the tensor core runs this one ----
-            if (kb >= 1) output(kb - 1);
-            pv_j = j;
-            pv_b = bi.b;
-            pv_h = bi.h;
-            pv_c = bi.c;
-            pv_valid = bi.valid;
-            pv_rho = bi.rho;
+            wg_sync(bar_id);
+            if (row == 0) mbar_arrive(bars + kBarMp0 + w);
+            // (g) state hand-over, after the previous block's update: H' = H U / kappa (f16)
+            //     for C'H', then decay + rescale to this block's unit
+            if (!pstart && kb >= 1) wait_phase(bars + kBarState, (kb - 1) & 1, abort_flag, p);
+            tc_fence_after();
+            {
+                const f2 to_hp = {U_prev * invk, U_prev * invk};
+                const float th = e_end * (U_prev * inv_U_new);
+                const f2 to_h = {th, th};
+#pragma unroll 1
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t hv[32];
+                    tmem_ld32(tmem_addr(tmem, lane_base, kColH + 32 * hh), hv);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t wq4[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const f2 v = fmul2(f2{__uint_as_float(hv[8 * q + 2 * i]),
+                                                  __uint_as_float(hv[8 * q + 2 * i + 1])}, to_hp);
+                            wq4[i] = pack_f16x2(v.x, v.y);
+                        }
+                        *reinterpret_cast<uint4*>(hp + sw128(row, 64 * hh + 16 * q)) =
+                            make_uint4(wq4[0], wq4[1], wq4[2], wq4[3]);
+                    }
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const f2 v = fmul2(f2{__uint_as_float(hv[2 * i]), __uint_as_float(hv[2 * i + 1])}, to_h);
+                        hv[2 * i] = __float_as_uint(v.x);
+                        hv[2 * i + 1] = __float_as_uint(v.y);
+                    }
+                    tmem_st32(tmem_addr(tmem, lane_base, kColH + 32 * hh), hv);
+                }
+            }
+            fence_proxy_async_smem();
+            tmem_st_wait();
+            tc_fence_before();
+            wg_sync(bar_id);
+            if (row == 0) mbar_arrive(bars + kBarPh0 + w);
+            // (h) C row scaled by 2^a_t -> C' in TMEM, and D, once the previous C'H' is done
+            if (kb >= 1) wait_phase(bars + kBarCh, (kb - 1) & 1, abort_flag, p);
+            tc_fence_after();
+            {
+                const __half2 f2h = __float2half2_rn(ex2f(incl));
+                uint4 wv = *reinterpret_cast<const uint4*>(stage + kStC + sw128(row, 0));
+#pragma unroll 1
+                for (int q = 0; q < 8; ++q) {
+                    uint4 nw = wv;
+                    if (q < 7) nw = *reinterpret_cast<const uint4*>(stage + kStC + sw128(row, 16 * (q + 1)));
+                    uint4 o0, o1;
+                    cvt16_scaled(wv, f2h, o0, o1);
+                    tmem_st8(tmem_addr(tmem, lane_base, kColC + 8 * q), o0, o1);
+                    wv = nw;
+                }
+                if (row < kP)
+                    *reinterpret_cast<__half*>(smem + kOffDm + sw128(row, 2 * row)) =
+                        __float2half_rn(D_h * sx * inv_rho);
+            }
+            fence_proxy_async_smem();
+            tmem_st_wait();
+            tc_fence_before();
+            wg_sync(bar_id);  // every thread is done with the stage, C' and D are written
+            if (row == 0) {
+                mbar_arrive(bars + kBarPc0 + w);
+                mbar_arrive(bars + kBarEmpty0 + w);
+            }
+            // bookkeeping for the output at this worker's next block, and the next block
+            pv_b = cur.b;
+            pv_h = cur.h;
+            pv_c = cur.c;
+            pv_valid = valid;
+            pv_rho = rho;
+            last_U = U_new;
+            kb_last = kb;
+            cur = nxt;
+            nxt.advance(rg);
+            nxt.advance(rg);
+            d = d_next;
         }
-        if (nb_total >= 1) output(nb_total - 1);
+        if (kb_last >= 0) output(kb_last);
+        // the CTA's last block ends its last piece: the worker that ran it stores the state
+        if (kb_last == nb_total - 1 && kb_last >= 0) {
+            wait_phase(bars + kBarState, kb_last & 1, abort_flag, p);
+            tc_fence_after();
+            int lb, lh, lcb, lce;
+            rg.seg(rg.nseg - 1, lb, lh, lcb, lce);
+            store_piece_state(p, tmem, row, lce == p.nblk, lce != p.nblk, lb, lh, last_U, bar_id);
+        }
     }
 
     // ---- teardown: nothing of ours may be in flight when TMEM is released ----
