@@ -219,6 +219,9 @@ def main():
     ap.add_argument("--batch", type=int, default=None,
                     help="sequences per rank (default: the workload's batch of 2); a smaller "
                          "batch of the same shape serves profiling captures")
+    ap.add_argument("--seqlen", type=int, default=None,
+                    help="tokens per sequence (default: the workload's 16384); a shorter "
+                         "sequence of the same shape serves profiling captures")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -249,7 +252,11 @@ def main():
     int8_peak_tops = bf16_peak * INT8_PER_BF16
 
     # ---- prefill workload: this rank's own batch (seeded per rank) ----
-    overrides = {} if args.batch is None else {"batch": args.batch}
+    overrides = {}
+    if args.batch is not None:
+        overrides["batch"] = args.batch
+    if args.seqlen is not None:
+        overrides["seqlen"] = args.seqlen
     case = W.make_prefill_config(PREFILL_CFG, seed=rank_seed(1000 + PREFILL_CFG, rank), **overrides)
     x, B, C = (torch.from_numpy(a).to(dev) for a in (case.x, case.B, case.C))
     dt = torch.from_numpy(case.dt).to(dev)

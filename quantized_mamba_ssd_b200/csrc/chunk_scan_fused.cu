@@ -742,7 +742,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             {
                 const int lt = row;
                 uint4 wv = *reinterpret_cast<const uint4*>(stage + kStX + (lt >> 2) * 64 + 16 * (lt & 3));
-#pragma unroll 1
+#pragma unroll 2
                 for (int i = 0; i < 4; ++i) {
                     const int idx = lt + 128 * i;
                     uint4 nw = wv;
@@ -761,7 +761,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             {
                 const __half2 w2 = __float2half2_rn(d * ex2f(tot - incl) * inv_U_new);
                 uint4 wv = *reinterpret_cast<const uint4*>(stage + kStB + sw128(row, 0));
-#pragma unroll 1
+#pragma unroll 2
                 for (int q = 0; q < 8; ++q) {
                     uint4 nw = wv;
                     if (q < 7) nw = *reinterpret_cast<const uint4*>(stage + kStB + sw128(row, 16 * (q + 1)));
@@ -889,7 +889,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             {
                 const __half2 f2h = __float2half2_rn(ex2f(incl));
                 uint4 wv = *reinterpret_cast<const uint4*>(stage + kStC + sw128(row, 0));
-#pragma unroll 1
+#pragma unroll 2
                 for (int q = 0; q < 8; ++q) {
                     uint4 nw = wv;
                     if (q < 7) nw = *reinterpret_cast<const uint4*>(stage + kStC + sw128(row, 16 * (q + 1)));
