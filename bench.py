@@ -21,6 +21,7 @@ import statistics
 import sys
 import threading
 import time
+from pathlib import Path
 
 import numpy as np
 
@@ -40,6 +41,22 @@ INT8_PER_BF16 = 2.0  # nominal dense int8 : bf16 tensor throughput ratio on B200
 # ------------------------------------------------------------------------------------------
 # algorithmic work of one call (bytes moved once, int8 MMA ops of the causal contractions)
 # ------------------------------------------------------------------------------------------
+# DRAM traffic (read + write) per token of the fused chunk-scan kernel, from one ncu capture,
+# keyed by the SHA-256 of the kernel source that ran under it; see
+# profiles/ncu_fused_chunk_scan_b2_L8192.md.  The traffic grows in proportion to the tokens of a
+# launch, so the bench scales it to the workload.  A changed kernel reports null.
+_CAPTURED_TRAFFIC_PER_TOKEN = {
+    "0897cbf91d4a87655447f0345ea36cd509618e0dd9275c23ef15d871cc86a1ac": (339.209472e6 + 119.024640e6) / 16384,
+}
+
+
+def captured_traffic(tokens: int):
+    import hashlib
+    src = Path(__file__).resolve().parent / "quantized_mamba_ssd_b200" / "csrc" / "chunk_scan_fused.cu"
+    per_token = _CAPTURED_TRAFFIC_PER_TOKEN.get(hashlib.sha256(src.read_bytes()).hexdigest())
+    return None if per_token is None else per_token * tokens
+
+
 def prefill_alg_bytes(c: W.PrefillCase, out_bytes: int, final_state: bool) -> int:
     b, L, H, P, N, G = c.batch, c.seqlen, c.nheads, c.headdim, c.dstate, c.ngroups
     n = b * L * H * P  # x in (int8)
@@ -340,7 +357,7 @@ def main():
     achieved_gbs = alg_bytes / (ms * 1e-3) / 1e9
     roofline = {
         "bound": bound, "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
-        "frac": achieved_gbs / hbm_peak, "traffic": None,
+        "frac": achieved_gbs / hbm_peak, "traffic": captured_traffic(bsz * L),
         "peak_kind": f"{peak_kind} HBM copy bandwidth",
         "alg_bytes_per_launch": alg_bytes, "alg_int8_ops_per_launch": alg_ops,
         "roofline_us": 1e6 * max(t_hbm, t_ops), "frac_of_roofline_time": 1e6 * max(t_hbm, t_ops) / (ms * 1e3),
