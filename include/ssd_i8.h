@@ -96,6 +96,53 @@ SSD_API ssd_status ssd_i8_chunk_scan(const int8_t *x, const int8_t *B, const int
                              float y_scale, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Workspace bytes of ssd_i8_chunk_scan_varlen for `nseq` sequences (about 8.4 MB plus 16 bytes
+ * per sequence); 0 for nseq < 0.
+ */
+SSD_API size_t ssd_i8_chunk_scan_varlen_workspace_size(int nseq);
+
+/*
+ * Chunked SSD scan over packed variable-length sequences and strided inputs: the same
+ * computation as ssd_i8_chunk_scan, with the state starting afresh (from init_state[s] or zero)
+ * at the first token of every sequence s.  This is the prefill of a serving batch whose prompts
+ * are packed back to back, reading x, B, C and dt straight out of a wider projection output.
+ *
+ *   cu_seqlens HOST int32 [nseq + 1]: sequence s is packed tokens [cu_seqlens[s],
+ *              cu_seqlens[s + 1]); non-decreasing, inside [0, total_tokens].  Empty sequences
+ *              are allowed (their final state is their initial state).  Tokens outside every
+ *              sequence are read but never written.
+ *   x          int8 rows of x_token_stride bytes, one per packed token; a row starts with the
+ *              nheads x headdim values of that token (x_token_stride >= nheads * headdim, a
+ *              multiple of 16).
+ *   B, C       int8 rows of bc_token_stride bytes, each starting with ngroups x dstate values
+ *              (bc_token_stride >= ngroups * dstate, a multiple of 16).
+ *   dt         float rows of dt_token_stride elements starting with nheads values
+ *              (dt_token_stride >= nheads).
+ *   A, D, scales, chunk_size, y_dtype, y_scale: as for ssd_i8_chunk_scan.
+ *   init_state float [nseq, nheads, headdim, dstate] or NULL; final_state likewise (not written
+ *              if NULL).
+ *   y          [total_tokens, nheads, headdim] of y_dtype, contiguous; rows of tokens outside
+ *              every sequence are left untouched.
+ *   workspace  at least ssd_i8_chunk_scan_varlen_workspace_size(nseq) bytes, 256-byte aligned.
+ * The sequence table is uploaded with cudaMemcpyAsync from host memory on `stream` (staged
+ * before the call returns), so the call cannot be captured into a CUDA graph.  Shapes, base
+ * alignments and error reporting are those of ssd_i8_chunk_scan; SSD_ERR_INVALID_ARG also
+ * covers malformed cu_seqlens and strides.
+ */
+SSD_API ssd_status ssd_i8_chunk_scan_varlen(const int8_t *x, long long x_token_stride,
+                                            const int8_t *B, const int8_t *C,
+                                            long long bc_token_stride, const float *dt,
+                                            long long dt_token_stride, const float *A,
+                                            const float *D, const float *x_scale,
+                                            const float *B_scale, const float *C_scale,
+                                            const int32_t *cu_seqlens, int nseq,
+                                            long long total_tokens, int nheads, int headdim,
+                                            int dstate, int ngroups, int chunk_size,
+                                            const float *init_state, float *final_state, void *y,
+                                            int y_dtype, float y_scale, void *workspace,
+                                            size_t workspace_bytes, void *stream);
+
+/*
  * Status of the last ssd_i8_chunk_scan call that ran on `workspace`: synchronises `stream`,
  * then returns SSD_ERR_TIMEOUT if a device-side wait of that call gave up (a CTA waiting for its
  * predecessor's state hand-off, or for a tensor-core / TMA completion) and SSD_OK otherwise.

@@ -2,6 +2,7 @@
 // caller's stream.  Declarations and their documentation live in include/ssd_i8.h.
 #include <cmath>
 #include <cstdint>
+#include <vector>
 
 #include "../../include/ssd_i8.h"
 #include "ssd_kernels.h"
@@ -95,6 +96,92 @@ ssd_status ssd_i8_chunk_scan(const int8_t* x, const int8_t* B, const int8_t* C, 
     ssd::ChunkScanArgs a{x, B, C, dt, A, D, x_scale, B_scale, C_scale, batch, seqlen, nheads,
                          headdim, dstate, ngroups, chunk_size, init_state, final_state, y,
                          y_dtype, inv, workspace};
+    return ssd::launch_chunk_scan(a, st) == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
+size_t ssd_i8_chunk_scan_varlen_workspace_size(int nseq) {
+    if (nseq < 0) return 0;
+    const size_t n = ssd::chunk_scan_varlen_workspace_bytes(nseq);
+    return (n + kWorkspaceAlign - 1) / kWorkspaceAlign * kWorkspaceAlign;
+}
+
+ssd_status ssd_i8_chunk_scan_varlen(const int8_t* x, long long x_token_stride, const int8_t* B,
+                                    const int8_t* C, long long bc_token_stride, const float* dt,
+                                    long long dt_token_stride, const float* A, const float* D,
+                                    const float* x_scale, const float* B_scale,
+                                    const float* C_scale, const int32_t* cu_seqlens, int nseq,
+                                    long long total_tokens, int nheads, int headdim, int dstate,
+                                    int ngroups, int chunk_size, const float* init_state,
+                                    float* final_state, void* y, int y_dtype, float y_scale,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+    if (nseq < 0 || total_tokens < 0 || total_tokens > 0x7fffffffLL || nheads <= 0 ||
+        headdim <= 0 || dstate <= 0 || ngroups <= 0 || chunk_size <= 0 ||
+        nheads % ngroups != 0 || !valid_out_dtype(y_dtype) || !cu_seqlens)
+        return SSD_ERR_INVALID_ARG;
+    if (!A || !D || !x_scale || !B_scale || !C_scale) return SSD_ERR_INVALID_ARG;
+    if (headdim != 64 || !chunk_dstate_ok(dstate) || !chunk_size_ok(chunk_size))
+        return SSD_ERR_UNSUPPORTED;
+    float inv = 1.f;
+    if (!out_scale(y_dtype, y_scale, &inv)) return SSD_ERR_INVALID_ARG;
+    // sequences: non-decreasing offsets inside [0, total_tokens]
+    if (nseq > 0 && (cu_seqlens[0] < 0 || cu_seqlens[nseq] > total_tokens)) return SSD_ERR_INVALID_ARG;
+    for (int s = 0; s < nseq; ++s)
+        if (cu_seqlens[s + 1] < cu_seqlens[s]) return SSD_ERR_INVALID_ARG;
+    // strides: TMA needs 16-byte multiples; rows must not overlap
+    if (x_token_stride < (long long)nheads * headdim || x_token_stride % 16 != 0 ||
+        bc_token_stride < (long long)ngroups * dstate || bc_token_stride % 16 != 0 ||
+        dt_token_stride < nheads)
+        return SSD_ERR_INVALID_ARG;
+    if (nseq == 0) return SSD_OK;
+    const size_t need = ssd_i8_chunk_scan_varlen_workspace_size(nseq);
+    if (!workspace || workspace_bytes < need ||
+        reinterpret_cast<uintptr_t>(workspace) % kWorkspaceAlign != 0)
+        return SSD_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t state_elems = (size_t)nheads * headdim * dstate;
+    // the table of non-empty sequences; an empty one only passes its initial state on
+    std::vector<int32_t> tab;
+    tab.reserve((size_t)nseq * 4);
+    long long blocks = 0;
+    for (int s = 0; s < nseq; ++s) {
+        const int len = cu_seqlens[s + 1] - cu_seqlens[s];
+        if (len == 0) {
+            if (final_state) {
+                float* dst = final_state + (size_t)s * state_elems;
+                const cudaError_t e =
+                    init_state ? cudaMemcpyAsync(dst, init_state + (size_t)s * state_elems,
+                                                 state_elems * sizeof(float),
+                                                 cudaMemcpyDeviceToDevice, st)
+                               : cudaMemsetAsync(dst, 0, state_elems * sizeof(float), st);
+                if (e != cudaSuccess) return SSD_ERR_CUDA;
+            }
+            continue;
+        }
+        tab.push_back(cu_seqlens[s]);
+        tab.push_back(len);
+        tab.push_back(static_cast<int32_t>(blocks));
+        tab.push_back(s);
+        blocks += (len + 127) / 128;
+    }
+    if (tab.empty()) return SSD_OK;
+    if (blocks > 0x7fffffffLL) return SSD_ERR_UNSUPPORTED;
+    if (!x || !B || !C || !dt || !y) return SSD_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(B) || !aligned16(C) || !aligned16(y)) return SSD_ERR_INVALID_ARG;
+    uint8_t* table = static_cast<uint8_t*>(workspace) + ssd::chunk_scan_varlen_table_offset();
+    // pageable source: the copy is staged before the call returns, so `tab` may go away
+    if (cudaMemcpyAsync(table, tab.data(), tab.size() * sizeof(int32_t), cudaMemcpyHostToDevice,
+                        st) != cudaSuccess)
+        return SSD_ERR_CUDA;
+    ssd::ChunkScanArgs a{x, B, C, dt, A, D, x_scale, B_scale, C_scale, 0, 0, nheads,
+                         headdim, dstate, ngroups, chunk_size, init_state, final_state, y,
+                         y_dtype, inv, workspace};
+    a.seq_tab = table;
+    a.nseq = static_cast<int>(tab.size() / 4);
+    a.total_tokens = total_tokens;
+    a.total_blocks = blocks;
+    a.x_token_stride = x_token_stride;
+    a.bc_token_stride = bc_token_stride;
+    a.dt_token_stride = dt_token_stride;
     return ssd::launch_chunk_scan(a, st) == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
 

@@ -1,7 +1,9 @@
 // Fused int8 SSD chunk scan for sm_100a: one persistent, warp-specialised CTA per SM, tcgen05
 // tensor cores, TMA-staged int8 tiles, the running state kept in tensor memory.
 //
-// Work: units u = (batch, head), each a sequence of nblk = ceil(L / 128) blocks of 128 tokens.
+// Work: units u = (sequence, head), each a run of ceil(len / 128) blocks of 128 tokens; the
+// sequences are either `batch` rows of L tokens or packed variable-length sequences (a table of
+// first token, length and block prefix per sequence; the state starts afresh in each).
 // The flattened (unit, block) list is cut into one contiguous range per CTA, so every SM gets
 // the same number of blocks.  A range holds at most one unit piece that starts mid-sequence
 // (its first) and one that ends mid-sequence (its last).  The CTA runs its last piece first and
@@ -113,12 +115,16 @@ struct FusedParams {
     const float* x_scale;
     const float* B_scale;
     const float* C_scale;
-    const float* init_state;
-    float* final_state;
-    void* y;
+    const float* init_state;     // [caller sequence][H][64][N] or null
+    float* final_state;          // [caller sequence][H][64][N] or null
+    void* y;                     // [packed token][H][64]
     float inv_y_scale;
-    int batch, L, H, G, N, nblk, nctas;
-    long long total;             // batch * H * nblk
+    // sequences: seq_tab[i] = {first packed token, tokens, block prefix, caller index} for the
+    // nseq non-empty sequences; without a table, nseq sequences of L tokens (nblk blocks) each
+    const int4* seq_tab;
+    int nseq, L, H, G, N, nblk, nctas;
+    long long dt_stride;         // elements between consecutive tokens of dt
+    long long total;             // H * (blocks of all sequences)
     float* slots;                // [nctas][128 n][64 p] handed-off states, units of s_x s_B
     unsigned long long* flags;   // [nctas] epoch of the published slot
     unsigned long long* status;  // [3]: epoch and code of a device-side failure, last epoch
@@ -127,45 +133,85 @@ struct FusedParams {
     int drop_publish;            // test hook: this CTA never publishes its hand-off (-1: none)
 };
 
+// {first packed token, tokens, block prefix, caller index} of non-empty sequence i
+__device__ __forceinline__ int4 seq_entry(const FusedParams& p, int i) {
+    if (p.seq_tab != nullptr) return p.seq_tab[i];
+    return make_int4(i * p.L, p.L, i * p.nblk, i);
+}
+
+// one piece of work: blocks [cb, ce) of head h of one sequence
+struct Piece {
+    int seq;   // caller index of the sequence (initial / final state)
+    int tok0;  // packed index of the sequence's first token
+    int len;   // tokens of the sequence
+    int nblk;  // 128-token blocks of the sequence
+    int h, cb, ce;
+};
+
 // the pieces of this CTA's range, in processing order (last piece first, first piece last)
 struct Range {
     long long ws, we, u_first, u_last;
-    int nseg, nblk, H;
+    int c_first, c_last, nseg, H;
+    // block f of the flattened (sequence, head, block) list
+    __device__ void locate(const FusedParams& p, long long f, long long& u, int& c) const {
+        int lo = 0, hi = p.nseq - 1;  // the last sequence whose first block is <= f
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (static_cast<long long>(H) * seq_entry(p, mid).z <= f) lo = mid;
+            else hi = mid - 1;
+        }
+        const int4 e = seq_entry(p, lo);
+        const int nb = (e.y + kBlk - 1) / kBlk;
+        const long long r = f - static_cast<long long>(H) * e.z;
+        u = static_cast<long long>(lo) * H + r / nb;
+        c = static_cast<int>(r % nb);
+    }
     __device__ void init(const FusedParams& p) {
         const long long W = p.total;
         ws = W * blockIdx.x / p.nctas;
         we = W * (blockIdx.x + 1) / p.nctas;
-        nblk = p.nblk;
         H = p.H;
-        u_first = ws / nblk;
-        u_last = we > ws ? (we - 1) / nblk : u_first;
-        nseg = we > ws ? static_cast<int>(u_last - u_first + 1) : 0;
+        nseg = 0;
+        u_first = u_last = 0;
+        c_first = c_last = 0;
+        if (we > ws) {
+            locate(p, ws, u_first, c_first);
+            locate(p, we - 1, u_last, c_last);
+            nseg = static_cast<int>(u_last - u_first + 1);
+        }
     }
-    __device__ void seg(int k, int& b, int& h, int& c_begin, int& c_end) const {
+    __device__ void seg(const FusedParams& p, int k, Piece& pc) const {
         const long long u = (k == 0) ? u_last : (k == nseg - 1 ? u_first : u_first + k);
-        c_begin = static_cast<int>(u == u_first ? ws - u * nblk : 0);
-        c_end = static_cast<int>(u == u_last ? we - u * nblk : nblk);
-        b = static_cast<int>(u / H);
-        h = static_cast<int>(u % H);
+        const int si = static_cast<int>(u / H);
+        const int4 e = seq_entry(p, si);
+        pc.seq = e.w;
+        pc.tok0 = e.x;
+        pc.len = e.y;
+        pc.nblk = (e.y + kBlk - 1) / kBlk;
+        pc.h = static_cast<int>(u % H);
+        pc.cb = u == u_first ? c_first : 0;
+        pc.ce = u == u_last ? c_last + 1 : pc.nblk;
     }
 };
 
 // position of a block in this CTA's processing order
 struct Cursor {
-    int seg, b, h, cb, ce, c;
-    __device__ void init(const Range& rg) {
+    int seg, c;
+    Piece pc;
+    __device__ void init(const FusedParams& p, const Range& rg) {
         seg = 0;
-        b = h = cb = ce = c = 0;
+        c = 0;
+        pc = Piece{0, 0, 0, 0, 0, 0, 0};
         if (rg.nseg > 0) {
-            rg.seg(0, b, h, cb, ce);
-            c = cb;
+            rg.seg(p, 0, pc);
+            c = pc.cb;
         }
     }
-    __device__ void advance(const Range& rg) {
-        if (++c >= ce && seg + 1 < rg.nseg) {
+    __device__ void advance(const FusedParams& p, const Range& rg) {
+        if (++c >= pc.ce && seg + 1 < rg.nseg) {
             ++seg;
-            rg.seg(seg, b, h, cb, ce);
-            c = cb;
+            rg.seg(p, seg, pc);
+            c = pc.cb;
         }
     }
 };
@@ -348,7 +394,7 @@ __device__ __forceinline__ void issue_cb(uint32_t d, uint32_t sC, uint32_t sB, i
 // `out_scale` converts TMEM units to units of s_x s_B.  Kept out of line: it runs once or twice
 // per CTA.
 __device__ __noinline__ void store_piece_state(const FusedParams& p, uint32_t tmem, int row,
-                                               bool final_piece, bool cta_end, int b, int h,
+                                               bool final_piece, bool cta_end, int seq, int h,
                                                float out_scale, int bar_id) {
     const uint32_t lane_base = static_cast<uint32_t>(row & ~31);
     uint32_t hv[2][32];
@@ -357,7 +403,7 @@ __device__ __noinline__ void store_piece_state(const FusedParams& p, uint32_t tm
     tmem_ld_wait();
     if (final_piece) {
         if (p.final_state != nullptr && row < p.N) {
-            float* dst = p.final_state + ((size_t)b * p.H + h) * kP * p.N;
+            float* dst = p.final_state + ((size_t)seq * p.H + h) * kP * p.N;
             const float s = out_scale * p.x_scale[h] * p.B_scale[h / (p.H / p.G)];
 #pragma unroll
             for (int jj = 0; jj < 64; ++jj)
@@ -384,14 +430,14 @@ __device__ __noinline__ void store_piece_state(const FusedParams& p, uint32_t tm
 // the caller's initial state (or zero) at sequence start, else the predecessor CTA's hand-off
 // slot after a bounded wait for its flag.  Returns max |state| over the piece's state.
 __device__ __noinline__ float load_piece_state(const FusedParams& p, uint32_t tmem, int row,
-                                               float* red, volatile uint32_t* abort_flag, int b,
+                                               float* red, volatile uint32_t* abort_flag, int seq,
                                                int h, int c_begin, float sigma, int bar_id) {
     const int warp = row >> 5, lane = row & 31;  // warp within the worker warpgroup
     const uint32_t lane_base = static_cast<uint32_t>(row & ~31);
     const float* src = nullptr;
     bool from_slot = false;
     if (c_begin == 0) {
-        if (p.init_state) src = p.init_state + ((size_t)b * p.H + h) * kP * p.N;
+        if (p.init_state) src = p.init_state + ((size_t)seq * p.H + h) * kP * p.N;
     } else {
         if (row == 0) {
             const unsigned long long* f = p.flags + (blockIdx.x - 1);
@@ -488,19 +534,20 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             tma_prefetch_map(&map_C);
             int kb = 0;
             for (int k = 0; k < rg.nseg && !*abort_flag; ++k) {
-                int b, h, cb, ce;
-                rg.seg(k, b, h, cb, ce);
-                const int g = h / (p.H / p.G);
-                for (int c = cb; c < ce; ++c, ++kb) {
+                Piece pc;
+                rg.seg(p, k, pc);
+                const int h = pc.h, g = h / (p.H / p.G);
+                for (int c = pc.cb; c < pc.ce; ++c, ++kb) {
                     const int s = kb & 1;
                     if (kb >= 2) wait_phase(bars + kBarEmpty0 + s, ((kb >> 1) - 1) & 1, abort_flag, p);
                     if (*abort_flag) break;  // after a failure no new load is started
                     uint8_t* stage = smem + s * kStageBytes;
                     uint64_t* bar = bars + kBarFull0 + s;
                     mbar_arrive_expect_tx(bar, kStageBytes);
-                    tma_load_4d(stage + kStX, &map_x, 0, h, c * kBlk, b, bar);
-                    tma_load_4d(stage + kStB, &map_B, 0, g, c * kBlk, b, bar);
-                    tma_load_4d(stage + kStC, &map_C, 0, g, c * kBlk, b, bar);
+                    const int t0 = pc.tok0 + c * kBlk;  // packed token of the block's first row
+                    tma_load_3d(stage + kStX, &map_x, 0, h, t0, bar);
+                    tma_load_3d(stage + kStB, &map_B, 0, g, t0, bar);
+                    tma_load_3d(stage + kStC, &map_C, 0, g, t0, bar);
                 }
             }
             // drain: both stages' last loads must have landed before the CTA exits
@@ -590,27 +637,27 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
         const uint32_t col_acc = kColAcc + 64u * w;
 
         Cursor cur, nxt;
-        cur.init(rg);
-        if (w == 1) cur.advance(rg);
+        cur.init(p, rg);
+        if (w == 1) cur.advance(p, rg);
         nxt = cur;
-        nxt.advance(rg);
-        nxt.advance(rg);
+        nxt.advance(p, rg);
+        nxt.advance(p, rg);
         auto dt_at = [&](const Cursor& q) -> float {
-            const int t = q.c * kBlk + row;
-            const bool in = t < p.L;
-            return ldg_early(p.dt + (in ? ((size_t)q.b * p.L + t) * p.H + q.h : 0), in);
+            const int t = q.c * kBlk + row;  // token within the sequence
+            const bool in = t < q.pc.len;
+            return ldg_early(p.dt + (in ? (size_t)(q.pc.tok0 + t) * p.dt_stride + q.pc.h : 0), in);
         };
         // per-piece constants
         int const_seg = -1;
         float sx = 1.f, sBg = 1.f, sCg = 1.f, A2h = 0.f, D_h = 0.f, d_bound = 0.f;
         float d = w < nb_total ? dt_at(cur) : 0.f;  // dt of this token, this block
         // this worker's previous block, whose output is pending
-        int pv_b = 0, pv_h = 0, pv_c = 0, pv_valid = 0;
+        int pv_tok = 0, pv_h = 0, pv_valid = 0;  // first packed token of the block
         float pv_rho = 1.f, last_U = 1.f;
         auto output = [&](int kb) {
             wait_phase(bars + kBarAcc0 + w, (kb >> 1) & 1, abort_flag, p);
             tc_fence_after();
-            const size_t ybase = (((size_t)pv_b * p.L + (size_t)pv_c * kBlk + row) * p.H + pv_h) * kP;
+            const size_t ybase = ((size_t)(pv_tok + row) * p.H + pv_h) * kP;
             const bool store = row < pv_valid;
             // two halves of 32 columns: a compact loop
 #pragma unroll 1
@@ -668,16 +715,16 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             const uint32_t ph = (kb >> 1) & 1;  // phase parity of this worker's barriers
             if (cur.seg != const_seg) {
                 const_seg = cur.seg;
-                const int g = cur.h / (p.H / p.G);
-                sx = p.x_scale[cur.h];
+                const int g = cur.pc.h / (p.H / p.G);
+                sx = p.x_scale[cur.pc.h];
                 sBg = p.B_scale[g];
                 sCg = p.C_scale[g];
-                A2h = p.A[cur.h] * kLog2e;
-                D_h = p.D[cur.h];
+                A2h = p.A[cur.pc.h] * kLog2e;
+                D_h = p.D[cur.pc.h];
                 d_bound = fabsf(D_h) / (sCg * sBg);  // |D s_x / rho| <= 2^14 needs kappa >= this / 2^14
             }
             const float sigma = sx * sBg;
-            const int valid = min(kBlk, p.L - cur.c * kBlk);
+            const int valid = min(kBlk, cur.pc.len - cur.c * kBlk);
             // dt of this worker's next block, in flight during this block
             const float d_next = kb + 2 < nb_total ? dt_at(nxt) : 0.f;
             // (a) output of this worker's previous block
@@ -710,7 +757,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             wg_sync(bar_id);  // a_t of every row written (read by the M' tables below)
             // (c) statistics chained through the workers: the bound hb on |H| / s_x s_B entering
             //     this block and the state unit U of the previous block
-            const bool pstart = cur.c == cur.cb;
+            const bool pstart = cur.c == cur.pc.cb;
             if (kb >= 1) wait_phase(bars + kBarSt0 + (w ^ 1), ((kb - 1) >> 1) & 1, abort_flag, p);
             const float4 sp = kb >= 1 ? stats[w ^ 1] : make_float4(1.f, 0.f, 1.f, 0.f);
             float hb, U_prev;
@@ -720,11 +767,13 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 if (kb >= 1) {
                     wait_phase(bars + kBarState, (kb - 1) & 1, abort_flag, p);
                     tc_fence_after();
-                    int pb, phh, pcb, pce;
-                    rg.seg(cur.seg - 1, pb, phh, pcb, pce);
-                    store_piece_state(p, tmem, row, pce == p.nblk, pce != p.nblk, pb, phh, sp.z, bar_id);
+                    Piece prev;
+                    rg.seg(p, cur.seg - 1, prev);
+                    store_piece_state(p, tmem, row, prev.ce == prev.nblk, prev.ce != prev.nblk, prev.seq,
+                                      prev.h, sp.z, bar_id);
                 }
-                hb = load_piece_state(p, tmem, row, red, abort_flag, cur.b, cur.h, cur.cb, sigma, bar_id);
+                hb = load_piece_state(p, tmem, row, red, abort_flag, cur.pc.seq, cur.pc.h, cur.pc.cb,
+                                      sigma, bar_id);
                 U_prev = 1.f;
             } else {
                 hb = sp.w * sp.x + 16129.f * sp.y;  // bound after block kb - 1's update
@@ -911,16 +960,15 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 mbar_arrive(bars + kBarEmpty0 + w);
             }
             // bookkeeping for the output at this worker's next block, and the next block
-            pv_b = cur.b;
-            pv_h = cur.h;
-            pv_c = cur.c;
+            pv_tok = cur.pc.tok0 + cur.c * kBlk;
+            pv_h = cur.pc.h;
             pv_valid = valid;
             pv_rho = rho;
             last_U = U_new;
             kb_last = kb;
             cur = nxt;
-            nxt.advance(rg);
-            nxt.advance(rg);
+            nxt.advance(p, rg);
+            nxt.advance(p, rg);
             d = d_next;
         }
         if (kb_last >= 0) output(kb_last);
@@ -928,9 +976,10 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
         if (kb_last == nb_total - 1 && kb_last >= 0) {
             wait_phase(bars + kBarState, kb_last & 1, abort_flag, p);
             tc_fence_after();
-            int lb, lh, lcb, lce;
-            rg.seg(rg.nseg - 1, lb, lh, lcb, lce);
-            store_piece_state(p, tmem, row, lce == p.nblk, lce != p.nblk, lb, lh, last_U, bar_id);
+            Piece last;
+            rg.seg(p, rg.nseg - 1, last);
+            store_piece_state(p, tmem, row, last.ce == last.nblk, last.ce != last.nblk, last.seq, last.h,
+                              last_U, bar_id);
         }
     }
 
@@ -1036,6 +1085,21 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
+// 3-D int8 map over packed tokens: [T][rows2][inner] with `tok_stride` bytes between tokens and
+// `inner` bytes between rows2 entries; box {box0, 1, rows}.
+bool make_map3(CUtensorMap* m, const void* base, int inner, int rows2, long long T,
+               long long tok_stride, int box0, int rows, CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows2, (cuuint64_t)T};
+    cuuint64_t strides[2] = {(cuuint64_t)inner, (cuuint64_t)tok_stride};
+    cuuint32_t box[3] = {(cuuint32_t)box0, 1, (cuuint32_t)rows};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 4-D int8 map over [batch][L][rows2][inner] with box {box0, 1, rows, 1}.
 bool make_map(CUtensorMap* m, const void* base, int inner, int rows2, int L, int batch, int box0,
               int rows, CUtensorMapSwizzle sw) {
@@ -1115,19 +1179,43 @@ size_t chunk_scan_workspace_bytes(int batch, int seqlen, int nheads, int headdim
     return 256 + kMaxCtas * 8 + (size_t)slots * 128 * kP * 4;
 }
 
+size_t chunk_scan_varlen_table_offset() { return 256 + kMaxCtas * 8 + (size_t)kMaxCtas * 128 * kP * 4; }
+
+size_t chunk_scan_varlen_workspace_bytes(int nseq) {
+    return chunk_scan_varlen_table_offset() + (size_t)(nseq > 0 ? nseq : 0) * 16;
+}
+
 cudaError_t launch_chunk_scan(const ChunkScanArgs& a, cudaStream_t st) {
+    const bool varlen = a.seq_tab != nullptr;
+    const long long T = varlen ? a.total_tokens : (long long)a.batch * a.seqlen;
+    const long long xs = varlen ? a.x_token_stride : (long long)a.nheads * kP;
+    const long long bcs = varlen ? a.bc_token_stride : (long long)a.ngroups * a.dstate;
     CUtensorMap mx, mB, mC;
-    if (!make_map(&mx, a.x, kP, a.nheads, a.seqlen, a.batch, kP, kBlk, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map(&mB, a.B, a.dstate, a.ngroups, a.seqlen, a.batch, 128, kBlk, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mC, a.C, a.dstate, a.ngroups, a.seqlen, a.batch, 128, kBlk, CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!make_map3(&mx, a.x, kP, a.nheads, T, xs, kP, kBlk, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map3(&mB, a.B, a.dstate, a.ngroups, T, bcs, 128, kBlk, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map3(&mC, a.C, a.dstate, a.ngroups, T, bcs, 128, kBlk, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     FusedParams p{};
     p.dt = a.dt; p.A = a.A; p.D = a.D; p.x_scale = a.x_scale; p.B_scale = a.B_scale;
     p.C_scale = a.C_scale; p.init_state = a.init_state; p.final_state = a.final_state;
     p.y = a.y; p.inv_y_scale = a.inv_y_scale;
-    p.batch = a.batch; p.L = a.seqlen; p.H = a.nheads; p.G = a.ngroups; p.N = a.dstate;
-    p.nblk = ceil_div(a.seqlen, kBlk);
-    p.total = total_blocks(a.batch, a.seqlen, a.nheads);
+    p.H = a.nheads; p.G = a.ngroups; p.N = a.dstate;
+    if (varlen) {
+        p.seq_tab = static_cast<const int4*>(a.seq_tab);
+        p.nseq = a.nseq;
+        p.L = 0;
+        p.nblk = 0;
+        p.total = (long long)a.nheads * a.total_blocks;
+        p.dt_stride = a.dt_token_stride;
+    } else {
+        p.seq_tab = nullptr;
+        p.nseq = a.batch;
+        p.L = a.seqlen;
+        p.nblk = ceil_div(a.seqlen, kBlk);
+        p.total = total_blocks(a.batch, a.seqlen, a.nheads);
+        p.dt_stride = a.nheads;
+    }
+    if (p.total <= 0) return cudaSuccess;
     const int sms = num_sms();
     if (sms <= 0) return cudaErrorInvalidDevice;
     p.nctas = static_cast<int>(std::min<long long>(std::min(sms, kMaxCtas), p.total));

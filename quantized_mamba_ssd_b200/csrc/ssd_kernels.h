@@ -24,6 +24,14 @@ struct ChunkScanArgs {
     int y_dtype;
     float inv_y_scale;
     void* workspace;
+    // packed variable-length sequences (seq_tab == null: `batch` contiguous rows of `seqlen`)
+    const void* seq_tab;        // device: int4 {first token, tokens, block prefix, caller index}
+    int nseq;                   // entries of seq_tab
+    long long total_tokens;     // packed tokens addressed by x, B, C, dt, y
+    long long total_blocks;     // sum over the table of ceil(tokens / 128)
+    long long x_token_stride;   // bytes between consecutive tokens of x (heads contiguous)
+    long long bc_token_stride;  // bytes between consecutive tokens of B and of C
+    long long dt_token_stride;  // elements between consecutive tokens of dt
 };
 
 struct StateUpdateArgs {
@@ -45,6 +53,9 @@ struct StateUpdateArgs {
 
 size_t chunk_scan_workspace_bytes(int batch, int seqlen, int nheads, int headdim, int dstate,
                                   int chunk_size);
+// workspace of the variable-length scan: header, flags, 256 slots, then the sequence table
+size_t chunk_scan_varlen_workspace_bytes(int nseq);
+size_t chunk_scan_varlen_table_offset();
 cudaError_t launch_chunk_scan(const ChunkScanArgs& a, cudaStream_t stream);
 cudaError_t launch_chunk_cb(const int8_t* C, const int8_t* B, int batch, int seqlen, int ngroups,
                             int dstate, int chunk_size, int32_t* cb, cudaStream_t stream);

@@ -25,7 +25,8 @@ OUT_DTYPES = {"f32": (0, torch.float32), "f16": (1, torch.float16), "i8": (2, to
 # names of every extern "C" symbol include/ssd_i8.h declares
 EXPORTED = ("ssd_i8_abi_version", "ssd_status_string", "ssd_i8_chunk_scan_workspace_size",
             "ssd_i8_chunk_scan", "ssd_i8_state_update", "ssd_i8_chunk_cb",
-            "ssd_i8_chunk_scan_noalloc", "ssd_i8_chunk_scan_status", "ssd_i8_debug_inject")
+            "ssd_i8_chunk_scan_noalloc", "ssd_i8_chunk_scan_status", "ssd_i8_debug_inject",
+            "ssd_i8_chunk_scan_varlen_workspace_size", "ssd_i8_chunk_scan_varlen")
 
 # built-in scratch of ssd_i8_chunk_scan_noalloc (bytes); larger problems are refused
 NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -74,6 +75,13 @@ def library() -> ctypes.CDLL:
         lib.ssd_i8_debug_inject.argtypes = [ci, ctypes.c_longlong]
         lib.ssd_i8_chunk_scan_status.restype = ci
         lib.ssd_i8_chunk_scan_status.argtypes = [vp, vp]
+        ll = ctypes.c_longlong
+        lib.ssd_i8_chunk_scan_varlen_workspace_size.restype = sz
+        lib.ssd_i8_chunk_scan_varlen_workspace_size.argtypes = [ci]
+        lib.ssd_i8_chunk_scan_varlen.restype = ci
+        lib.ssd_i8_chunk_scan_varlen.argtypes = ([vp, ll, vp, vp, ll, vp, ll] + [vp] * 5 +
+                                                 [vp, ci, ll] + [ci] * 5 +
+                                                 [vp, vp, vp, ci, cf, vp, sz, vp])
         lib.ssd_i8_chunk_scan_noalloc.restype = ci
         lib.ssd_i8_chunk_scan_noalloc.argtypes = [vp] * 9 + [ci] * 7 + [vp, vp, vp, ci, cf, vp]
         _lib = lib
@@ -162,6 +170,89 @@ def ssd_i8_chunk_scan(x: torch.Tensor, B: torch.Tensor, C: torch.Tensor, dt: tor
         _stream(stream),
     ]
     _check("ssd_i8_chunk_scan", library().ssd_i8_chunk_scan(*args))
+    return y
+
+
+def _rows_ptr(t: torch.Tensor, name: str, dtype: torch.dtype, inner_shape) -> tuple:
+    """Pointer and token stride (elements) of a [T, *inner_shape] view whose inner dims are
+    contiguous (a column slice of a wider row-major buffer is accepted)."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape[1:]) != tuple(inner_shape):
+        raise ValueError(f"{name} must have shape [T, {', '.join(map(str, inner_shape))}], "
+                         f"got {tuple(t.shape)}")
+    inner = 1
+    for d in range(t.dim() - 1, 0, -1):
+        if t.shape[d] > 1 and t.stride(d) != inner:
+            raise ValueError(f"{name}: the dims after the token dim must be contiguous")
+        inner *= t.shape[d]
+    return (t.data_ptr() if t.numel() else None), (t.stride(0) if t.shape[0] > 1 else inner)
+
+
+def ssd_i8_chunk_scan_varlen_workspace_size(nseq: int) -> int:
+    return int(library().ssd_i8_chunk_scan_varlen_workspace_size(int(nseq)))
+
+
+def ssd_i8_chunk_scan_varlen(x: torch.Tensor, B: torch.Tensor, C: torch.Tensor, dt: torch.Tensor,
+                             A: torch.Tensor, D: torch.Tensor, x_scale: torch.Tensor,
+                             B_scale: torch.Tensor, C_scale: torch.Tensor, cu_seqlens,
+                             chunk_size: int, *, init_state: Optional[torch.Tensor] = None,
+                             final_state: Optional[torch.Tensor] = None,
+                             y: Optional[torch.Tensor] = None, y_dtype: str = "f16",
+                             y_scale: float = 1.0, workspace: Optional[torch.Tensor] = None,
+                             stream=None) -> torch.Tensor:
+    """Chunked int8 SSD scan over packed variable-length sequences (see
+    ``ssd_i8_chunk_scan_varlen`` in include/ssd_i8.h).
+
+    x int8 [T,h,p], B, C int8 [T,g,n], dt f32 [T,h]: token-major views whose inner dims are
+    contiguous (column slices of a projection output are fine; B and C share a token stride);
+    ``cu_seqlens``: host sequence of nseq + 1 token offsets; init_state / final_state f32
+    [nseq,h,p,n]; returns y [T,h,p] of ``y_dtype``.
+    """
+    if x.dim() != 3 or B.dim() != 3 or C.dim() != 3 or dt.dim() != 2:
+        raise ValueError("x must be [T,h,p], B/C [T,g,n] and dt [T,h]")
+    T, H, P = x.shape
+    G, N = B.shape[1], B.shape[2]
+    cu = [int(v) for v in (cu_seqlens.tolist() if hasattr(cu_seqlens, "tolist") else cu_seqlens)]
+    nseq = len(cu) - 1
+    if nseq < 0:
+        raise ValueError("cu_seqlens needs at least one entry")
+    code, tdt = OUT_DTYPES[y_dtype]
+    if y is None:
+        y = torch.empty((T, H, P), dtype=tdt, device=x.device)
+    xp, xs = _rows_ptr(x, "x", torch.int8, (H, P))
+    bp, bs = _rows_ptr(B, "B", torch.int8, (G, N))
+    cp, cs = _rows_ptr(C, "C", torch.int8, (G, N))
+    dp, ds = _rows_ptr(dt, "dt", torch.float32, (H,))
+    if bs != cs:
+        raise ValueError("B and C must have the same token stride")
+    if B.shape[0] != T or C.shape[0] != T or dt.shape[0] != T:
+        raise ValueError("x, B, C and dt must have the same number of tokens")
+    need = ssd_i8_chunk_scan_varlen_workspace_size(nseq)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    cu_arr = (ctypes.c_int32 * len(cu))(*cu)
+    args = [
+        xp, xs, bp, cp, bs, dp, ds,
+        _ptr(A, "A", torch.float32, (H,)),
+        _ptr(D, "D", torch.float32, (H,)),
+        _ptr(x_scale, "x_scale", torch.float32, (H,)),
+        _ptr(B_scale, "B_scale", torch.float32, (G,)),
+        _ptr(C_scale, "C_scale", torch.float32, (G,)),
+        ctypes.cast(cu_arr, ctypes.c_void_p), nseq, T, H, P, N, G, int(chunk_size),
+        _ptr(init_state, "init_state", torch.float32, (nseq, H, P, N)),
+        _ptr(final_state, "final_state", torch.float32, (nseq, H, P, N)),
+        _ptr(y, "y", tdt, (T, H, P)),
+        code, float(y_scale),
+        _ptr(workspace, "workspace", torch.uint8),
+        workspace.numel(),
+        _stream(stream),
+    ]
+    _check("ssd_i8_chunk_scan_varlen", library().ssd_i8_chunk_scan_varlen(*args))
     return y
 
 
