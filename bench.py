@@ -80,9 +80,12 @@ def prefill_alg_ops(c: W.PrefillCase) -> float:
     return 2.0 * (cb + mx + st + ch)
 
 
-def decode_alg_bytes(d: W.DecodeCase, out_bytes: int) -> int:
+def decode_alg_bytes(d: W.DecodeCase, out_bytes: int, state_bytes: int = 4) -> int:
+    """Bytes one decode step moves: the state read and written once (fp32, or int8 codes plus
+    one fp32 scale per (batch, head) read and written), x, B, C, dt and y."""
     b, H, P, N, G = d.batch, d.nheads, d.headdim, d.dstate, d.ngroups
-    return 2 * 4 * b * H * P * N + b * H * P + 2 * b * G * N + 4 * b * H + out_bytes * b * H * P
+    state = 2 * state_bytes * b * H * P * N + (2 * 4 * b * H if state_bytes == 1 else 0)
+    return state + b * H * P + 2 * b * G * N + 4 * b * H + out_bytes * b * H * P
 
 
 def load_peaks():
@@ -410,6 +413,46 @@ def main():
             "roofline": {"bound": "hbm", "achieved": dgbs, "peak": hbm_peak, "unit": "GB/s",
                          "frac": dgbs / hbm_peak, "traffic": None,
                          "alg_bytes_per_launch": decode_alg_bytes(d, 2)},
+        }
+        del graph
+
+        # the same 512 steps on the int8 cached state (one byte per state element)
+        sq, ss = ssd_i8.ssd_i8_state_quantize(torch.from_numpy(d.state).to(dev))
+
+        def decode_pass_q8():
+            for s in range(d.steps):
+                ssd_i8.ssd_i8_state_update_q8(sq, ss, dx[s], dB[s], dC[s], ddt[s], dA, dD, dsx,
+                                              dsb, dsc, y=dy[s], y_dtype="f16")
+
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            decode_pass_q8()
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            decode_pass_q8()
+        for _ in range(max(1, args.warmup // 2)):
+            graph.replay()
+        torch.cuda.synchronize()
+        barrier()
+        ev0.record(stream)
+        for _ in range(args.decode_passes):
+            graph.replay()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        qms = max_over_ranks(ev0.elapsed_time(ev1) / args.decode_passes, dev)
+        qstep = decode_alg_bytes(d, 2, state_bytes=1)
+        qgbs = qstep * d.steps / (qms * 1e-3) / 1e9
+        decode["int8_state"] = {
+            "metric": "SSD decode state-update tokens/s (int8 in, int8 cached state)",
+            "value": d.batch * d.steps * world / (qms * 1e-3), "unit": UNIT,
+            "ms_per_512_steps": qms, "us_per_step": 1e3 * qms / d.steps,
+            "gpu_launches_per_pass": d.steps,
+            "roofline": {"bound": "hbm", "achieved": qgbs, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": qgbs / hbm_peak, "traffic": None,
+                         "alg_bytes_per_launch": qstep},
         }
         del graph
 

@@ -211,6 +211,35 @@ SSD_API ssd_status ssd_i8_state_update(float *state, const int8_t *x, const int8
                                void *y, int y_dtype, float y_scale, void *stream);
 
 /*
+ * int8 cached SSM state (the quantized cached states of the Quamba2 rebuttal's generation-time
+ * discussion, Tables R7/R8): the state of one (batch, head) is kept as int8 codes with one fp32
+ * scale, h = state_scale[b, h] * state_q[b, h, p, n], i.e. one byte per element instead of four.
+ * Quantisation rule (used by both calls below): scale = max|h| / 127 over the (batch, head)
+ * state, code = clamp(round_half_even(h / scale), -127, 127); an all-zero state gets scale 0.
+ *
+ * ssd_i8_state_quantize: fp32 state [batch, nheads, headdim, dstate] (for instance the
+ * final_state of a prefill) -> state_q int8 [same shape] and state_scale float [batch, nheads].
+ */
+SSD_API ssd_status ssd_i8_state_quantize(const float *state, int8_t *state_q, float *state_scale,
+                                         int batch, int nheads, int headdim, int dstate,
+                                         void *stream);
+
+/*
+ * One decode step on the int8 cached state, in place: dequantise, apply the step of
+ * ssd_i8_state_update in fp32 (y from the updated fp32 state), then requantise with the rule
+ * above (a fresh scale per step).  Arguments as for ssd_i8_state_update, with state_q /
+ * state_scale in place of the fp32 state.
+ * Supported: dstate in {16, 32, 64, 128, 256}; headdim * dstate <= 16384; nheads % ngroups == 0;
+ * state_q, B and C 16-byte aligned.
+ */
+SSD_API ssd_status ssd_i8_state_update_q8(int8_t *state_q, float *state_scale, const int8_t *x,
+                                          const int8_t *B, const int8_t *C, const float *dt,
+                                          const float *A, const float *D, const float *x_scale,
+                                          const float *B_scale, const float *C_scale, int batch,
+                                          int nheads, int headdim, int dstate, int ngroups,
+                                          void *y, int y_dtype, float y_scale, void *stream);
+
+/*
  * ChunkBMM of SSDi8 (Table 5): the exact int32 products CB[b, c, g, t, s] =
  * sum_n Cq[b, c*Q+t, g, n] * Bq[b, c*Q+s, g, n] for every chunk c of length Q, the full
  * Q x Q block (no causal mask), zero where c*Q+t or c*Q+s >= seqlen.  Computed by the same

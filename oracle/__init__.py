@@ -12,6 +12,8 @@ definitions and their sources):
 * :func:`step` -- one decode step on an fp64 state.
 * :func:`chunk_cb` -- SSDi8's ChunkBMM matrix CB = Cq Bq^T per chunk and group, int64.
 * :func:`requant` -- static symmetric int8 requantization of an output.
+* :func:`quantize_state` / :func:`step_q8` -- the int8 cached decode state (one scale per
+  (batch, head), max|h| / 127) and one decode step on it: dequantize, fp64 step, requantize.
 """
 from __future__ import annotations
 
@@ -28,7 +30,7 @@ _LIB = os.path.join(_HERE, "libssd_oracle.so")
 _lock = threading.Lock()
 _lib = None
 
-__all__ = ["build", "load", "scan", "step", "chunk_cb", "requant"]
+__all__ = ["build", "load", "scan", "step", "chunk_cb", "requant", "quantize_state", "step_q8"]
 
 
 def build(force: bool = False) -> str:
@@ -155,3 +157,28 @@ def requant(y, y_scale: float):
     if r < 0:
         raise ValueError("ssd_oracle_requant failed")
     return q
+
+
+def quantize_state(state):
+    """int8 cached state: per (batch, head) scale = max|h| / 127 over [p, n] and codes
+    clamp(rne(h / scale), -127, 127) decided in fp64 (an all-zero state gets scale 0 and codes
+    0).  state [b,h,p,n]; returns (codes int8 [b,h,p,n], scales float64 [b,h])."""
+    st = np.asarray(state, dtype=np.float64)
+    bsz, H = st.shape[:2]
+    scales = np.abs(st).reshape(bsz, H, -1).max(axis=2) / 127.0
+    codes = np.zeros(st.shape, dtype=np.int8)
+    for b in range(bsz):
+        for h in range(H):
+            if scales[b, h] > 0:
+                codes[b, h] = requant(st[b, h], scales[b, h])
+    return codes, scales
+
+
+def step_q8(codes, scales, x, B, C, dt, A, D, x_scale, B_scale, C_scale):
+    """One decode step on an int8 cached state: h = scale * code (fp64), the fp64 step of
+    :func:`step`, then :func:`quantize_state` of the updated state.  Returns (y, codes, scales)."""
+    state = np.ascontiguousarray(np.asarray(codes, dtype=np.float64)
+                                 * np.asarray(scales, dtype=np.float64)[:, :, None, None])
+    y = step(state, x, B, C, dt, A, D, x_scale, B_scale, C_scale)
+    c2, s2 = quantize_state(state)
+    return y, c2, s2

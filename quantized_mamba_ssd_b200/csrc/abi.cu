@@ -208,6 +208,43 @@ ssd_status ssd_i8_state_update(float* state, const int8_t* x, const int8_t* B, c
                : SSD_ERR_CUDA;
 }
 
+ssd_status ssd_i8_state_quantize(const float* state, int8_t* state_q, float* state_scale,
+                                 int batch, int nheads, int headdim, int dstate, void* stream) {
+    if (batch < 0 || nheads <= 0 || headdim <= 0 || dstate <= 0) return SSD_ERR_INVALID_ARG;
+    if (!ssd::state_q8_shape_ok(headdim, dstate)) return SSD_ERR_UNSUPPORTED;
+    if (batch == 0) return SSD_OK;
+    if (!state || !state_q || !state_scale) return SSD_ERR_INVALID_ARG;
+    if (!aligned16(state) || !aligned16(state_q)) return SSD_ERR_INVALID_ARG;
+    return ssd::launch_state_quantize(state, state_q, state_scale, batch * nheads, headdim, dstate,
+                                      static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? SSD_OK
+               : SSD_ERR_CUDA;
+}
+
+ssd_status ssd_i8_state_update_q8(int8_t* state_q, float* state_scale, const int8_t* x,
+                                  const int8_t* B, const int8_t* C, const float* dt,
+                                  const float* A, const float* D, const float* x_scale,
+                                  const float* B_scale, const float* C_scale, int batch,
+                                  int nheads, int headdim, int dstate, int ngroups, void* y,
+                                  int y_dtype, float y_scale, void* stream) {
+    if (batch < 0 || nheads <= 0 || headdim <= 0 || dstate <= 0 || ngroups <= 0 ||
+        nheads % ngroups != 0 || !valid_out_dtype(y_dtype))
+        return SSD_ERR_INVALID_ARG;
+    if (!ssd::state_q8_shape_ok(headdim, dstate)) return SSD_ERR_UNSUPPORTED;
+    float inv = 1.f;
+    if (!out_scale(y_dtype, y_scale, &inv)) return SSD_ERR_INVALID_ARG;
+    if (batch == 0) return SSD_OK;
+    if (!state_q || !state_scale || !x || !B || !C || !dt || !A || !D || !x_scale || !B_scale ||
+        !C_scale || !y)
+        return SSD_ERR_INVALID_ARG;
+    if (!aligned16(state_q) || !aligned16(B) || !aligned16(C)) return SSD_ERR_INVALID_ARG;
+    ssd::StateUpdateQ8Args a{state_q, state_scale, x, B, C, dt, A, D, x_scale, B_scale,
+                             C_scale, batch, nheads, headdim, dstate, ngroups, y, y_dtype, inv};
+    return ssd::launch_state_update_q8(a, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? SSD_OK
+               : SSD_ERR_CUDA;
+}
+
 ssd_status ssd_i8_chunk_cb(const int8_t* C, const int8_t* B, int batch, int seqlen, int ngroups,
                            int dstate, int chunk_size, int32_t* cb, void* stream) {
     if (batch < 0 || seqlen < 0 || ngroups <= 0 || dstate <= 0 || chunk_size <= 0)

@@ -51,6 +51,24 @@ struct StateUpdateArgs {
     float inv_y_scale;
 };
 
+struct StateUpdateQ8Args {
+    int8_t* state_q;     // [batch, nheads, headdim, dstate] codes
+    float* state_scale;  // [batch, nheads]
+    const int8_t* x;
+    const int8_t* B;
+    const int8_t* C;
+    const float* dt;
+    const float* A;
+    const float* D;
+    const float* x_scale;
+    const float* B_scale;
+    const float* C_scale;
+    int batch, nheads, headdim, dstate, ngroups;
+    void* y;
+    int y_dtype;
+    float inv_y_scale;
+};
+
 size_t chunk_scan_workspace_bytes(int batch, int seqlen, int nheads, int headdim, int dstate,
                                   int chunk_size);
 // workspace of the variable-length scan: header, flags, 256 slots, then the sequence table
@@ -60,6 +78,10 @@ cudaError_t launch_chunk_scan(const ChunkScanArgs& a, cudaStream_t stream);
 cudaError_t launch_chunk_cb(const int8_t* C, const int8_t* B, int batch, int seqlen, int ngroups,
                             int dstate, int chunk_size, int32_t* cb, cudaStream_t stream);
 cudaError_t launch_state_update(const StateUpdateArgs& a, cudaStream_t stream);
+bool state_q8_shape_ok(int headdim, int dstate);
+cudaError_t launch_state_update_q8(const StateUpdateQ8Args& a, cudaStream_t stream);
+cudaError_t launch_state_quantize(const float* state, int8_t* q, float* scale, int count,
+                                  int headdim, int dstate, cudaStream_t stream);
 void arm_fault_injection(int drop_publish_cta, long long wait_cycles);
 
 }  // namespace ssd

@@ -26,7 +26,8 @@ OUT_DTYPES = {"f32": (0, torch.float32), "f16": (1, torch.float16), "i8": (2, to
 EXPORTED = ("ssd_i8_abi_version", "ssd_status_string", "ssd_i8_chunk_scan_workspace_size",
             "ssd_i8_chunk_scan", "ssd_i8_state_update", "ssd_i8_chunk_cb",
             "ssd_i8_chunk_scan_noalloc", "ssd_i8_chunk_scan_status", "ssd_i8_debug_inject",
-            "ssd_i8_chunk_scan_varlen_workspace_size", "ssd_i8_chunk_scan_varlen")
+            "ssd_i8_chunk_scan_varlen_workspace_size", "ssd_i8_chunk_scan_varlen",
+            "ssd_i8_state_quantize", "ssd_i8_state_update_q8")
 
 # built-in scratch of ssd_i8_chunk_scan_noalloc (bytes); larger problems are refused
 NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -82,6 +83,10 @@ def library() -> ctypes.CDLL:
         lib.ssd_i8_chunk_scan_varlen.argtypes = ([vp, ll, vp, vp, ll, vp, ll] + [vp] * 5 +
                                                  [vp, ci, ll] + [ci] * 5 +
                                                  [vp, vp, vp, ci, cf, vp, sz, vp])
+        lib.ssd_i8_state_quantize.restype = ci
+        lib.ssd_i8_state_quantize.argtypes = [vp, vp, vp] + [ci] * 4 + [vp]
+        lib.ssd_i8_state_update_q8.restype = ci
+        lib.ssd_i8_state_update_q8.argtypes = [vp] * 11 + [ci] * 5 + [vp, ci, cf, vp]
         lib.ssd_i8_chunk_scan_noalloc.restype = ci
         lib.ssd_i8_chunk_scan_noalloc.argtypes = [vp] * 9 + [ci] * 7 + [vp, vp, vp, ci, cf, vp]
         _lib = lib
@@ -285,6 +290,59 @@ def ssd_i8_state_update(state: torch.Tensor, x: torch.Tensor, B: torch.Tensor, C
         _stream(stream),
     ]
     _check("ssd_i8_state_update", library().ssd_i8_state_update(*args))
+    return y
+
+
+def ssd_i8_state_quantize(state: torch.Tensor, state_q: Optional[torch.Tensor] = None,
+                          state_scale: Optional[torch.Tensor] = None, stream=None):
+    """fp32 state [b,h,p,n] -> (int8 codes [b,h,p,n], float32 scales [b,h]) with scale =
+    max|h| / 127 per (batch, head) (see ``ssd_i8_state_quantize`` in include/ssd_i8.h)."""
+    bsz, H, P, N = state.shape
+    if state_q is None:
+        state_q = torch.empty((bsz, H, P, N), dtype=torch.int8, device=state.device)
+    if state_scale is None:
+        state_scale = torch.empty((bsz, H), dtype=torch.float32, device=state.device)
+    _check("ssd_i8_state_quantize", library().ssd_i8_state_quantize(
+        _ptr(state, "state", torch.float32, (bsz, H, P, N)),
+        _ptr(state_q, "state_q", torch.int8, (bsz, H, P, N)),
+        _ptr(state_scale, "state_scale", torch.float32, (bsz, H)), bsz, H, P, N,
+        _stream(stream)))
+    return state_q, state_scale
+
+
+def ssd_i8_state_update_q8(state_q: torch.Tensor, state_scale: torch.Tensor, x: torch.Tensor,
+                           B: torch.Tensor, C: torch.Tensor, dt: torch.Tensor, A: torch.Tensor,
+                           D: torch.Tensor, x_scale: torch.Tensor, B_scale: torch.Tensor,
+                           C_scale: torch.Tensor, *, y: Optional[torch.Tensor] = None,
+                           y_dtype: str = "f16", y_scale: float = 1.0,
+                           stream=None) -> torch.Tensor:
+    """One decode step on the int8 cached state, in place (see ``ssd_i8_state_update_q8``).
+
+    state_q int8 [b,h,p,n] and state_scale f32 [b,h] are updated; x int8 [b,h,p]; B, C int8
+    [b,g,n]; dt f32 [b,h]; returns y [b,h,p] of ``y_dtype``."""
+    bsz, H, P, N = state_q.shape
+    G = B.shape[1]
+    code, tdt = OUT_DTYPES[y_dtype]
+    if y is None:
+        y = torch.empty((bsz, H, P), dtype=tdt, device=state_q.device)
+    args = [
+        _ptr(state_q, "state_q", torch.int8, (bsz, H, P, N)),
+        _ptr(state_scale, "state_scale", torch.float32, (bsz, H)),
+        _ptr(x, "x", torch.int8, (bsz, H, P)),
+        _ptr(B, "B", torch.int8, (bsz, G, N)),
+        _ptr(C, "C", torch.int8, (bsz, G, N)),
+        _ptr(dt, "dt", torch.float32, (bsz, H)),
+        _ptr(A, "A", torch.float32, (H,)),
+        _ptr(D, "D", torch.float32, (H,)),
+        _ptr(x_scale, "x_scale", torch.float32, (H,)),
+        _ptr(B_scale, "B_scale", torch.float32, (G,)),
+        _ptr(C_scale, "C_scale", torch.float32, (G,)),
+        bsz, H, P, N, G,
+        _ptr(y, "y", tdt, (bsz, H, P)),
+        code, float(y_scale),
+        _stream(stream),
+    ]
+    _check("ssd_i8_state_update_q8", library().ssd_i8_state_update_q8(*args))
     return y
 
 

@@ -377,3 +377,58 @@ def test_pins_reject_planted_mistake(mutant, monkeypatch):
         assert not _pins_pass(), f"planted mistake {mutant} passed every pin"
     finally:
         shutil.rmtree(tmp, ignore_errors=True)
+
+
+# ---- int8 cached decode state (quantize_state / step_q8) ----
+
+def _random_state(seed, shape=(2, 3, 8, 16), sd=0.7):
+    return np.random.default_rng(seed).normal(0.0, sd, size=shape)
+
+
+def test_quantize_state_rule():
+    st = _random_state(21)
+    codes, scales = oracle.quantize_state(st)
+    deq = codes.astype(np.float64) * scales[:, :, None, None]
+    # every element within half a step of its code, the largest one at the end of the range
+    assert (np.abs(deq - st) <= 0.5 * scales[:, :, None, None] * (1 + 1e-12)).all()
+    for b in range(st.shape[0]):
+        for h in range(st.shape[1]):
+            i = np.unravel_index(np.abs(st[b, h]).argmax(), st[b, h].shape)
+            assert abs(int(codes[b, h][i])) == 127
+            assert np.isclose(scales[b, h], np.abs(st[b, h]).max() / 127.0, rtol=0, atol=0)
+    # an all-zero state quantizes to scale 0 and codes 0
+    z_codes, z_scales = oracle.quantize_state(np.zeros((1, 2, 4, 16)))
+    assert (z_codes == 0).all() and (z_scales == 0).all()
+
+
+def test_quantize_state_is_idempotent_on_codes():
+    st = _random_state(22)
+    codes, scales = oracle.quantize_state(st)
+    codes2, scales2 = oracle.quantize_state(codes.astype(np.float64) * scales[:, :, None, None])
+    assert np.array_equal(codes, codes2)
+    assert np.allclose(scales, scales2, rtol=1e-15, atol=0)
+
+
+def test_step_q8_with_zero_dt_keeps_the_cache():
+    # dt = 0: decay exp(0) = 1 and no input, so the dequantised state comes back unchanged
+    bsz, H, P, N, G = 2, 4, 8, 16, 2
+    codes, scales = oracle.quantize_state(_random_state(23, (bsz, H, P, N)))
+    rng = np.random.default_rng(24)
+    x = rng.integers(-127, 128, size=(bsz, H, P), dtype=np.int8)
+    B = rng.integers(-127, 128, size=(bsz, G, N), dtype=np.int8)
+    C = rng.integers(-127, 128, size=(bsz, G, N), dtype=np.int8)
+    A = -np.exp(rng.uniform(0, np.log(16), H)).astype(np.float32)
+    D = rng.normal(size=H).astype(np.float32)
+    sx = np.full(H, 0.02, np.float32)
+    sB = np.full(G, 0.03, np.float32)
+    sC = np.full(G, 0.04, np.float32)
+    dt = np.zeros((bsz, H), np.float32)
+    y, c2, s2 = oracle.step_q8(codes, scales, x, B, C, dt, A, D, sx, sB, sC)
+    assert np.array_equal(codes, c2)
+    assert np.allclose(scales, s2, rtol=1e-15, atol=0)
+    # y = C h + D x of the unchanged state
+    h = codes.astype(np.float64) * scales[:, :, None, None]
+    g = np.arange(H) // (H // G)
+    yref = np.einsum("bhpn,bhn->bhp", h, C[:, g].astype(np.float64) * sC[g][None, :, None]) \
+        + D.astype(np.float64)[None, :, None] * sx.astype(np.float64)[None, :, None] * x
+    assert np.allclose(y, yref, rtol=1e-12, atol=1e-12)
