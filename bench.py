@@ -320,6 +320,23 @@ def main():
     tokens_all = bsz * L * world
     value = aggregate_tokens_per_s(bsz * L, world, ms_max)
 
+    # ---- the same call with the Hadamard-transformed output (SSD_OUT_HADAMARD) ----
+    def step_had():
+        ssd_i8.ssd_i8_chunk_scan(x, B, C, dt, A, Dp, sx, sb, sc, Q, final_state=fs, y=y,
+                                 y_dtype="i8", y_scale=y_scale, workspace=ws, hadamard=True)
+
+    for _ in range(args.warmup):
+        step_had()
+    torch.cuda.synchronize()
+    barrier()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step_had()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    had_ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dev)
+
     # ---- end to end: pinned host inputs in, int8 output back, every step ----
     hx, hB, hC, hdt = (torch.from_numpy(a).pin_memory() for a in (case.x, case.B, case.C, case.dt))
     hy = torch.empty((bsz, L, H, P), dtype=torch.int8).pin_memory()
@@ -365,6 +382,15 @@ def main():
         "alg_bytes_per_launch": alg_bytes, "alg_int8_ops_per_launch": alg_ops,
         "roofline_us": 1e6 * max(t_hbm, t_ops), "frac_of_roofline_time": 1e6 * max(t_hbm, t_ops) / (ms * 1e3),
         "int8_peak_tops": int8_peak_tops,
+    }
+
+    had_gbs = alg_bytes / (had_ms * 1e-3) / 1e9
+    hadamard_out = {
+        "metric": "SSD scan tokens/s (int8 in), output y' = H y / 8 over headdim, int8",
+        "value": aggregate_tokens_per_s(bsz * L, world, had_ms), "unit": UNIT,
+        "ms_per_step": had_ms, "gpu_launches": args.steps * ssd_i8.KERNELS_PER_CHUNK_SCAN,
+        "roofline": {"bound": "hbm", "achieved": had_gbs, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": had_gbs / hbm_peak, "traffic": None},
     }
 
     # ---- decode state update, 512 steps of batch 128 (CUDA graph replay) ----
@@ -476,7 +502,7 @@ def main():
             "e2e": e2e,
             "gpu_launches": args.steps * ssd_i8.KERNELS_PER_CHUNK_SCAN,
             "clocks": clocks.summary(),
-            "decode": decode,
+            "hadamard_out": hadamard_out, "decode": decode,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -14,6 +14,7 @@ definitions and their sources):
 * :func:`requant` -- static symmetric int8 requantization of an output.
 * :func:`quantize_state` / :func:`step_q8` -- the int8 cached decode state (one scale per
   (batch, head), max|h| / 127) and one decode step on it: dequantize, fp64 step, requantize.
+* :func:`hadamard` -- the orthonormal Walsh-Hadamard transform of the SSD output over headdim.
 """
 from __future__ import annotations
 
@@ -30,7 +31,8 @@ _LIB = os.path.join(_HERE, "libssd_oracle.so")
 _lock = threading.Lock()
 _lib = None
 
-__all__ = ["build", "load", "scan", "step", "chunk_cb", "requant", "quantize_state", "step_q8"]
+__all__ = ["build", "load", "scan", "step", "chunk_cb", "requant", "quantize_state", "step_q8",
+           "hadamard"]
 
 
 def build(force: bool = False) -> str:
@@ -182,3 +184,14 @@ def step_q8(codes, scales, x, B, C, dt, A, D, x_scale, B_scale, C_scale):
     y = step(state, x, B, C, dt, A, D, x_scale, B_scale, C_scale)
     c2, s2 = quantize_state(state)
     return y, c2, s2
+
+
+def hadamard(y):
+    """Orthonormal Walsh-Hadamard transform over the last axis (length a power of two, Sylvester
+    order): y' = H y / sqrt(P), H from scipy.linalg.hadamard.  The transform of the SSD output
+    ahead of out_proj used with the Table R10 runs of the Quamba2 OpenReview rebuttal."""
+    from scipy.linalg import hadamard as _sylvester
+    y = np.asarray(y, dtype=np.float64)
+    P = y.shape[-1]
+    Hm = _sylvester(P).astype(np.float64) / np.sqrt(P)
+    return y @ Hm.T

@@ -14,6 +14,9 @@ constexpr size_t kWorkspaceAlign = 256;
 
 bool valid_out_dtype(int d) { return d == SSD_OUT_F32 || d == SSD_OUT_F16 || d == SSD_OUT_I8; }
 
+// chunk-scan outputs may also carry the Hadamard flag
+bool valid_scan_out(int d) { return valid_out_dtype(d & ~SSD_OUT_HADAMARD); }
+
 bool chunk_dstate_ok(int n) { return n == 16 || n == 32 || n == 64 || n == 128; }
 
 bool chunk_size_ok(int q) { return q == 64 || q == 128 || q == 256; }
@@ -24,7 +27,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // kernels multiply by its fp32 reciprocal.
 bool out_scale(int y_dtype, float y_scale, float* inv) {
     *inv = 1.f;
-    if (y_dtype != SSD_OUT_I8) return true;
+    if ((y_dtype & ~SSD_OUT_HADAMARD) != SSD_OUT_I8) return true;
     if (!(y_scale > 0.f) || !std::isfinite(y_scale)) return false;
     *inv = 1.f / y_scale;
     return std::isfinite(*inv);
@@ -66,7 +69,7 @@ ssd_status ssd_i8_chunk_scan(const int8_t* x, const int8_t* B, const int8_t* C, 
                              float y_scale, void* workspace, size_t workspace_bytes,
                              void* stream) {
     if (batch < 0 || seqlen < 0 || nheads <= 0 || headdim <= 0 || dstate <= 0 || ngroups <= 0 ||
-        chunk_size <= 0 || nheads % ngroups != 0 || !valid_out_dtype(y_dtype))
+        chunk_size <= 0 || nheads % ngroups != 0 || !valid_scan_out(y_dtype))
         return SSD_ERR_INVALID_ARG;
     if (!A || !D || !x_scale || !B_scale || !C_scale) return SSD_ERR_INVALID_ARG;
     if (headdim != 64 || !chunk_dstate_ok(dstate) || !chunk_size_ok(chunk_size))
@@ -116,7 +119,7 @@ ssd_status ssd_i8_chunk_scan_varlen(const int8_t* x, long long x_token_stride, c
                                     void* workspace, size_t workspace_bytes, void* stream) {
     if (nseq < 0 || total_tokens < 0 || total_tokens > 0x7fffffffLL || nheads <= 0 ||
         headdim <= 0 || dstate <= 0 || ngroups <= 0 || chunk_size <= 0 ||
-        nheads % ngroups != 0 || !valid_out_dtype(y_dtype) || !cu_seqlens)
+        nheads % ngroups != 0 || !valid_scan_out(y_dtype) || !cu_seqlens)
         return SSD_ERR_INVALID_ARG;
     if (!A || !D || !x_scale || !B_scale || !C_scale) return SSD_ERR_INVALID_ARG;
     if (headdim != 64 || !chunk_dstate_ok(dstate) || !chunk_size_ok(chunk_size))

@@ -242,6 +242,37 @@ __device__ __forceinline__ f2 fadd2(f2 a, f2 b) {
     return r;
 }
 
+__device__ __forceinline__ f2 fsub2(f2 a, f2 b) {
+    f2 r;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+
+// In-place Walsh-Hadamard transform of 64 values (Sylvester order, unnormalised):
+// v[q] <- sum_p (-1)^popcount(p & q) v[p].  Butterflies two at a time in packed pairs.
+__device__ __forceinline__ void fwht64(float (&v)[64]) {
+#pragma unroll
+    for (int hs = 1; hs < 64; hs <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+            // butterfly (i, i + hs) for i with bit hs clear, two of them per packed op: i and
+            // the next such i (i + 1 when hs > 1, i + 2 when hs == 1)
+            const int step = hs == 1 ? 2 : 1;
+            if ((i & hs) != 0 || (i & step) != 0) continue;
+            const int j = i + step;
+            const f2 a = {v[i], v[j]}, b = {v[i + hs], v[j + hs]};
+            const f2 s = fadd2(a, b), d = fsub2(a, b);
+            v[i] = s.x;
+            v[j] = s.y;
+            v[i + hs] = d.x;
+            v[j + hs] = d.y;
+        }
+    }
+}
+
 // hardware base-2 exponential and logarithm (MUFU; subnormal results flush to zero)
 __device__ __forceinline__ float ex2f(float v) {
     float r;
@@ -485,7 +516,7 @@ __device__ __noinline__ float load_piece_state(const FusedParams& p, uint32_t tm
 // start column of quad q's off-diagonal column factors (q = 1, 2, 3 hold 32 q entries)
 __host__ __device__ constexpr int colf_off(int q) { return 16 * q * (q - 1); }
 
-template <int YT>
+template <int YT, bool HAD>
 __global__ void __launch_bounds__(kThreads, 1)
 fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                         const __grid_constant__ CUtensorMap map_B,
@@ -659,56 +690,120 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             tc_fence_after();
             const size_t ybase = ((size_t)(pv_tok + row) * p.H + pv_h) * kP;
             const bool store = row < pv_valid;
-            // two halves of 32 columns: a compact loop
-#pragma unroll 1
-            for (int hq = 0; hq < 2; ++hq) {
-                uint32_t r[32];
-                tmem_ld32(tmem_addr(tmem, lane_base, col_acc + 32 * hq), r);
-                tmem_ld_wait();
-                if (!store) continue;
+            if constexpr (HAD) {
+                // y' = H y / 8 over the 64 head channels before the dtype conversion: the whole
+                // row in registers, a butterfly transform, the 1/8 folded into the scale
+                float v[64];
+                {
+                    uint32_t r0[32], r1[32];
+                    tmem_ld32(tmem_addr(tmem, lane_base, col_acc), r0);
+                    tmem_ld32(tmem_addr(tmem, lane_base, col_acc + 32), r1);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        v[i] = __uint_as_float(r0[i]);
+                        v[32 + i] = __uint_as_float(r1[i]);
+                    }
+                }
+                tc_fence_before();
+                wg_sync(bar_id);
+                if (row == 0) mbar_arrive(bars + kBarAccFree0 + w);
+                if (!store) return;
+                fwht64(v);
+                const float rs = pv_rho * 0.125f;
                 if constexpr (YT == SSD_OUT_I8) {
-                    // q = clamp(rint(fp32(acc * rho / s_y))): the same rounding as the fp32 output
-                    const float sc = pv_rho * p.inv_y_scale;
+                    const float sc = rs * p.inv_y_scale;
                     const f2 s2 = {sc, sc}, rnd = {kRound, kRound};
-                    uint32_t wv[8];
+                    uint4* yo = reinterpret_cast<uint4*>(static_cast<int8_t*>(p.y) + ybase);
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        uint32_t wv[4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const int o = 16 * q4 + 4 * q;
+                            const f2 v0 = fadd2(fmul2(f2{v[o], v[o + 1]}, s2), rnd);
+                            const f2 v1 = fadd2(fmul2(f2{v[o + 2], v[o + 3]}, s2), rnd);
+                            const uint32_t lo = __byte_perm(clamp_code(v0.x), clamp_code(v0.y), 0x0040);
+                            const uint32_t hi = __byte_perm(clamp_code(v1.x), clamp_code(v1.y), 0x0040);
+                            wv[q] = __byte_perm(lo, hi, 0x5410);
+                        }
+                        yo[q4] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                    }
+                } else if constexpr (YT == SSD_OUT_F16) {
+                    const f2 s2 = {rs, rs};
+                    uint4* yo = reinterpret_cast<uint4*>(static_cast<__half*>(p.y) + ybase);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
-                        const f2 v0 = fadd2(fmul2(f2{__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1])}, s2), rnd);
-                        const f2 v1 = fadd2(fmul2(f2{__uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])}, s2), rnd);
-                        const uint32_t lo = __byte_perm(clamp_code(v0.x), clamp_code(v0.y), 0x0040);
-                        const uint32_t hi = __byte_perm(clamp_code(v1.x), clamp_code(v1.y), 0x0040);
-                        wv[q] = __byte_perm(lo, hi, 0x5410);
-                    }
-                    uint4* yo = reinterpret_cast<uint4*>(static_cast<int8_t*>(p.y) + ybase) + 2 * hq;
-                    yo[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-                    yo[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
-                } else if constexpr (YT == SSD_OUT_F16) {
-                    const f2 s2 = {pv_rho, pv_rho};
-                    uint4* yo = reinterpret_cast<uint4*>(static_cast<__half*>(p.y) + ybase) + 4 * hq;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
                         uint32_t wq4[4];
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
-                            const f2 v = fmul2(f2{__uint_as_float(r[8 * q + 2 * i]), __uint_as_float(r[8 * q + 2 * i + 1])}, s2);
-                            wq4[i] = pack_f16x2(v.x, v.y);
+                            const f2 t = fmul2(f2{v[8 * q + 2 * i], v[8 * q + 2 * i + 1]}, s2);
+                            wq4[i] = pack_f16x2(t.x, t.y);
                         }
                         yo[q] = make_uint4(wq4[0], wq4[1], wq4[2], wq4[3]);
                     }
                 } else {
-                    const f2 s2 = {pv_rho, pv_rho};
-                    float4* yo = reinterpret_cast<float4*>(static_cast<float*>(p.y) + ybase) + 8 * hq;
+                    const f2 s2 = {rs, rs};
+                    float4* yo = reinterpret_cast<float4*>(static_cast<float*>(p.y) + ybase);
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const f2 v0 = fmul2(f2{__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1])}, s2);
-                        const f2 v1 = fmul2(f2{__uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])}, s2);
-                        yo[q] = make_float4(v0.x, v0.y, v1.x, v1.y);
+                    for (int q = 0; q < 16; ++q) {
+                        const f2 t0 = fmul2(f2{v[4 * q], v[4 * q + 1]}, s2);
+                        const f2 t1 = fmul2(f2{v[4 * q + 2], v[4 * q + 3]}, s2);
+                        yo[q] = make_float4(t0.x, t0.y, t1.x, t1.y);
                     }
                 }
+            } else {
+                // two halves of 32 columns: a compact loop
+#pragma unroll 1
+                for (int hq = 0; hq < 2; ++hq) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem_addr(tmem, lane_base, col_acc + 32 * hq), r);
+                    tmem_ld_wait();
+                    if (!store) continue;
+                    if constexpr (YT == SSD_OUT_I8) {
+                        // q = clamp(rint(fp32(acc * rho / s_y))): the same rounding as the fp32 output
+                        const float sc = pv_rho * p.inv_y_scale;
+                        const f2 s2 = {sc, sc}, rnd = {kRound, kRound};
+                        uint32_t wv[8];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const f2 v0 = fadd2(fmul2(f2{__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1])}, s2), rnd);
+                            const f2 v1 = fadd2(fmul2(f2{__uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])}, s2), rnd);
+                            const uint32_t lo = __byte_perm(clamp_code(v0.x), clamp_code(v0.y), 0x0040);
+                            const uint32_t hi = __byte_perm(clamp_code(v1.x), clamp_code(v1.y), 0x0040);
+                            wv[q] = __byte_perm(lo, hi, 0x5410);
+                        }
+                        uint4* yo = reinterpret_cast<uint4*>(static_cast<int8_t*>(p.y) + ybase) + 2 * hq;
+                        yo[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                        yo[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+                    } else if constexpr (YT == SSD_OUT_F16) {
+                        const f2 s2 = {pv_rho, pv_rho};
+                        uint4* yo = reinterpret_cast<uint4*>(static_cast<__half*>(p.y) + ybase) + 4 * hq;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint32_t wq4[4];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const f2 v = fmul2(f2{__uint_as_float(r[8 * q + 2 * i]), __uint_as_float(r[8 * q + 2 * i + 1])}, s2);
+                                wq4[i] = pack_f16x2(v.x, v.y);
+                            }
+                            yo[q] = make_uint4(wq4[0], wq4[1], wq4[2], wq4[3]);
+                        }
+                    } else {
+                        const f2 s2 = {pv_rho, pv_rho};
+                        float4* yo = reinterpret_cast<float4*>(static_cast<float*>(p.y) + ybase) + 8 * hq;
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const f2 v0 = fmul2(f2{__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1])}, s2);
+                            const f2 v1 = fmul2(f2{__uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])}, s2);
+                            yo[q] = make_float4(v0.x, v0.y, v1.x, v1.y);
+                        }
+                    }
+                }
+                tc_fence_before();
+                wg_sync(bar_id);
+                if (row == 0) mbar_arrive(bars + kBarAccFree0 + w);
             }
-            tc_fence_before();
-            wg_sync(bar_id);
-            if (row == 0) mbar_arrive(bars + kBarAccFree0 + w);
         };
         int kb_last = -1;
         for (int kb = w; kb < nb_total; kb += 2) {
@@ -1158,13 +1253,13 @@ long long total_blocks(int batch, int seqlen, int nheads) {
     return (long long)batch * nheads * ceil_div(seqlen, kBlk);
 }
 
-template <int YT>
+template <int YT, bool HAD>
 cudaError_t launch_fused(const CUtensorMap& mx, const CUtensorMap& mB, const CUtensorMap& mC,
                          const FusedParams& p, cudaStream_t st) {
-    cudaError_t e = cudaFuncSetAttribute(fused_chunk_scan_kernel<YT>,
+    cudaError_t e = cudaFuncSetAttribute(fused_chunk_scan_kernel<YT, HAD>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    fused_chunk_scan_kernel<YT><<<p.nctas, kThreads, kSmemBytes, st>>>(mx, mB, mC, p);
+    fused_chunk_scan_kernel<YT, HAD><<<p.nctas, kThreads, kSmemBytes, st>>>(mx, mB, mC, p);
     return cudaGetLastError();
 }
 
@@ -1235,9 +1330,12 @@ cudaError_t launch_chunk_scan(const ChunkScanArgs& a, cudaStream_t st) {
         }
     }
     switch (a.y_dtype) {
-        case SSD_OUT_F32: return launch_fused<SSD_OUT_F32>(mx, mB, mC, p, st);
-        case SSD_OUT_F16: return launch_fused<SSD_OUT_F16>(mx, mB, mC, p, st);
-        case SSD_OUT_I8: return launch_fused<SSD_OUT_I8>(mx, mB, mC, p, st);
+        case SSD_OUT_F32: return launch_fused<SSD_OUT_F32, false>(mx, mB, mC, p, st);
+        case SSD_OUT_F16: return launch_fused<SSD_OUT_F16, false>(mx, mB, mC, p, st);
+        case SSD_OUT_I8: return launch_fused<SSD_OUT_I8, false>(mx, mB, mC, p, st);
+        case SSD_OUT_F32 | SSD_OUT_HADAMARD: return launch_fused<SSD_OUT_F32, true>(mx, mB, mC, p, st);
+        case SSD_OUT_F16 | SSD_OUT_HADAMARD: return launch_fused<SSD_OUT_F16, true>(mx, mB, mC, p, st);
+        case SSD_OUT_I8 | SSD_OUT_HADAMARD: return launch_fused<SSD_OUT_I8, true>(mx, mB, mC, p, st);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -21,6 +21,7 @@ SSD_OK = 0
 STATUS_NAMES = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED",
                 3: "SSD_ERR_WORKSPACE", 4: "SSD_ERR_CUDA", 5: "SSD_ERR_TIMEOUT"}
 OUT_DTYPES = {"f32": (0, torch.float32), "f16": (1, torch.float16), "i8": (2, torch.int8)}
+OUT_HADAMARD = 16  # flag: y' = H y / 8 over headdim before the conversion (include/ssd_i8.h)
 
 # names of every extern "C" symbol include/ssd_i8.h declares
 EXPORTED = ("ssd_i8_abi_version", "ssd_status_string", "ssd_i8_chunk_scan_workspace_size",
@@ -136,8 +137,9 @@ def ssd_i8_chunk_scan(x: torch.Tensor, B: torch.Tensor, C: torch.Tensor, dt: tor
                       final_state: Optional[torch.Tensor] = None,
                       y: Optional[torch.Tensor] = None, y_dtype: str = "f16",
                       y_scale: float = 1.0, workspace: Optional[torch.Tensor] = None,
-                      stream=None) -> torch.Tensor:
-    """Chunked int8 SSD scan (see ``ssd_i8_chunk_scan`` in include/ssd_i8.h).
+                      stream=None, hadamard: bool = False) -> torch.Tensor:
+    """Chunked int8 SSD scan (see ``ssd_i8_chunk_scan`` in include/ssd_i8.h).  ``hadamard``
+    applies the output transform y' = H y / 8 over headdim (``SSD_OUT_HADAMARD``).
 
     x int8 [b,l,h,p]; B, C int8 [b,l,g,n]; dt f32 [b,l,h]; A, D, x_scale f32 [h];
     B_scale, C_scale f32 [g]; optional init_state / final_state f32 [b,h,p,n]; returns y
@@ -169,7 +171,7 @@ def ssd_i8_chunk_scan(x: torch.Tensor, B: torch.Tensor, C: torch.Tensor, dt: tor
         _ptr(init_state, "init_state", torch.float32, (bsz, H, P, N)),
         _ptr(final_state, "final_state", torch.float32, (bsz, H, P, N)),
         _ptr(y, "y", tdt, (bsz, L, H, P)),
-        code, float(y_scale),
+        code | (OUT_HADAMARD if hadamard else 0), float(y_scale),
         _ptr(workspace, "workspace", torch.uint8),
         workspace.numel(),
         _stream(stream),
@@ -209,7 +211,7 @@ def ssd_i8_chunk_scan_varlen(x: torch.Tensor, B: torch.Tensor, C: torch.Tensor, 
                              final_state: Optional[torch.Tensor] = None,
                              y: Optional[torch.Tensor] = None, y_dtype: str = "f16",
                              y_scale: float = 1.0, workspace: Optional[torch.Tensor] = None,
-                             stream=None) -> torch.Tensor:
+                             stream=None, hadamard: bool = False) -> torch.Tensor:
     """Chunked int8 SSD scan over packed variable-length sequences (see
     ``ssd_i8_chunk_scan_varlen`` in include/ssd_i8.h).
 
@@ -252,7 +254,7 @@ def ssd_i8_chunk_scan_varlen(x: torch.Tensor, B: torch.Tensor, C: torch.Tensor, 
         _ptr(init_state, "init_state", torch.float32, (nseq, H, P, N)),
         _ptr(final_state, "final_state", torch.float32, (nseq, H, P, N)),
         _ptr(y, "y", tdt, (T, H, P)),
-        code, float(y_scale),
+        code | (OUT_HADAMARD if hadamard else 0), float(y_scale),
         _ptr(workspace, "workspace", torch.uint8),
         workspace.numel(),
         _stream(stream),

@@ -1,0 +1,142 @@
+"""GPU parity of the Hadamard-transformed SSD output (y_dtype | SSD_OUT_HADAMARD).
+
+The kernel applies y' = H y / 8 over the 64 head channels (Sylvester order) in its epilogue,
+before the dtype conversion.  The oracle is the fp64 scan followed by the orthonormal transform
+from scipy; both tolerances carry over unchanged because the transform is orthonormal (it keeps
+the L2 norm of the error).  The state path does not see the flag, so final states must be
+bit-identical to a call without it.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from quantized_mamba_ssd_b200 import build as qbuild
+from quantized_mamba_ssd_b200 import ssd_i8
+from quantized_mamba_ssd_b200 import workloads as W
+from parity_util import check_close, check_i8, head_subset
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    qbuild.build()
+    ssd_i8.library()
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+
+
+def run(case, y_dtype="f32", y_scale=1.0, hadamard=True):
+    bsz, H, P, N = case.batch, case.nheads, case.headdim, case.dstate
+    fs = torch.empty((bsz, H, P, N), dtype=torch.float32, device=DEV)
+    y = ssd_i8.ssd_i8_chunk_scan(
+        dev(case.x), dev(case.B), dev(case.C), dev(case.dt), dev(case.A), dev(case.D),
+        dev(case.x_scale), dev(case.B_scale), dev(case.C_scale), case.chunk_size,
+        init_state=None if case.init_state is None else dev(case.init_state), final_state=fs,
+        y_dtype=y_dtype, y_scale=y_scale, hadamard=hadamard)
+    torch.cuda.synchronize()
+    return y.float().cpu().numpy(), fs.cpu().numpy()
+
+
+def oracle_hy(case):
+    yr, fr = oracle.scan(case.x, case.B, case.C, case.dt, case.A, case.D, case.x_scale,
+                         case.B_scale, case.C_scale, init_state=case.init_state)[:2]
+    return oracle.hadamard(yr), fr
+
+
+CASES = [
+    # b, L, H, G, N, Q, law, init
+    (2, 300, 8, 2, 128, 256, "laplace_outliers_all", True),
+    (1, 517, 4, 4, 64, 128, "laplace_spread", False),
+    (3, 130, 4, 1, 16, 64, "normal", True),
+    (1, 1, 2, 1, 128, 256, "laplace_outliers_x", True),
+]
+
+
+@pytest.mark.parametrize("b,L,H,G,N,Q,law,init", CASES)
+@pytest.mark.parametrize("out", ["f32", "f16"])
+def test_hadamard_output_matches_oracle(b, L, H, G, N, Q, law, init, out):
+    case = W.make_prefill(b, L, H, 64, N, G, Q, law=law, seed=L + N + Q,
+                          with_init_state=init)
+    y, fs = run(case, y_dtype=out)
+    yr, fr = oracle_hy(case)
+    check_close(y, yr, "H y / 8")
+    check_close(fs, fr, "final_state")
+
+
+@pytest.mark.parametrize("Q", [64, 256])
+def test_hadamard_int8_output(Q):
+    case = W.make_prefill(2, 700, 8, 64, 128, 2, Q, law="laplace_outliers_all", seed=Q,
+                          with_init_state=True)
+    yr, _ = oracle_hy(case)
+    s_y = float(np.abs(yr).max() / 127.0)
+    yq, _ = run(case, y_dtype="i8", y_scale=s_y)
+    check_i8(yq, oracle.requant(yr, s_y))
+
+
+def test_transform_is_applied_to_the_plain_output():
+    # the kernel's own untransformed fp32 output, transformed in fp64, agrees with its
+    # transformed output to fp32 rounding (a wrong sign, order or scale would not)
+    case = W.make_prefill(2, 400, 8, 64, 128, 2, 256, law="laplace_outliers_all", seed=5,
+                          with_init_state=True)
+    y_plain, f_plain = run(case, hadamard=False)
+    y_had, f_had = run(case, hadamard=True)
+    ref = oracle.hadamard(y_plain)
+    err = np.abs(y_had - ref).max()
+    assert err <= 4e-6 * np.abs(ref).max(), f"transform error {err:.3e}"
+    assert np.array_equal(f_plain, f_had), "the flag changed the final state"
+
+
+def test_int8_hadamard_is_the_fp32_hadamard_requantized():
+    case = W.make_prefill(1, 600, 4, 64, 128, 1, 256, law="laplace_spread", seed=8)
+    y32, _ = run(case, y_dtype="f32")
+    s_y = float(np.abs(y32).max() / 127.0)
+    yq, _ = run(case, y_dtype="i8", y_scale=s_y)
+    # the same fp32 value, rounded by the kernel's requantization rule
+    expect = np.clip(np.rint((y32.astype(np.float32) * np.float32(1.0 / s_y))), -127, 127)
+    d = np.abs(yq - expect)
+    assert d.max() <= 1 and (d == 0).mean() >= 0.9999
+
+
+def test_hadamard_varlen():
+    lengths = [300, 1, 129, 0, 1000, 57]
+    T = sum(lengths)
+    case = W.make_prefill(1, T, 8, 64, 128, 2, 256, law="laplace_outliers_all", seed=21)
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    init = np.random.default_rng(22).normal(0.0, 0.5, size=(len(lengths), 8, 64, 128))
+    init = init.astype(np.float32)
+    y = ssd_i8.ssd_i8_chunk_scan_varlen(
+        dev(case.x[0]), dev(case.B[0]), dev(case.C[0]), dev(case.dt[0]), dev(case.A),
+        dev(case.D), dev(case.x_scale), dev(case.B_scale), dev(case.C_scale), cu, 256,
+        init_state=dev(init), y_dtype="f32", hadamard=True)
+    torch.cuda.synchronize()
+    y = y.cpu().numpy()
+    for s in range(len(lengths)):
+        a, b = int(cu[s]), int(cu[s + 1])
+        if b == a:
+            continue
+        yr = oracle.scan(case.x[:, a:b], case.B[:, a:b], case.C[:, a:b], case.dt[:, a:b],
+                         case.A, case.D, case.x_scale, case.B_scale, case.C_scale,
+                         init_state=init[s][None])[0][0]
+        check_close(y[a:b], oracle.hadamard(yr), f"H y / 8 of sequence {s}")
+
+
+def test_hadamard_at_workload_size_sampled():
+    # the int8-output prefill workload (batch 2, 16384 tokens, 128 heads, dstate 128, 8 groups,
+    # chunk 256) in the benchmark's launch configuration, with the transform on; the oracle
+    # runs sampled (batch, head) pairs whole
+    case = W.make_prefill_config(3)
+    pairs = [(0, 0), (1, 77), (0, 127)]
+    refs = {}
+    for b, h in pairs:
+        yr, _, _ = oracle.scan(**head_subset(case, [h], batches=[b]))
+        refs[(b, h)] = oracle.hadamard(yr[0, :, 0, :])
+    s_y = float(max(np.abs(r).max() for r in refs.values()) / 127.0)
+    yq, _ = run(case, y_dtype="i8", y_scale=s_y)
+    for (b, h), r in refs.items():
+        check_i8(yq[b, :, h, :], oracle.requant(r, s_y))

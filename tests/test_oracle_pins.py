@@ -432,3 +432,24 @@ def test_step_q8_with_zero_dt_keeps_the_cache():
     yref = np.einsum("bhpn,bhn->bhp", h, C[:, g].astype(np.float64) * sC[g][None, :, None]) \
         + D.astype(np.float64)[None, :, None] * sx.astype(np.float64)[None, :, None] * x
     assert np.allclose(y, yref, rtol=1e-12, atol=1e-12)
+
+
+# ---- Hadamard output transform ----
+
+def test_hadamard_is_an_involution():
+    y = np.random.default_rng(31).normal(size=(5, 3, 64))
+    assert np.allclose(oracle.hadamard(oracle.hadamard(y)), y, rtol=0, atol=1e-12)
+
+
+def test_hadamard_of_constant_and_one_hot_rows():
+    P = 64
+    c = np.full(P, 0.5)
+    out = oracle.hadamard(c)
+    assert np.isclose(out[0], 0.5 * np.sqrt(P)) and np.allclose(out[1:], 0.0, atol=1e-15)
+    for p in (0, 1, 5, 63):
+        e = np.zeros(P)
+        e[p] = 1.0
+        col = oracle.hadamard(e)
+        # Sylvester order: entry q is (-1)^popcount(p & q) / sqrt(P)
+        want = np.array([(-1) ** bin(p & q).count("1") for q in range(P)]) / np.sqrt(P)
+        assert np.allclose(col, want, rtol=0, atol=1e-15)
