@@ -33,6 +33,7 @@ from quantized_mamba_ssd_b200 import workloads as W  # noqa: E402
 from quantized_mamba_ssd_b200.dist_util import aggregate_tokens_per_s, max_over_ranks, rank_seed  # noqa: E402
 
 PREFILL_CFG = 3
+PER_TENSOR_CFG = 4  # the same layer under the per-tensor percentile-clipped recipe
 METRIC = "SSD scan tokens/s (int8 in) at 1 B200; achieved fraction of HBM/int8 roofline"
 UNIT = "tokens/s"
 INT8_PER_BF16 = 2.0  # nominal dense int8 : bf16 tensor throughput ratio on B200 (4.5 : 2.25)
@@ -233,6 +234,8 @@ def main():
                     help="timed passes of the 512-step decode run (0 skips the decode report)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) leg")
+    ap.add_argument("--no-per-tensor", action="store_true",
+                    help="skip the per-tensor percentile-clipped workload leg")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="decode batch per rank (default: the workload's 128); smaller batches "
                          "of the same shape serve profiling captures")
@@ -368,6 +371,44 @@ def main():
         e2e = {"value": aggregate_tokens_per_s(bsz * L, world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
+    # ---- the per-tensor static recipe on the same layer: x clipped at the 99.99th percentile,
+    # B and C per-tensor absmax (same shapes, so the same algorithmic bytes) ----
+    per_tensor = None
+    if not args.no_per_tensor:
+        pcase = W.make_prefill_config(PER_TENSOR_CFG, seed=rank_seed(1000 + PER_TENSOR_CFG, rank),
+                                      **overrides)
+        px, pB, pC = (torch.from_numpy(a).to(dev) for a in (pcase.x, pcase.B, pcase.C))
+        pdt = torch.from_numpy(pcase.dt).to(dev)
+        pA, pD, psx, psb, psc = (torch.from_numpy(a).to(dev) for a in
+                                 (pcase.A, pcase.D, pcase.x_scale, pcase.B_scale, pcase.C_scale))
+
+        def step_pt():
+            ssd_i8.ssd_i8_chunk_scan(px, pB, pC, pdt, pA, pD, psx, psb, psc, Q, final_state=fs,
+                                     y=y, y_dtype="i8", y_scale=y_scale, workspace=ws)
+
+        for _ in range(args.warmup):
+            step_pt()
+        torch.cuda.synchronize()
+        barrier()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step_pt()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        pt_ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dev)
+        pt_gbs = prefill_alg_bytes(pcase, 1, True) / (pt_ms * 1e-3) / 1e9
+        per_tensor = {
+            "metric": "SSD scan tokens/s (int8 in), per-tensor static scales, x clipped at the "
+                      "99.99th percentile", "workload": pcase.name,
+            "value": aggregate_tokens_per_s(bsz * L, world, pt_ms), "unit": UNIT,
+            "ms_per_step": pt_ms, "gpu_launches": args.steps * ssd_i8.KERNELS_PER_CHUNK_SCAN,
+            "saturated_x_fraction": float((np.abs(pcase.x.astype(np.int16)) == 127).mean()),
+            "roofline": {"bound": "hbm", "achieved": pt_gbs, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": pt_gbs / hbm_peak, "traffic": None},
+        }
+        del px, pB, pC, pdt, pcase
+
     # ---- roofline of the timed call ----
     alg_bytes = prefill_alg_bytes(case, 1, True)
     alg_ops = prefill_alg_ops(case)
@@ -502,7 +543,8 @@ def main():
             "e2e": e2e,
             "gpu_launches": args.steps * ssd_i8.KERNELS_PER_CHUNK_SCAN,
             "clocks": clocks.summary(),
-            "hadamard_out": hadamard_out, "decode": decode,
+            "hadamard_out": hadamard_out, "per_tensor_percentile": per_tensor,
+            "decode": decode,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

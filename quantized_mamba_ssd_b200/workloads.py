@@ -8,7 +8,9 @@ Workloads follow the shapes the pages measure on (Mamba-2 1.3B / 2.7B / 8B SSD l
 
 * x, B, C arrive as int8 with static symmetric scales: per tensor (Quamba project page,
   "static per-tensor quantization") or per head for x and per group for B/C
-  (SSDi8 page, Table 10 "quantization axis": per-H(G)).
+  (SSDi8 page, Table 10 "quantization axis": per-H(G)).  The per-tensor Mamba-2 baseline of
+  the Quamba2 OpenReview rebuttal (the response listing Table R9) clips x at a percentile of
+  |x| and quantizes B and C per tensor by their absmax: ``scales="percentile"``.
 * x is head-structured with outlier channels (SSDi8 page, Figure 2; Quamba2 rebuttal,
   channel persistence), stood in for by Laplace values with 1 % of the (h, p) channels
   scaled x20, or a head-wise magnitude spread.
@@ -31,6 +33,7 @@ __all__ = [
     "PREFILL_CONFIGS",
     "DECODE_CONFIG",
     "quantize_symmetric",
+    "percentile_scale",
     "make_prefill",
     "make_prefill_config",
     "make_decode",
@@ -107,7 +110,16 @@ PREFILL_CONFIGS = {
     3: dict(name="mamba2-8b-ssd-long-prefill b2 L16384 h128 p64 n128 g8 Q256 int8-out", batch=2,
             seqlen=16384, nheads=128, headdim=64, dstate=128, ngroups=8, chunk_size=256,
             law="laplace_outliers_all", scales="head", out_dtype="i8"),
+    # the same layer and activations under the per-tensor static recipe: x clipped at the
+    # 99.99th percentile of |x|, B and C per-tensor absmax
+    4: dict(name="mamba2-8b-ssd-long-prefill per-tensor x-p99.99 b2 L16384 h128 p64 n128 g8 Q256 "
+                 "int8-out", batch=2, seqlen=16384, nheads=128, headdim=64, dstate=128,
+            ngroups=8, chunk_size=256, law="laplace_outliers_all", scales="percentile",
+            out_dtype="i8"),
 }
+
+# tokens of a large activation that calibrate a percentile scale (a calibration set's worth)
+CALIB_TOKENS = 2048
 
 DECODE_CONFIG = dict(name="mamba2-8b-ssd-decode b128 x512 steps h128 p64 n128 g8", batch=128,
                      steps=512, nheads=128, headdim=64, dstate=128, ngroups=8, out_dtype="f16")
@@ -143,6 +155,31 @@ def quantize_symmetric(v: np.ndarray, scale_axis: Optional[int]) -> tuple[np.nda
     return q, s
 
 
+def percentile_scale(v: np.ndarray, percentile: float) -> np.float32:
+    """Static per-tensor scale clipped at a percentile: s = P_percentile(|v|) / 127 (numpy's
+    linear interpolation between order statistics).  Values above the percentile saturate at
+    +-127 when quantized with it.
+
+    ``v`` is [batch, tokens, ...]; at most CALIB_TOKENS tokens, evenly spaced, calibrate the
+    percentile (every token when there are fewer), all channels of each.
+    """
+    v = np.asarray(v, dtype=F32)
+    step = max(1, -(-v.shape[1] // CALIB_TOKENS))
+    sample = np.abs(v[:, ::step]).reshape(-1)
+    t = float(np.percentile(sample, percentile)) if sample.size else 0.0
+    return F32(t / 127.0) if t > 0 else F32(1.0)
+
+
+def _quantize_with(v: np.ndarray, s: np.float32) -> np.ndarray:
+    """q = clamp(rne(v / s), -127, 127) with one fp32 scale, in slabs along axis 0."""
+    q = np.empty(v.shape, dtype=np.int8)
+    for i in range(v.shape[0]):
+        r = np.rint(v[i] / s)
+        np.clip(r, -127, 127, out=r)
+        q[i] = r.astype(np.int8)
+    return q
+
+
 def _laplace(rng: np.random.Generator, shape) -> np.ndarray:
     """Laplace(0, 1) in fp32: an Exp(1) magnitude with a fair random sign."""
     out = np.empty(shape, dtype=F32)
@@ -169,14 +206,15 @@ def _dt_A_D(rng: np.random.Generator, dt_shape, nheads: int):
 def make_prefill(batch: int, seqlen: int, nheads: int, headdim: int, dstate: int, ngroups: int,
                  chunk_size: int, *, law: str = "normal", scales: str = "head",
                  out_dtype: str = "f16", seed: int = 0, with_init_state: bool = False,
-                 name: Optional[str] = None) -> PrefillCase:
+                 name: Optional[str] = None, clip_percentile: float = 99.99) -> PrefillCase:
     """Draw one seeded prefill problem.
 
     law: "normal" (x, B, C ~ N(0,1)); "laplace_outliers_x" (x Laplace with 1 % outlier
     channels x20 over (h,p); B, C ~ N(0,1)); "laplace_spread" (x, B, C Laplace, x scaled
     per head and B, C per group by U(0.5, 8)); "laplace_outliers_all" (x, B, C Laplace with
     1 % outlier channels x20: x over (h,p), B and C over (g,n)).
-    scales: "tensor" (one scale per tensor, broadcast) or "head" (x per head, B/C per group).
+    scales: "tensor" (one scale per tensor, broadcast), "head" (x per head, B/C per group) or
+    "percentile" (per tensor; x clipped at ``clip_percentile`` of |x|, B/C by absmax).
     """
     if nheads % ngroups:
         raise ValueError("nheads must be a multiple of ngroups")
@@ -217,6 +255,14 @@ def make_prefill(batch: int, seqlen: int, nheads: int, headdim: int, dstate: int
         sx = np.full(nheads, sx[0], dtype=F32)
         sb = np.full(ngroups, sb[0], dtype=F32)
         sc = np.full(ngroups, sc[0], dtype=F32)
+    elif scales == "percentile":
+        s_x = percentile_scale(x, clip_percentile)
+        xq = _quantize_with(x, s_x)
+        Bq, sb = quantize_symmetric(Bf, None)
+        Cq, sc = quantize_symmetric(Cf, None)
+        sx = np.full(nheads, s_x, dtype=F32)
+        sb = np.full(ngroups, sb[0], dtype=F32)
+        sc = np.full(ngroups, sc[0], dtype=F32)
     elif scales == "head":
         xq, sx = quantize_symmetric(x, 2)
         Bq, sb = quantize_symmetric(Bf, 2)
@@ -235,7 +281,7 @@ def make_prefill(batch: int, seqlen: int, nheads: int, headdim: int, dstate: int
 
 
 def make_prefill_config(index: int, seed: Optional[int] = None, **overrides) -> PrefillCase:
-    """The prefill workload ``index`` (0..3) with its default seed 1000 + index."""
+    """The prefill workload ``index`` (0..4) with its default seed 1000 + index."""
     spec = dict(PREFILL_CONFIGS[index])
     spec.update(overrides)
     name = spec.pop("name")

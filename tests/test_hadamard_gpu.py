@@ -95,12 +95,13 @@ def test_transform_is_applied_to_the_plain_output():
 def test_int8_hadamard_is_the_fp32_hadamard_requantized():
     case = W.make_prefill(1, 600, 4, 64, 128, 1, 256, law="laplace_spread", seed=8)
     y32, _ = run(case, y_dtype="f32")
-    s_y = float(np.abs(y32).max() / 127.0)
-    yq, _ = run(case, y_dtype="i8", y_scale=s_y)
-    # the same fp32 value, rounded by the kernel's requantization rule
-    expect = np.clip(np.rint((y32.astype(np.float32) * np.float32(1.0 / s_y))), -127, 127)
-    d = np.abs(yq - expect)
-    assert d.max() <= 1 and (d == 0).mean() >= 0.9999
+    s_y = np.float32(np.abs(y32).max() / 100.0)
+    yq, _ = run(case, y_dtype="i8", y_scale=float(s_y))
+    # the per-block scale and the 1/8 are powers of two, so scaling commutes with rounding and
+    # the int8 output is exactly the f32 output requantized with fp32(1 / s_y)
+    inv = np.float32(1.0) / s_y
+    expect = np.clip(np.rint(y32.astype(np.float32) * inv), -127, 127)
+    assert np.array_equal(yq, expect)
 
 
 def test_hadamard_varlen():

@@ -67,6 +67,9 @@ SMALL = [
     (2, 257, 4, 2, 64, 256, "laplace_outliers_all", "head", False, "f16"),
     (1, 1, 4, 2, 128, 256, "normal", "head", True, "f32"),
     (1, 63, 2, 1, 128, 64, "normal", "head", True, "f32"),
+    # per-tensor static scales with x clipped at the 99.99th percentile (saturated codes)
+    (2, 600, 8, 2, 128, 256, "laplace_outliers_all", "percentile", True, "f32"),
+    (1, 300, 4, 1, 64, 128, "laplace_outliers_x", "percentile", False, "f16"),
 ]
 
 
@@ -106,7 +109,8 @@ def test_int8_output_is_the_fp32_output_requantized():
 # ---------------------------------------------------------------------------------------
 SAMPLES = {0: None, 1: [(0, 0), (3, 63), (1, 17), (2, 40)],
            2: [(0, 0), (7, 79), (3, 33), (5, 61)],
-           3: [(0, 0), (1, 127), (0, 77), (1, 35), (0, 16), (1, 100)]}
+           3: [(0, 0), (1, 127), (0, 77), (1, 35), (0, 16), (1, 100)],
+           4: [(0, 5), (1, 126), (0, 64), (1, 31)]}
 
 
 def _compare_sampled(case, y, fs, pairs, out):
@@ -119,7 +123,7 @@ def _compare_sampled(case, y, fs, pairs, out):
         check_close(fs[b, h], fr[0, 0], f"final_state[b={b},h={h}]")
 
 
-@pytest.mark.parametrize("cfg", [0, 1, 2, 3])
+@pytest.mark.parametrize("cfg", [0, 1, 2, 3, 4])
 def test_workload_prefill_matches_oracle(cfg):
     case = W.make_prefill_config(cfg)
     out = case.out_dtype
