@@ -80,8 +80,8 @@ constexpr int kOffDm = kOffHp + 2 * 16384;      // D s_x / rho on the diagonal o
 constexpr int kOffColf = kOffDm + 8192;         // off-diagonal column factors [2][192] f32
 constexpr int kOffNb = kOffColf + 2 * 768;      // -beta_s = log2(dt_s / kappa) - a_s [2][128]
 constexpr int kOffA2 = kOffNb + 2 * 512;        // a_t [2][128]
-constexpr int kOffStats = kOffA2 + 2 * 512;     // per-block statistics handed between workers [2]
-constexpr int kOffRed = kOffStats + 2 * 16;     // worker scratch [2][16] f32
+constexpr int kOffStats = kOffA2 + 2 * 512;     // per-block statistics handed between workers [2][2]
+constexpr int kOffRed = kOffStats + 4 * 16;     // worker scratch [2][16] f32
 constexpr int kOffBar = kOffRed + 2 * 64;       // mbarriers [32]
 constexpr int kOffMisc = kOffBar + 32 * 8;      // TMEM base, abort flag
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
@@ -854,7 +854,10 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             //     this block and the state unit U of the previous block
             const bool pstart = cur.c == cur.pc.cb;
             if (kb >= 1) wait_phase(bars + kBarSt0 + (w ^ 1), ((kb - 1) >> 1) & 1, abort_flag, p);
-            const float4 sp = kb >= 1 ? stats[w ^ 1] : make_float4(1.f, 0.f, 1.f, 0.f);
+            // (double-buffered by block pair: a slot is rewritten only after every reader of it
+            // has passed a later barrier)
+            const float4 sp = kb >= 1 ? stats[2 * (w ^ 1) + (((kb - 1) >> 1) & 1)]
+                                      : make_float4(1.f, 0.f, 1.f, 0.f);
             float hb, U_prev;
             if (pstart) {
                 // piece start: the previous piece (this CTA's previous segment) ends with block
@@ -878,7 +881,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             const float inv_U_new = inv_pow2(U_new);
             const float e_end = ex2f(tot);
             if (row == 0) {
-                stats[w] = make_float4(e_end, dsum, U_new, hb);
+                stats[2 * w + ph] = make_float4(e_end, dsum, U_new, hb);
                 mbar_arrive(bars + kBarSt0 + w);
             }
             // (d) x -> f16 and B row scaled by w_t / U -> B'

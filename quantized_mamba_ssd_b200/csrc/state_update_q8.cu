@@ -22,24 +22,72 @@ namespace {
 constexpr int kMaxThreads = 256;
 constexpr int kMaxChunksPerThread = 4;  // headdim * dstate <= 16384
 
-// 16 int8 codes (one 16-byte chunk) -> 16 floats, exactly and on the full-rate pipes: the
-// byte (sign bit flipped) becomes the low mantissa byte of 2^23, and 2^23 + 128 comes off again
-__device__ __forceinline__ void unpack16(const uint4 w, float (&v)[16]) {
+// packed fp32 pairs: one instruction for two lanes of work on sm_100
+struct f2 {
+    float x, y;
+};
+
+__device__ __forceinline__ f2 fmul2(f2 a, f2 b) {
+    f2 r;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+
+__device__ __forceinline__ f2 fadd2(f2 a, f2 b) {
+    f2 r;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+
+// a * b + c, one rounding
+__device__ __forceinline__ f2 ffma2(f2 a, f2 b, f2 c) {
+    f2 r;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return r;
+}
+
+// 16 int8 codes (one 16-byte chunk) -> 8 pairs of floats, exactly: the byte (sign bit flipped)
+// becomes the low mantissa byte of 2^23, and 2^23 + 128 comes off again (one packed subtract
+// per pair)
+__device__ __forceinline__ void unpack16(const uint4 w, f2 (&v)[8]) {
     const uint32_t ww[4] = {w.x ^ 0x80808080u, w.y ^ 0x80808080u, w.z ^ 0x80808080u,
                             w.w ^ 0x80808080u};
+    const f2 off = {-8388736.f, -8388736.f};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        v[4 * i + 0] = __uint_as_float(__byte_perm(ww[i], 0x4B000000u, 0x7540)) - 8388736.f;
-        v[4 * i + 1] = __uint_as_float(__byte_perm(ww[i], 0x4B000000u, 0x7541)) - 8388736.f;
-        v[4 * i + 2] = __uint_as_float(__byte_perm(ww[i], 0x4B000000u, 0x7542)) - 8388736.f;
-        v[4 * i + 3] = __uint_as_float(__byte_perm(ww[i], 0x4B000000u, 0x7543)) - 8388736.f;
+        v[2 * i] = fadd2(f2{__uint_as_float(__byte_perm(ww[i], 0x4B000000u, 0x7540)),
+                            __uint_as_float(__byte_perm(ww[i], 0x4B000000u, 0x7541))}, off);
+        v[2 * i + 1] = fadd2(f2{__uint_as_float(__byte_perm(ww[i], 0x4B000000u, 0x7542)),
+                                __uint_as_float(__byte_perm(ww[i], 0x4B000000u, 0x7543))}, off);
     }
 }
 
 // q = rne(fp32(v * inv)) of 16 values -> one 16-byte chunk, for inv = 127 / max|v| taken over the
 // same fp32 values: then |v * inv| <= 127 (1 + 2^-22) < 127.5, so no clamp is needed.  Adding
 // 1.5 * 2^23 rounds to an integer (half to even) in the low mantissa bits, whose low byte is then
-// the code.
+// the code.  The multiply and the add are separate roundings (no contraction).
+__device__ __forceinline__ uint4 pack16(const f2 (&v)[8], float inv) {
+    const f2 i2 = {inv, inv}, rnd = {12582912.f, 12582912.f};
+    uint32_t ww[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const f2 a = fadd2(fmul2(v[2 * i], i2), rnd), b = fadd2(fmul2(v[2 * i + 1], i2), rnd);
+        ww[i] = __byte_perm(__byte_perm(__float_as_uint(a.x), __float_as_uint(a.y), 0x0040),
+                            __byte_perm(__float_as_uint(b.x), __float_as_uint(b.y), 0x0040), 0x5410);
+    }
+    return make_uint4(ww[0], ww[1], ww[2], ww[3]);
+}
+
+// scalar form of pack16 for the fp32 quantiser
 __device__ __forceinline__ uint4 pack16(const float (&v)[16], float inv) {
     constexpr float kRound = 12582912.f;
     uint32_t ww[4];
@@ -68,111 +116,140 @@ __device__ __forceinline__ float block_max(float v, float* scratch) {
     return m;
 }
 
+// 16-byte asynchronous copy global -> shared (bypasses L1), and its group fences
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int K>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(K) : "memory"); }
+
+// Persistent CTAs, each walking the (batch, head) items blockIdx.x, + gridDim.x, ...  Every
+// thread copies its own 16-byte state chunks (and the B or C chunk it stages) of the NEXT item
+// into its private slots of a two-stage shared buffer while it computes the current one, so
+// the loads stay in flight without holding registers; the current item's update is kept in
+// registers between the y / max pass and the requantisation.
 template <int N, int TPB, int CH>
-__global__ void __launch_bounds__(TPB)
+__global__ void __launch_bounds__(TPB, (CH >= 4 ? 512 : 640) / TPB)  // the update in registers
 state_update_q8_kernel(int8_t* __restrict__ state_q, float* __restrict__ state_scale,
                        const int8_t* __restrict__ x, const int8_t* __restrict__ Bq,
                        const int8_t* __restrict__ Cq, const float* __restrict__ dt,
                        const float* __restrict__ A, const float* __restrict__ D,
                        const float* __restrict__ x_scale, const float* __restrict__ B_scale,
-                       const float* __restrict__ C_scale, int H, int P, int G,
+                       const float* __restrict__ C_scale, int count, int H, int P, int G,
                        void* __restrict__ y, int y_dtype, float inv_y_scale) {
     constexpr int CPR = N / 16;  // 16-byte chunks per state row (lanes per row, <= 16)
     __shared__ float scratch[TPB / kWarp];
-    __shared__ __align__(16) float sbv[N], scv[N];  // s_B B_n and s_C C_n of this (batch, group)
-    const int h = blockIdx.x, b = blockIdx.y;
-    const int g = h / (H / G);
+    // s_B B_n and s_C C_n (double-buffered), float4 j of chunk cc at [j * CPR + cc]: the lanes
+    // of a warp read consecutive 16-byte words (chunk cc of state row p pairs with B, C chunk cc)
+    __shared__ __align__(16) float4 sbv[2][N / 4], scv[2][N / 4];
+    // copies in flight: [stage][chunk k][thread] state chunks, [stage][thread < 2 CPR] B/C chunks
+    __shared__ __align__(16) uint4 sq[2][CH][TPB];
+    __shared__ __align__(16) uint4 sbc[2][2 * CPR];
     const int tid = threadIdx.x, lane = tid & (kWarp - 1);
-    const size_t bh = (size_t)b * H + h;
     const int nchunks = P * CPR;
+    int item = blockIdx.x;
+    if (item >= count) return;
 
-    const int8_t* brow = Bq + ((size_t)b * G + g) * N;
-    const int8_t* crow = Cq + ((size_t)b * G + g) * N;
-    const int8_t* xrow = x + bh * P;
-    uint4* st = reinterpret_cast<uint4*>(state_q + bh * P * N);
-    // every global load of the step is issued here, before anything waits on one: the codes
-    // (they stay in registers, a quarter of the floats; the update is recomputed for the
-    // requantisation, so registers, not ALU work, bound the CTAs with loads in flight), the
-    // token's x of this thread's rows, and the scalars
-    uint4 qv[CH];
-    float xq[CH];
+    // issue the copies of `it`'s chunks into stage `s` (one commit group), and return its x
+    auto prefetch = [&](int it, int s, float (&xq)[CH]) {
+        const int b = it / H, h = it % H, g = h / (H / G);
+        const uint4* st = reinterpret_cast<const uint4*>(state_q + (size_t)it * P * N);
+        const int8_t* xrow = x + (size_t)it * P;
 #pragma unroll
-    for (int k = 0; k < CH; ++k) {
-        const int u = tid + k * TPB;
-        const bool in = k * TPB < nchunks && u < nchunks;
-        qv[k] = in ? st[u] : make_uint4(0u, 0u, 0u, 0u);
-        xq[k] = in ? static_cast<float>(xrow[u / CPR]) : 0.f;
-    }
-    const float dtv = dt[bh];
-    const float decay = __expf(dtv * A[h]);
-    const float s_old = state_scale[bh];
-    const float sx = x_scale[h], sB = B_scale[g], sC = C_scale[g], Dh = D[h];
-    if (tid < 2 * CPR) {
-        const int cc = tid % CPR;
-        float v[16];
-        unpack16(*reinterpret_cast<const uint4*>((tid < CPR ? brow : crow) + 16 * cc), v);
-        float* dst = (tid < CPR ? sbv : scv) + 16 * cc;
-        const float sc = tid < CPR ? sB : sC;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) dst[i] = sc * v[i];
-    }
-    __syncthreads();
+        for (int k = 0; k < CH; ++k) {
+            const int u = tid + k * TPB;
+            const bool in = k * TPB < nchunks && u < nchunks;
+            if (in) cp_async16(&sq[s][k][tid], st + u);
+            xq[k] = in ? static_cast<float>(xrow[u / CPR]) : 0.f;
+        }
+        if (tid < 2 * CPR) {
+            const int8_t* row = (tid < CPR ? Bq : Cq) + ((size_t)b * G + g) * N;
+            cp_async16(&sbc[s][tid], row + 16 * (tid % CPR));
+        }
+        cp_async_commit();
+    };
 
-    const float ds = decay * s_old;  // decayed dequantisation factor
-    float amax = 0.f;
-    // the loop bound is warp-uniform (multiples of the CTA size) so that every lane reaches
-    // the shuffles
+    float xq[CH], xq_n[CH];
+    prefetch(item, 0, xq);
+    float dtv = dt[item], s_old = state_scale[item];
+    for (int it = 0;; ++it) {
+        const int s = it & 1;
+        const int next = item + gridDim.x;
+        float dt_n = 0.f, s_old_n = 0.f;
+        if (next < count) {
+            prefetch(next, s ^ 1, xq_n);
+            dt_n = dt[next];
+            s_old_n = state_scale[next];
+            cp_async_wait<1>();  // this item's group has landed (the next one may be in flight)
+        } else {
+            cp_async_wait<0>();
+        }
+        const int h = item % H, g = h / (H / G);
+        const float sx = x_scale[h], Dh = D[h];
+        const float decay = __expf(dtv * A[h]);
+        float4* sb = sbv[s];
+        float4* sc = scv[s];
+        if (tid < 2 * CPR) {
+            f2 v[8];
+            unpack16(sbc[s][tid], v);
+            const float sv = tid < CPR ? B_scale[g] : C_scale[g];
+            float4* dst = (tid < CPR ? sb : sc) + tid % CPR;
 #pragma unroll
-    for (int k = 0; k < CH; ++k) {
-        if (k * TPB >= nchunks) break;
-        const int u = tid + k * TPB;
-        const bool in = u < nchunks;
-        const int p = in ? u / CPR : 0, cc = u % CPR;
-        const float4* bq4 = reinterpret_cast<const float4*>(sbv + 16 * cc);
-        const float4* cq4 = reinterpret_cast<const float4*>(scv + 16 * cc);
-        float hv[16];
-        unpack16(qv[k], hv);
-        const float xv = sx * xq[k];
-        const float dx = dtv * xv;
-        float acc = 0.f;
+            for (int i = 0; i < 4; ++i)
+                dst[i * CPR] = make_float4(sv * v[2 * i].x, sv * v[2 * i].y, sv * v[2 * i + 1].x, sv * v[2 * i + 1].y);
+        }
+        __syncthreads();
+
+        const f2 ds = {decay * s_old, decay * s_old};  // decayed dequantisation factor
+        float amax = 0.f;
+        f2 hv[CH][8];
+        // the loop bound is warp-uniform (multiples of the CTA size) so that every lane reaches
+        // the shuffles
 #pragma unroll
-        for (int i4 = 0; i4 < 4; ++i4) {
-            const float4 b4 = bq4[i4], c4 = cq4[i4];
-            const float bb[4] = {b4.x, b4.y, b4.z, b4.w}, cc4[4] = {c4.x, c4.y, c4.z, c4.w};
+        for (int k = 0; k < CH; ++k) {
+            if (k * TPB >= nchunks) break;
+            const int u = tid + k * TPB;
+            const bool in = u < nchunks;
+            const int p = in ? u / CPR : 0, cc = u % CPR;
+            // (a thread past the last chunk copied nothing: its zero codes keep the max clean)
+            unpack16(in ? sq[s][k][tid] : make_uint4(0u, 0u, 0u, 0u), hv[k]);
+            const float xv = sx * xq[k];
+            const f2 dx = {dtv * xv, dtv * xv};
+            f2 acc = {0.f, 0.f};
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float v = fmaf(ds, hv[4 * i4 + j], dx * bb[j]);
-                acc = fmaf(cc4[j], v, acc);
-                amax = fmaxf(amax, fabsf(v));
+            for (int i = 0; i < 4; ++i) {
+                const float4 bb = sb[i * CPR + cc], cq = sc[i * CPR + cc];
+                hv[k][2 * i] = ffma2(ds, hv[k][2 * i], fmul2(dx, f2{bb.x, bb.y}));
+                hv[k][2 * i + 1] = ffma2(ds, hv[k][2 * i + 1], fmul2(dx, f2{bb.z, bb.w}));
+                acc = ffma2(f2{cq.x, cq.y}, hv[k][2 * i], acc);
+                acc = ffma2(f2{cq.z, cq.w}, hv[k][2 * i + 1], acc);
+                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(hv[k][2 * i].x), fabsf(hv[k][2 * i].y)),
+                                         fmaxf(fabsf(hv[k][2 * i + 1].x), fabsf(hv[k][2 * i + 1].y))));
             }
+            float a = acc.x + acc.y;
+#pragma unroll
+            for (int o = CPR / 2; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+            if (in && (lane % CPR) == 0) store_out(y, (size_t)item * P + p, a + Dh * xv, y_dtype, inv_y_scale);
         }
+        amax = block_max<TPB>(amax, scratch);
+        const float inv = amax > 0.f ? 127.f / amax : 0.f;
+        uint4* st = reinterpret_cast<uint4*>(state_q + (size_t)item * P * N);
 #pragma unroll
-        for (int o = CPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (in && (lane % CPR) == 0) store_out(y, bh * P + p, acc + Dh * xv, y_dtype, inv_y_scale);
-    }
-    amax = block_max<TPB>(amax, scratch);
-    const float inv = amax > 0.f ? 127.f / amax : 0.f;
-#pragma unroll
-    for (int k = 0; k < CH; ++k) {
-        if (k * TPB >= nchunks) break;
-        const int u = tid + k * TPB;
-        if (u >= nchunks) continue;
-        const int cc = u % CPR;
-        const float4* bq4 = reinterpret_cast<const float4*>(sbv + 16 * cc);
-        const float dx = dtv * (sx * xq[k]);
-        float hv[16];
-        unpack16(qv[k], hv);
-#pragma unroll
-        for (int i4 = 0; i4 < 4; ++i4) {
-            const float4 b4 = bq4[i4];
-            hv[4 * i4 + 0] = fmaf(ds, hv[4 * i4 + 0], dx * b4.x);
-            hv[4 * i4 + 1] = fmaf(ds, hv[4 * i4 + 1], dx * b4.y);
-            hv[4 * i4 + 2] = fmaf(ds, hv[4 * i4 + 2], dx * b4.z);
-            hv[4 * i4 + 3] = fmaf(ds, hv[4 * i4 + 3], dx * b4.w);
+        for (int k = 0; k < CH; ++k) {
+            if (k * TPB >= nchunks) break;
+            const int u = tid + k * TPB;
+            if (u < nchunks) st[u] = pack16(hv[k], inv);
         }
-        st[u] = pack16(hv, inv);
+        if (tid == 0) state_scale[item] = amax / 127.f;
+        if (next >= count) break;
+        item = next;
+        dtv = dt_n;
+        s_old = s_old_n;
+#pragma unroll
+        for (int k = 0; k < CH; ++k) xq[k] = xq_n[k];
     }
-    if (tid == 0) state_scale[bh] = amax / 127.f;
 }
 
 // fp32 state -> int8 codes + per-(batch, head) scale (the same rule as the update's requant)
@@ -223,14 +300,36 @@ cudaError_t with_shape(int nchunks, F&& f) {
     return f(std::integral_constant<int, 256>(), std::integral_constant<int, 4>());
 }
 
+// Resident CTAs of `kernel` on the current device (SMs x CTAs per SM), looked up once per
+// device and kernel.
+template <typename K>
+int resident_ctas(K kernel, int tpb) {
+    constexpr int kMaxDevices = 64;
+    static int cache[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+    if (cache[dev] == 0) {
+        int sms = 0, per_sm = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, tpb, 0) != cudaSuccess)
+            return 0;
+        cache[dev] = sms * (per_sm > 0 ? per_sm : 1);
+    }
+    return cache[dev];
+}
+
 template <int N>
 cudaError_t launch_q8_n(const StateUpdateQ8Args& a, cudaStream_t st) {
-    dim3 grid(a.nheads, a.batch);
+    const int count = a.batch * a.nheads;
     return with_shape(a.headdim * N / 16, [&](auto tpb, auto ch) {
-        state_update_q8_kernel<N, decltype(tpb)::value, decltype(ch)::value>
-            <<<grid, decltype(tpb)::value, 0, st>>>(
-                a.state_q, a.state_scale, a.x, a.B, a.C, a.dt, a.A, a.D, a.x_scale, a.B_scale,
-                a.C_scale, a.nheads, a.headdim, a.ngroups, a.y, a.y_dtype, a.inv_y_scale);
+        constexpr int TPB = decltype(tpb)::value, CH = decltype(ch)::value;
+        auto kernel = state_update_q8_kernel<N, TPB, CH>;
+        const int resident = resident_ctas(kernel, TPB);
+        if (resident <= 0) return cudaErrorUnknown;
+        const int grid = count < resident ? count : resident;
+        kernel<<<grid, TPB, 0, st>>>(a.state_q, a.state_scale, a.x, a.B, a.C, a.dt, a.A, a.D,
+                                     a.x_scale, a.B_scale, a.C_scale, count, a.nheads, a.headdim,
+                                     a.ngroups, a.y, a.y_dtype, a.inv_y_scale);
         return cudaGetLastError();
     });
 }
