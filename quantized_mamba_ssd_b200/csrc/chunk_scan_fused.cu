@@ -251,13 +251,13 @@ __device__ __forceinline__ f2 fsub2(f2 a, f2 b) {
     return r;
 }
 
-// In-place Walsh-Hadamard transform of 64 values (Sylvester order, unnormalised):
+// In-place Walsh-Hadamard transform of 32 values (Sylvester order, unnormalised):
 // v[q] <- sum_p (-1)^popcount(p & q) v[p].  Butterflies two at a time in packed pairs.
-__device__ __forceinline__ void fwht64(float (&v)[64]) {
+__device__ __forceinline__ void fwht32(float (&v)[32]) {
 #pragma unroll
-    for (int hs = 1; hs < 64; hs <<= 1) {
+    for (int hs = 1; hs < 32; hs <<= 1) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
+        for (int i = 0; i < 32; ++i) {
             // butterfly (i, i + hs) for i with bit hs clear, two of them per packed op: i and
             // the next such i (i + 1 when hs > 1, i + 2 when hs == 1)
             const int step = hs == 1 ? 2 : 1;
@@ -685,72 +685,86 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
         // this worker's previous block, whose output is pending
         int pv_tok = 0, pv_h = 0, pv_valid = 0;  // first packed token of the block
         float pv_rho = 1.f, last_U = 1.f;
+        // 32 output values of this thread's row (columns [32 hq, 32 hq + 32)), times s, in the
+        // output dtype
+        auto store32 = [&](const float (&v)[32], float s, size_t ybase, int hq) {
+            if constexpr (YT == SSD_OUT_I8) {
+                // q = clamp(rint(fp32(acc * s / s_y))): the same rounding as the fp32 output
+                const float sc = s * p.inv_y_scale;
+                const f2 s2 = {sc, sc}, rnd = {kRound, kRound};
+                uint32_t wv[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const f2 v0 = fadd2(fmul2(f2{v[4 * q], v[4 * q + 1]}, s2), rnd);
+                    const f2 v1 = fadd2(fmul2(f2{v[4 * q + 2], v[4 * q + 3]}, s2), rnd);
+                    const uint32_t lo = __byte_perm(clamp_code(v0.x), clamp_code(v0.y), 0x0040);
+                    const uint32_t hi = __byte_perm(clamp_code(v1.x), clamp_code(v1.y), 0x0040);
+                    wv[q] = __byte_perm(lo, hi, 0x5410);
+                }
+                uint4* yo = reinterpret_cast<uint4*>(static_cast<int8_t*>(p.y) + ybase) + 2 * hq;
+                yo[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                yo[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+            } else if constexpr (YT == SSD_OUT_F16) {
+                const f2 s2 = {s, s};
+                uint4* yo = reinterpret_cast<uint4*>(static_cast<__half*>(p.y) + ybase) + 4 * hq;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t wq4[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const f2 t = fmul2(f2{v[8 * q + 2 * i], v[8 * q + 2 * i + 1]}, s2);
+                        wq4[i] = pack_f16x2(t.x, t.y);
+                    }
+                    yo[q] = make_uint4(wq4[0], wq4[1], wq4[2], wq4[3]);
+                }
+            } else {
+                const f2 s2 = {s, s};
+                float4* yo = reinterpret_cast<float4*>(static_cast<float*>(p.y) + ybase) + 8 * hq;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const f2 t0 = fmul2(f2{v[4 * q], v[4 * q + 1]}, s2);
+                    const f2 t1 = fmul2(f2{v[4 * q + 2], v[4 * q + 3]}, s2);
+                    yo[q] = make_float4(t0.x, t0.y, t1.x, t1.y);
+                }
+            }
+        };
         auto output = [&](int kb) {
             wait_phase(bars + kBarAcc0 + w, (kb >> 1) & 1, abort_flag, p);
             tc_fence_after();
             const size_t ybase = ((size_t)(pv_tok + row) * p.H + pv_h) * kP;
             const bool store = row < pv_valid;
             if constexpr (HAD) {
-                // y' = H y / 8 over the 64 head channels before the dtype conversion: the whole
-                // row in registers, a butterfly transform, the 1/8 folded into the scale
-                float v[64];
+                // y' = H y / 8 with H = [[H32, H32], [H32, -H32]] (Sylvester): columns [0, 32) of
+                // y' are H32 (y_lo + y_hi), columns [32, 64) are H32 (y_lo - y_hi); one compact
+                // loop over the two halves, the 1/8 folded into the scale
+                float sv[32], dv[32];
                 {
                     uint32_t r0[32], r1[32];
                     tmem_ld32(tmem_addr(tmem, lane_base, col_acc), r0);
                     tmem_ld32(tmem_addr(tmem, lane_base, col_acc + 32), r1);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        v[i] = __uint_as_float(r0[i]);
-                        v[32 + i] = __uint_as_float(r1[i]);
+                    for (int i = 0; i < 16; ++i) {
+                        const f2 a = {__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1])};
+                        const f2 b = {__uint_as_float(r1[2 * i]), __uint_as_float(r1[2 * i + 1])};
+                        const f2 su = fadd2(a, b), di = fsub2(a, b);
+                        sv[2 * i] = su.x;
+                        sv[2 * i + 1] = su.y;
+                        dv[2 * i] = di.x;
+                        dv[2 * i + 1] = di.y;
                     }
                 }
                 tc_fence_before();
                 wg_sync(bar_id);
                 if (row == 0) mbar_arrive(bars + kBarAccFree0 + w);
                 if (!store) return;
-                fwht64(v);
                 const float rs = pv_rho * 0.125f;
-                if constexpr (YT == SSD_OUT_I8) {
-                    const float sc = rs * p.inv_y_scale;
-                    const f2 s2 = {sc, sc}, rnd = {kRound, kRound};
-                    uint4* yo = reinterpret_cast<uint4*>(static_cast<int8_t*>(p.y) + ybase);
+#pragma unroll 1
+                for (int hq = 0; hq < 2; ++hq) {
+                    fwht32(sv);
+                    store32(sv, rs, ybase, hq);
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        uint32_t wv[4];
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const int o = 16 * q4 + 4 * q;
-                            const f2 v0 = fadd2(fmul2(f2{v[o], v[o + 1]}, s2), rnd);
-                            const f2 v1 = fadd2(fmul2(f2{v[o + 2], v[o + 3]}, s2), rnd);
-                            const uint32_t lo = __byte_perm(clamp_code(v0.x), clamp_code(v0.y), 0x0040);
-                            const uint32_t hi = __byte_perm(clamp_code(v1.x), clamp_code(v1.y), 0x0040);
-                            wv[q] = __byte_perm(lo, hi, 0x5410);
-                        }
-                        yo[q4] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-                    }
-                } else if constexpr (YT == SSD_OUT_F16) {
-                    const f2 s2 = {rs, rs};
-                    uint4* yo = reinterpret_cast<uint4*>(static_cast<__half*>(p.y) + ybase);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        uint32_t wq4[4];
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const f2 t = fmul2(f2{v[8 * q + 2 * i], v[8 * q + 2 * i + 1]}, s2);
-                            wq4[i] = pack_f16x2(t.x, t.y);
-                        }
-                        yo[q] = make_uint4(wq4[0], wq4[1], wq4[2], wq4[3]);
-                    }
-                } else {
-                    const f2 s2 = {rs, rs};
-                    float4* yo = reinterpret_cast<float4*>(static_cast<float*>(p.y) + ybase);
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const f2 t0 = fmul2(f2{v[4 * q], v[4 * q + 1]}, s2);
-                        const f2 t1 = fmul2(f2{v[4 * q + 2], v[4 * q + 3]}, s2);
-                        yo[q] = make_float4(t0.x, t0.y, t1.x, t1.y);
-                    }
+                    for (int i = 0; i < 32; ++i) sv[i] = dv[i];
                 }
             } else {
                 // two halves of 32 columns: a compact loop
@@ -760,45 +774,10 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                     tmem_ld32(tmem_addr(tmem, lane_base, col_acc + 32 * hq), r);
                     tmem_ld_wait();
                     if (!store) continue;
-                    if constexpr (YT == SSD_OUT_I8) {
-                        // q = clamp(rint(fp32(acc * rho / s_y))): the same rounding as the fp32 output
-                        const float sc = pv_rho * p.inv_y_scale;
-                        const f2 s2 = {sc, sc}, rnd = {kRound, kRound};
-                        uint32_t wv[8];
+                    float v[32];
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            const f2 v0 = fadd2(fmul2(f2{__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1])}, s2), rnd);
-                            const f2 v1 = fadd2(fmul2(f2{__uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])}, s2), rnd);
-                            const uint32_t lo = __byte_perm(clamp_code(v0.x), clamp_code(v0.y), 0x0040);
-                            const uint32_t hi = __byte_perm(clamp_code(v1.x), clamp_code(v1.y), 0x0040);
-                            wv[q] = __byte_perm(lo, hi, 0x5410);
-                        }
-                        uint4* yo = reinterpret_cast<uint4*>(static_cast<int8_t*>(p.y) + ybase) + 2 * hq;
-                        yo[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-                        yo[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
-                    } else if constexpr (YT == SSD_OUT_F16) {
-                        const f2 s2 = {pv_rho, pv_rho};
-                        uint4* yo = reinterpret_cast<uint4*>(static_cast<__half*>(p.y) + ybase) + 4 * hq;
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint32_t wq4[4];
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const f2 v = fmul2(f2{__uint_as_float(r[8 * q + 2 * i]), __uint_as_float(r[8 * q + 2 * i + 1])}, s2);
-                                wq4[i] = pack_f16x2(v.x, v.y);
-                            }
-                            yo[q] = make_uint4(wq4[0], wq4[1], wq4[2], wq4[3]);
-                        }
-                    } else {
-                        const f2 s2 = {pv_rho, pv_rho};
-                        float4* yo = reinterpret_cast<float4*>(static_cast<float*>(p.y) + ybase) + 8 * hq;
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            const f2 v0 = fmul2(f2{__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1])}, s2);
-                            const f2 v1 = fmul2(f2{__uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])}, s2);
-                            yo[q] = make_float4(v0.x, v0.y, v1.x, v1.y);
-                        }
-                    }
+                    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+                    store32(v, pv_rho, ybase, hq);
                 }
                 tc_fence_before();
                 wg_sync(bar_id);
