@@ -47,7 +47,7 @@ INT8_PER_BF16 = 2.0  # nominal dense int8 : bf16 tensor throughput ratio on B200
 # profiles/ncu_fused_chunk_scan_b2_L8192.md.  The traffic grows in proportion to the tokens of a
 # launch, so the bench scales it to the workload.  A changed kernel reports null.
 _CAPTURED_TRAFFIC_PER_TOKEN = {
-    "0897cbf91d4a87655447f0345ea36cd509618e0dd9275c23ef15d871cc86a1ac": (339.209472e6 + 119.024640e6) / 16384,
+    "908438e75786a1238d8443323545ff01890339c19ad4aa2c80502b385ada0975": (342.448384e6 + 118.953984e6) / 16384,
 }
 
 
