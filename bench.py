@@ -37,6 +37,7 @@ PER_TENSOR_CFG = 4  # the same layer under the per-tensor percentile-clipped rec
 METRIC = "SSD scan tokens/s (int8 in) at 1 B200; achieved fraction of HBM/int8 roofline"
 UNIT = "tokens/s"
 INT8_PER_BF16 = 2.0  # nominal dense int8 : bf16 tensor throughput ratio on B200 (4.5 : 2.25)
+NOMINAL_HBM_GBS = 7700.0  # B200 HBM3e datasheet bandwidth (HGX), context for the measured peak
 
 
 # ------------------------------------------------------------------------------------------
@@ -342,9 +343,9 @@ def main():
 
     # ---- end to end: pinned host inputs in, int8 output back, every step ----
     hx, hB, hC, hdt = (torch.from_numpy(a).pin_memory() for a in (case.x, case.B, case.C, case.dt))
-    hy = torch.empty((bsz, L, H, P), dtype=torch.int8).pin_memory()
+    hys = [torch.empty((bsz, L, H, P), dtype=torch.int8).pin_memory() for _ in range(2)]
     h2d = sum(t_.numel() * t_.element_size() for t_ in (hx, hB, hC, hdt))
-    d2h = hy.numel() * hy.element_size()
+    d2h = hys[0].numel() * hys[0].element_size()
 
     def e2e_step():
         x.copy_(hx, non_blocking=True)
@@ -352,11 +353,12 @@ def main():
         C.copy_(hC, non_blocking=True)
         dt.copy_(hdt, non_blocking=True)
         step()
-        hy.copy_(y, non_blocking=True)
+        hys[0].copy_(y, non_blocking=True)
 
     e2e = None
     if not args.no_e2e:
         e2e_steps = max(3, min(args.steps, 10))
+        # serial: copy in, scan, copy out, one after the other on one stream
         for _ in range(3):
             e2e_step()
         torch.cuda.synchronize()
@@ -367,9 +369,53 @@ def main():
         ev1.record(stream)
         torch.cuda.synchronize()
         barrier()
+        serial_ms = max_over_ranks(ev0.elapsed_time(ev1) / e2e_steps, dev)
+        # pipelined: step i's inputs go up on one copy stream while step i - 1 computes and step
+        # i - 2's output comes down on another (two device buffer sets, two host output buffers)
+        bufs = [(x, B, C, dt, y), tuple(torch.empty_like(t_) for t_ in (x, B, C, dt, y))]
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+
+        def e2e_pipe(i):
+            j = i % 2
+            bx, bB, bC, bdt, by = bufs[j]
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(ev_done[j])  # the scan of step i - 2 has read buffer j
+                for dst, src in ((bx, hx), (bB, hB), (bC, hC), (bdt, hdt)):
+                    dst.copy_(src, non_blocking=True)
+                ev_in[j].record(s_in)
+            stream.wait_event(ev_in[j])
+            stream.wait_event(ev_out[j])  # step i - 2's output has left buffer j
+            ssd_i8.ssd_i8_chunk_scan(bx, bB, bC, bdt, A, Dp, sx, sb, sc, Q, final_state=fs, y=by,
+                                     y_dtype="i8", y_scale=y_scale, workspace=ws)
+            ev_done[j].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_done[j])
+                hys[j].copy_(by, non_blocking=True)
+                ev_out[j].record(s_out)
+
+        for i in range(3):
+            e2e_pipe(i)
+        torch.cuda.synchronize()
+        barrier()
+        ev0.record(stream)
+        s_in.wait_event(ev0)
+        for i in range(e2e_steps):
+            e2e_pipe(i)
+        for j in range(2):
+            stream.wait_event(ev_out[j])
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
         e2e_ms = max_over_ranks(ev0.elapsed_time(ev1) / e2e_steps, dev)
         e2e = {"value": aggregate_tokens_per_s(bsz * L, world, e2e_ms), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e2e_ms, "pipelined": True,
+               "serial_value": aggregate_tokens_per_s(bsz * L, world, serial_ms),
+               "serial_ms_per_step": serial_ms}
+        del bufs
 
     # ---- the per-tensor static recipe on the same layer: x clipped at the 99.99th percentile,
     # B and C per-tensor absmax (same shapes, so the same algorithmic bytes) ----
@@ -423,6 +469,7 @@ def main():
         "alg_bytes_per_launch": alg_bytes, "alg_int8_ops_per_launch": alg_ops,
         "roofline_us": 1e6 * max(t_hbm, t_ops), "frac_of_roofline_time": 1e6 * max(t_hbm, t_ops) / (ms * 1e3),
         "int8_peak_tops": int8_peak_tops,
+        "nominal_hbm_gbs": NOMINAL_HBM_GBS, "frac_of_nominal_hbm": achieved_gbs / NOMINAL_HBM_GBS,
     }
 
     had_gbs = alg_bytes / (had_ms * 1e-3) / 1e9

@@ -285,6 +285,8 @@ def make_prefill_config(index: int, seed: Optional[int] = None, **overrides) -> 
     spec = dict(PREFILL_CONFIGS[index])
     spec.update(overrides)
     name = spec.pop("name")
+    if overrides:  # a smaller case of the same shape (profiling captures) says so in its name
+        name += " [" + ", ".join(f"{k}={v}" for k, v in sorted(overrides.items())) + "]"
     return make_prefill(seed=1000 + index if seed is None else seed, name=name, **spec)
 
 
@@ -318,4 +320,6 @@ def make_decode_config(seed: Optional[int] = None, **overrides) -> DecodeCase:
     spec = dict(DECODE_CONFIG)
     spec.update(overrides)
     name = spec.pop("name")
+    if overrides:
+        name += " [" + ", ".join(f"{k}={v}" for k, v in sorted(overrides.items())) + "]"
     return make_decode(seed=1004 if seed is None else seed, name=name, **spec)
