@@ -51,12 +51,14 @@ typedef enum ssd_status {
 typedef enum ssd_out_dtype { SSD_OUT_F32 = 0, SSD_OUT_F16 = 1, SSD_OUT_I8 = 2 } ssd_out_dtype;
 
 /*
- * Flag OR-ed into the y_dtype of ssd_i8_chunk_scan / _varlen / _noalloc: the output is
- * y' = H y / 8 per (token, head) over the 64 head channels (H the 64 x 64 Hadamard matrix in
+ * Flag OR-ed into the y_dtype of ssd_i8_chunk_scan / _varlen / _noalloc and of the decode steps
+ * ssd_i8_state_update / _q8: the output is y' = H y / 8 per (token, head) over the 64 head
+ * channels (H the 64 x 64 Hadamard matrix in
  * Sylvester order, H[q][p] = (-1)^popcount(p & q), so y' is an orthonormal transform of y),
  * applied before the conversion to y_dtype -- the Hadamard transform of the SSD output ahead of
  * out_proj that the Quamba2 OpenReview rebuttal uses with its Table R10 runs, fused into the
- * kernel's epilogue.  For SSD_OUT_I8, y_scale quantises y'.  Requires headdim 64.
+ * kernel's epilogue.  For SSD_OUT_I8, y_scale quantises y'.  Requires headdim 64 (else
+ * SSD_ERR_UNSUPPORTED).  The states are not affected.
  */
 #define SSD_OUT_HADAMARD 16
 

@@ -194,10 +194,10 @@ ssd_status ssd_i8_state_update(float* state, const int8_t* x, const int8_t* B, c
                                int batch, int nheads, int headdim, int dstate, int ngroups,
                                void* y, int y_dtype, float y_scale, void* stream) {
     if (batch < 0 || nheads <= 0 || headdim <= 0 || dstate <= 0 || ngroups <= 0 ||
-        nheads % ngroups != 0 || !valid_out_dtype(y_dtype))
+        nheads % ngroups != 0 || !valid_scan_out(y_dtype))
         return SSD_ERR_INVALID_ARG;
     if (!(dstate == 16 || dstate == 32 || dstate == 64 || dstate == 128 || dstate == 256) ||
-        headdim > 256)
+        headdim > 256 || ((y_dtype & SSD_OUT_HADAMARD) && headdim != 64))
         return SSD_ERR_UNSUPPORTED;
     float inv = 1.f;
     if (!out_scale(y_dtype, y_scale, &inv)) return SSD_ERR_INVALID_ARG;
@@ -205,7 +205,8 @@ ssd_status ssd_i8_state_update(float* state, const int8_t* x, const int8_t* B, c
     if (!state || !x || !B || !C || !dt || !A || !D || !x_scale || !B_scale || !C_scale || !y)
         return SSD_ERR_INVALID_ARG;
     ssd::StateUpdateArgs a{state, x, B, C, dt, A, D, x_scale, B_scale, C_scale, batch, nheads,
-                           headdim, dstate, ngroups, y, y_dtype, inv};
+                           headdim, dstate, ngroups, y, y_dtype & ~SSD_OUT_HADAMARD, inv,
+                           (y_dtype & SSD_OUT_HADAMARD) ? 1 : 0};
     return ssd::launch_state_update(a, static_cast<cudaStream_t>(stream)) == cudaSuccess
                ? SSD_OK
                : SSD_ERR_CUDA;
@@ -231,9 +232,11 @@ ssd_status ssd_i8_state_update_q8(int8_t* state_q, float* state_scale, const int
                                   int nheads, int headdim, int dstate, int ngroups, void* y,
                                   int y_dtype, float y_scale, void* stream) {
     if (batch < 0 || nheads <= 0 || headdim <= 0 || dstate <= 0 || ngroups <= 0 ||
-        nheads % ngroups != 0 || !valid_out_dtype(y_dtype))
+        nheads % ngroups != 0 || !valid_scan_out(y_dtype))
         return SSD_ERR_INVALID_ARG;
-    if (!ssd::state_q8_shape_ok(headdim, dstate)) return SSD_ERR_UNSUPPORTED;
+    if (!ssd::state_q8_shape_ok(headdim, dstate) ||
+        ((y_dtype & SSD_OUT_HADAMARD) && headdim != 64))
+        return SSD_ERR_UNSUPPORTED;
     float inv = 1.f;
     if (!out_scale(y_dtype, y_scale, &inv)) return SSD_ERR_INVALID_ARG;
     if (batch == 0) return SSD_OK;
@@ -242,7 +245,8 @@ ssd_status ssd_i8_state_update_q8(int8_t* state_q, float* state_scale, const int
         return SSD_ERR_INVALID_ARG;
     if (!aligned16(state_q) || !aligned16(B) || !aligned16(C)) return SSD_ERR_INVALID_ARG;
     ssd::StateUpdateQ8Args a{state_q, state_scale, x, B, C, dt, A, D, x_scale, B_scale,
-                             C_scale, batch, nheads, headdim, dstate, ngroups, y, y_dtype, inv};
+                             C_scale, batch, nheads, headdim, dstate, ngroups, y,
+                             y_dtype & ~SSD_OUT_HADAMARD, inv, (y_dtype & SSD_OUT_HADAMARD) ? 1 : 0};
     return ssd::launch_state_update_q8(a, static_cast<cudaStream_t>(stream)) == cudaSuccess
                ? SSD_OK
                : SSD_ERR_CUDA;

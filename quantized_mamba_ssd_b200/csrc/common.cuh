@@ -67,4 +67,25 @@ __device__ __forceinline__ void store_out(void* y, size_t idx, float v, int dtyp
     }
 }
 
+// y' = H y / 8 of the 64 values ys[0..63] (H the Sylvester-ordered 64 x 64 Hadamard matrix,
+// H = [[H32, H32], [H32, -H32]]), stored at y[ybase + q] in the output dtype.  Called by one
+// whole warp: lane l holds y'[l] = H32 (y_lo + y_hi) and y'[l + 32] = H32 (y_lo - y_hi), the
+// 32-point transforms as five butterfly stages across the lanes.
+__device__ __forceinline__ void hadamard64_store(const float* ys, void* y, size_t ybase, int dtype,
+                                                 float inv_scale) {
+    const int lane = threadIdx.x & (kWarp - 1);
+    const float a = ys[lane], b = ys[lane + 32];
+    float s = a + b, d = a - b;
+#pragma unroll
+    for (int hs = 16; hs >= 1; hs >>= 1) {
+        const float ps = __shfl_xor_sync(0xffffffffu, s, hs);
+        const float pd = __shfl_xor_sync(0xffffffffu, d, hs);
+        const bool upper = (lane & hs) != 0;  // element i + hs of the butterfly (i, i + hs)
+        s = upper ? ps - s : s + ps;
+        d = upper ? pd - d : d + pd;
+    }
+    store_out(y, ybase + lane, 0.125f * s, dtype, inv_scale);
+    store_out(y, ybase + lane + 32, 0.125f * d, dtype, inv_scale);
+}
+
 }  // namespace ssd

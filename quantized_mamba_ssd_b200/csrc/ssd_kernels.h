@@ -47,8 +47,9 @@ struct StateUpdateArgs {
     const float* C_scale;
     int batch, nheads, headdim, dstate, ngroups;
     void* y;
-    int y_dtype;
+    int y_dtype;  // SSD_OUT_* without the Hadamard flag
     float inv_y_scale;
+    int hadamard;  // 1: y' = H y / 8 over headdim (64) before the conversion
 };
 
 struct StateUpdateQ8Args {
@@ -65,8 +66,9 @@ struct StateUpdateQ8Args {
     const float* C_scale;
     int batch, nheads, headdim, dstate, ngroups;
     void* y;
-    int y_dtype;
+    int y_dtype;  // SSD_OUT_* without the Hadamard flag
     float inv_y_scale;
+    int hadamard;  // 1: y' = H y / 8 over headdim (64) before the conversion
 };
 
 size_t chunk_scan_workspace_bytes(int batch, int seqlen, int nheads, int headdim, int dstate,

@@ -14,7 +14,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kUnroll = 4;  // rows in flight per lane
 
-template <int N>
+template <int N, bool HAD>
 __global__ void __launch_bounds__(kThreads)
 state_update_kernel(float* __restrict__ state, const int8_t* __restrict__ x,
                     const int8_t* __restrict__ Bq, const int8_t* __restrict__ Cq,
@@ -22,6 +22,7 @@ state_update_kernel(float* __restrict__ state, const int8_t* __restrict__ x,
                     const float* __restrict__ D, const float* __restrict__ x_scale,
                     const float* __restrict__ B_scale, const float* __restrict__ C_scale,
                     int H, int P, int G, void* __restrict__ y, int y_dtype, float inv_y_scale) {
+    __shared__ float ys[HAD ? 64 : 1];  // y of this (batch, head) to be transformed (P = 64)
     constexpr int VEC = N / 4;                          // float4 per state row
     constexpr int LPR = VEC < kWarp ? VEC : kWarp;      // lanes per row
     constexpr int VPL = VEC / LPR;                      // float4 per lane per row
@@ -82,18 +83,25 @@ state_update_kernel(float* __restrict__ state, const int8_t* __restrict__ x,
             }
 #pragma unroll
             for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-            if (sub == 0 && p < P) store_out(y, ybase + p, acc + Dh * xv, y_dtype, inv_y_scale);
+            if (sub == 0 && p < P) {
+                if constexpr (HAD) ys[p] = acc + Dh * xv;
+                else store_out(y, ybase + p, acc + Dh * xv, y_dtype, inv_y_scale);
+            }
         }
+    }
+    if constexpr (HAD) {
+        __syncthreads();
+        if (warp == 0) hadamard64_store(ys, y, ybase, y_dtype, inv_y_scale);
     }
 }
 
 template <int N>
 cudaError_t launch_n(const StateUpdateArgs& a, cudaStream_t st) {
     dim3 grid(a.nheads, a.batch);
-    state_update_kernel<N><<<grid, kThreads, 0, st>>>(a.state, a.x, a.B, a.C, a.dt, a.A, a.D,
-                                                      a.x_scale, a.B_scale, a.C_scale, a.nheads,
-                                                      a.headdim, a.ngroups, a.y, a.y_dtype,
-                                                      a.inv_y_scale);
+    auto kernel = a.hadamard ? state_update_kernel<N, true> : state_update_kernel<N, false>;
+    kernel<<<grid, kThreads, 0, st>>>(a.state, a.x, a.B, a.C, a.dt, a.A, a.D, a.x_scale, a.B_scale,
+                                      a.C_scale, a.nheads, a.headdim, a.ngroups, a.y, a.y_dtype,
+                                      a.inv_y_scale);
     return cudaGetLastError();
 }
 

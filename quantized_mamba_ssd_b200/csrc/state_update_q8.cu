@@ -130,7 +130,7 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 // into its private slots of a two-stage shared buffer while it computes the current one, so
 // the loads stay in flight without holding registers; the current item's update is kept in
 // registers between the y / max pass and the requantisation.
-template <int N, int TPB, int CH>
+template <int N, int TPB, int CH, bool HAD>
 __global__ void __launch_bounds__(TPB, (CH >= 4 ? 512 : 640) / TPB)  // the update in registers
 state_update_q8_kernel(int8_t* __restrict__ state_q, float* __restrict__ state_scale,
                        const int8_t* __restrict__ x, const int8_t* __restrict__ Bq,
@@ -147,6 +147,9 @@ state_update_q8_kernel(int8_t* __restrict__ state_q, float* __restrict__ state_s
     // copies in flight: [stage][chunk k][thread] state chunks, [stage][thread < 2 CPR] B/C chunks
     __shared__ __align__(16) uint4 sq[2][CH][TPB];
     __shared__ __align__(16) uint4 sbc[2][2 * CPR];
+    // y of the current item when it is Hadamard-transformed (P = 64); it is rewritten only
+    // after the next item's staging barrier, which the transforming warp 0 reaches last
+    __shared__ float ys[HAD ? 64 : 1];
     const int tid = threadIdx.x, lane = tid & (kWarp - 1);
     const int nchunks = P * CPR;
     int item = blockIdx.x;
@@ -231,9 +234,15 @@ state_update_q8_kernel(int8_t* __restrict__ state_q, float* __restrict__ state_s
             float a = acc.x + acc.y;
 #pragma unroll
             for (int o = CPR / 2; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-            if (in && (lane % CPR) == 0) store_out(y, (size_t)item * P + p, a + Dh * xv, y_dtype, inv_y_scale);
+            if (in && (lane % CPR) == 0) {
+                if constexpr (HAD) ys[p] = a + Dh * xv;
+                else store_out(y, (size_t)item * P + p, a + Dh * xv, y_dtype, inv_y_scale);
+            }
         }
-        amax = block_max<TPB>(amax, scratch);
+        amax = block_max<TPB>(amax, scratch);  // (its barrier also completes ys)
+        if constexpr (HAD) {
+            if (tid < kWarp) hadamard64_store(ys, y, (size_t)item * P, y_dtype, inv_y_scale);
+        }
         const float inv = amax > 0.f ? 127.f / amax : 0.f;
         uint4* st = reinterpret_cast<uint4*>(state_q + (size_t)item * P * N);
 #pragma unroll
@@ -300,10 +309,10 @@ cudaError_t with_shape(int nchunks, F&& f) {
     return f(std::integral_constant<int, 256>(), std::integral_constant<int, 4>());
 }
 
-// Resident CTAs of `kernel` on the current device (SMs x CTAs per SM), looked up once per
-// device and kernel.
-template <typename K>
-int resident_ctas(K kernel, int tpb) {
+// Resident CTAs of state_update_q8_kernel<N, TPB, CH, HAD> on the current device (SMs x CTAs
+// per SM), looked up once per device and instantiation.
+template <int N, int TPB, int CH, bool HAD>
+int resident_ctas() {
     constexpr int kMaxDevices = 64;
     static int cache[kMaxDevices] = {};
     int dev = 0;
@@ -311,27 +320,32 @@ int resident_ctas(K kernel, int tpb) {
     if (cache[dev] == 0) {
         int sms = 0, per_sm = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, tpb, 0) != cudaSuccess)
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                &per_sm, state_update_q8_kernel<N, TPB, CH, HAD>, TPB, 0) != cudaSuccess)
             return 0;
         cache[dev] = sms * (per_sm > 0 ? per_sm : 1);
     }
     return cache[dev];
 }
 
-template <int N>
-cudaError_t launch_q8_n(const StateUpdateQ8Args& a, cudaStream_t st) {
+template <int N, bool HAD>
+cudaError_t launch_q8_nh(const StateUpdateQ8Args& a, cudaStream_t st) {
     const int count = a.batch * a.nheads;
     return with_shape(a.headdim * N / 16, [&](auto tpb, auto ch) {
         constexpr int TPB = decltype(tpb)::value, CH = decltype(ch)::value;
-        auto kernel = state_update_q8_kernel<N, TPB, CH>;
-        const int resident = resident_ctas(kernel, TPB);
+        const int resident = resident_ctas<N, TPB, CH, HAD>();
         if (resident <= 0) return cudaErrorUnknown;
         const int grid = count < resident ? count : resident;
-        kernel<<<grid, TPB, 0, st>>>(a.state_q, a.state_scale, a.x, a.B, a.C, a.dt, a.A, a.D,
-                                     a.x_scale, a.B_scale, a.C_scale, count, a.nheads, a.headdim,
-                                     a.ngroups, a.y, a.y_dtype, a.inv_y_scale);
+        state_update_q8_kernel<N, TPB, CH, HAD><<<grid, TPB, 0, st>>>(
+            a.state_q, a.state_scale, a.x, a.B, a.C, a.dt, a.A, a.D, a.x_scale, a.B_scale,
+            a.C_scale, count, a.nheads, a.headdim, a.ngroups, a.y, a.y_dtype, a.inv_y_scale);
         return cudaGetLastError();
     });
+}
+
+template <int N>
+cudaError_t launch_q8_n(const StateUpdateQ8Args& a, cudaStream_t st) {
+    return a.hadamard ? launch_q8_nh<N, true>(a, st) : launch_q8_nh<N, false>(a, st);
 }
 
 template <int N>

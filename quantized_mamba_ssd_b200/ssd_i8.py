@@ -267,9 +267,10 @@ def ssd_i8_state_update(state: torch.Tensor, x: torch.Tensor, B: torch.Tensor, C
                         dt: torch.Tensor, A: torch.Tensor, D: torch.Tensor,
                         x_scale: torch.Tensor, B_scale: torch.Tensor, C_scale: torch.Tensor, *,
                         y: Optional[torch.Tensor] = None, y_dtype: str = "f16",
-                        y_scale: float = 1.0, stream=None) -> torch.Tensor:
+                        y_scale: float = 1.0, stream=None, hadamard: bool = False) -> torch.Tensor:
     """One decode step, state f32 [b,h,p,n] updated in place; x int8 [b,h,p]; B, C int8
-    [b,g,n]; dt f32 [b,h].  Returns y [b,h,p] of ``y_dtype``."""
+    [b,g,n]; dt f32 [b,h].  Returns y [b,h,p] of ``y_dtype`` (``hadamard``: y' = H y / 8 over
+    headdim, ``SSD_OUT_HADAMARD``)."""
     bsz, H, P, N = state.shape
     G = B.shape[1]
     code, tdt = OUT_DTYPES[y_dtype]
@@ -288,7 +289,7 @@ def ssd_i8_state_update(state: torch.Tensor, x: torch.Tensor, B: torch.Tensor, C
         _ptr(C_scale, "C_scale", torch.float32, (G,)),
         bsz, H, P, N, G,
         _ptr(y, "y", tdt, (bsz, H, P)),
-        code, float(y_scale),
+        code | (OUT_HADAMARD if hadamard else 0), float(y_scale),
         _stream(stream),
     ]
     _check("ssd_i8_state_update", library().ssd_i8_state_update(*args))
@@ -317,11 +318,12 @@ def ssd_i8_state_update_q8(state_q: torch.Tensor, state_scale: torch.Tensor, x: 
                            D: torch.Tensor, x_scale: torch.Tensor, B_scale: torch.Tensor,
                            C_scale: torch.Tensor, *, y: Optional[torch.Tensor] = None,
                            y_dtype: str = "f16", y_scale: float = 1.0,
-                           stream=None) -> torch.Tensor:
+                           stream=None, hadamard: bool = False) -> torch.Tensor:
     """One decode step on the int8 cached state, in place (see ``ssd_i8_state_update_q8``).
 
     state_q int8 [b,h,p,n] and state_scale f32 [b,h] are updated; x int8 [b,h,p]; B, C int8
-    [b,g,n]; dt f32 [b,h]; returns y [b,h,p] of ``y_dtype``."""
+    [b,g,n]; dt f32 [b,h]; returns y [b,h,p] of ``y_dtype`` (``hadamard``: y' = H y / 8 over
+    headdim)."""
     bsz, H, P, N = state_q.shape
     G = B.shape[1]
     code, tdt = OUT_DTYPES[y_dtype]
@@ -341,7 +343,7 @@ def ssd_i8_state_update_q8(state_q: torch.Tensor, state_scale: torch.Tensor, x: 
         _ptr(C_scale, "C_scale", torch.float32, (G,)),
         bsz, H, P, N, G,
         _ptr(y, "y", tdt, (bsz, H, P)),
-        code, float(y_scale),
+        code | (OUT_HADAMARD if hadamard else 0), float(y_scale),
         _stream(stream),
     ]
     _check("ssd_i8_state_update_q8", library().ssd_i8_state_update_q8(*args))

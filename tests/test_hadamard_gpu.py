@@ -141,3 +141,67 @@ def test_hadamard_at_workload_size_sampled():
     yq, _ = run(case, y_dtype="i8", y_scale=s_y)
     for (b, h), r in refs.items():
         check_i8(yq[b, :, h, :], oracle.requant(r, s_y))
+
+
+# ---------------------------------------------------------------------------------------
+# decode: the same transform of the single-token output, on the fp32 and the int8 state
+# ---------------------------------------------------------------------------------------
+def _decode_case(seed):
+    d = W.make_decode(8, 1, 16, 64, 128, 4, seed=seed)
+    return d, dict(x=d.x[0], B=d.B[0], C=d.C[0], dt=d.dt[0])
+
+
+def _dec_args(d, tok):
+    return (dev(tok["x"]), dev(tok["B"]), dev(tok["C"]), dev(tok["dt"]), dev(d.A), dev(d.D),
+            dev(d.x_scale), dev(d.B_scale), dev(d.C_scale))
+
+
+@pytest.mark.parametrize("out", ["f32", "f16", "i8"])
+def test_hadamard_decode_fp32_state(out):
+    d, tok = _decode_case(61)
+    ref_state = d.state.astype(np.float64)
+    yr = oracle.hadamard(oracle.step(ref_state, tok["x"], tok["B"], tok["C"], tok["dt"], d.A,
+                                     d.D, d.x_scale, d.B_scale, d.C_scale))
+    s_y = float(np.abs(yr).max() / 127.0)
+    st = dev(d.state)
+    y = ssd_i8.ssd_i8_state_update(st, *_dec_args(d, tok), y_dtype=out, y_scale=s_y,
+                                   hadamard=True)
+    st_plain = dev(d.state)
+    ssd_i8.ssd_i8_state_update(st_plain, *_dec_args(d, tok), y_dtype="f32")
+    torch.cuda.synchronize()
+    if out == "i8":
+        check_i8(y.cpu().numpy(), oracle.requant(yr, s_y))
+    else:
+        check_close(y.float().cpu().numpy(), yr, "H y / 8 (decode)")
+    assert torch.equal(st, st_plain), "the flag changed the state update"
+
+
+@pytest.mark.parametrize("out", ["f32", "i8"])
+def test_hadamard_decode_int8_state(out):
+    d, tok = _decode_case(62)
+    codes, scales = oracle.quantize_state(d.state)
+    scales32 = scales.astype(np.float32)
+    yr = oracle.hadamard(oracle.step_q8(codes, scales32, tok["x"], tok["B"], tok["C"],
+                                        tok["dt"], d.A, d.D, d.x_scale, d.B_scale,
+                                        d.C_scale)[0])
+    s_y = float(np.abs(yr).max() / 127.0)
+    q, s = dev(codes), dev(scales32)
+    y = ssd_i8.ssd_i8_state_update_q8(q, s, *_dec_args(d, tok), y_dtype=out, y_scale=s_y,
+                                      hadamard=True)
+    q2, s2 = dev(codes), dev(scales32)
+    ssd_i8.ssd_i8_state_update_q8(q2, s2, *_dec_args(d, tok), y_dtype="f32")
+    torch.cuda.synchronize()
+    if out == "i8":
+        check_i8(y.cpu().numpy(), oracle.requant(yr, s_y))
+    else:
+        check_close(y.cpu().numpy(), yr, "H y / 8 (int8-state decode)")
+    assert torch.equal(q, q2) and torch.equal(s, s2), "the flag changed the cached state"
+
+
+def test_hadamard_needs_headdim_64():
+    d = W.make_decode(2, 1, 4, 32, 16, 1, seed=63)
+    st = dev(d.state)
+    with pytest.raises(ssd_i8.SSDError):
+        ssd_i8.ssd_i8_state_update(st, dev(d.x[0]), dev(d.B[0]), dev(d.C[0]), dev(d.dt[0]),
+                                   dev(d.A), dev(d.D), dev(d.x_scale), dev(d.B_scale),
+                                   dev(d.C_scale), y_dtype="f32", hadamard=True)
