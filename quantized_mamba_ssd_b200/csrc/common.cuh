@@ -13,46 +13,6 @@ constexpr int kWarp = 32;
 
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
-// int8 x int8 dot product of 4 lanes accumulated in int32 (exact).
-__device__ __forceinline__ int dot4_i8(int a, int b, int acc) { return __dp4a(a, b, acc); }
-
-// Inclusive prefix sum over one warp (shuffle-up scan).
-__device__ __forceinline__ float warp_inclusive_scan(float v) {
-    const int lane = threadIdx.x & (kWarp - 1);
-#pragma unroll
-    for (int o = 1; o < kWarp; o <<= 1) {
-        float u = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += u;
-    }
-    return v;
-}
-
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-    for (int o = kWarp / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
-}
-
-// Inclusive block-wide prefix sum of one value per thread; `scratch` holds >= 32 floats.
-// Every thread of the block must call it.
-__device__ __forceinline__ float block_inclusive_scan(float v, float* scratch) {
-    const int lane = threadIdx.x & (kWarp - 1);
-    const int warp = threadIdx.x / kWarp;
-    const int nwarps = blockDim.x / kWarp;
-    v = warp_inclusive_scan(v);
-    if (lane == kWarp - 1) scratch[warp] = v;
-    __syncthreads();
-    if (warp == 0) {
-        float w = lane < nwarps ? scratch[lane] : 0.f;
-        w = warp_inclusive_scan(w);
-        if (lane < nwarps) scratch[lane] = w;
-    }
-    __syncthreads();
-    if (warp > 0) v += scratch[warp - 1];
-    __syncthreads();
-    return v;
-}
-
 // Output store in the requested dtype.  I8 applies q = clamp(rne(y * inv_scale), -127, 127)
 // with inv_scale = 1 / y_scale computed once in fp32 on the host.
 __device__ __forceinline__ void store_out(void* y, size_t idx, float v, int dtype, float inv_scale) {

@@ -48,22 +48,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return done != 0;
 }
 
-// Same test, but a thread whose phase is not complete yet may sleep for up to `suspend_ns`
-// nanoseconds (it wakes as soon as the phase completes), so that waiting warps take no issue
-// slots from the working ones.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity,
-                                                    uint32_t suspend_ns) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
-        : "memory");
-    return done != 0;
-}
-
 // Bounded wait for the phase with the given parity to complete.  Returns false if it did not
 // complete within `max_cycles` SM clocks (the caller then reports a timeout and bails out).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long max_cycles) {
