@@ -128,10 +128,12 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 // Persistent CTAs, each walking the (batch, head) items blockIdx.x, + gridDim.x, ...  Every
 // thread copies its own 16-byte state chunks (and the B or C chunk it stages) of the NEXT item
 // into its private slots of a two-stage shared buffer while it computes the current one, so
-// the loads stay in flight without holding registers; the current item's update is kept in
-// registers between the y / max pass and the requantisation.
+// the loads stay in flight without holding registers.  The requantisation pass recomputes the
+// update from the codes in shared memory: that costs a fifth more instructions than keeping it
+// in registers, but the smaller register budget fits six CTAs per SM instead of four, and the
+// step is bound by latency more than by issue.
 template <int N, int TPB, int CH, bool HAD>
-__global__ void __launch_bounds__(TPB, (CH >= 4 ? 512 : 640) / TPB)  // the update in registers
+__global__ void __launch_bounds__(TPB, 768 / TPB)  // 24 warps per SM
 state_update_q8_kernel(int8_t* __restrict__ state_q, float* __restrict__ state_scale,
                        const int8_t* __restrict__ x, const int8_t* __restrict__ Bq,
                        const int8_t* __restrict__ Cq, const float* __restrict__ dt,
@@ -207,7 +209,6 @@ state_update_q8_kernel(int8_t* __restrict__ state_q, float* __restrict__ state_s
 
         const f2 ds = {decay * s_old, decay * s_old};  // decayed dequantisation factor
         float amax = 0.f;
-        f2 hv[CH][8];
         // the loop bound is warp-uniform (multiples of the CTA size) so that every lane reaches
         // the shuffles
 #pragma unroll
@@ -217,19 +218,20 @@ state_update_q8_kernel(int8_t* __restrict__ state_q, float* __restrict__ state_s
             const bool in = u < nchunks;
             const int p = in ? u / CPR : 0, cc = u % CPR;
             // (a thread past the last chunk copied nothing: its zero codes keep the max clean)
-            unpack16(in ? sq[s][k][tid] : make_uint4(0u, 0u, 0u, 0u), hv[k]);
+            f2 hv[8];
+            unpack16(in ? sq[s][k][tid] : make_uint4(0u, 0u, 0u, 0u), hv);
             const float xv = sx * xq[k];
             const f2 dx = {dtv * xv, dtv * xv};
             f2 acc = {0.f, 0.f};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const float4 bb = sb[i * CPR + cc], cq = sc[i * CPR + cc];
-                hv[k][2 * i] = ffma2(ds, hv[k][2 * i], fmul2(dx, f2{bb.x, bb.y}));
-                hv[k][2 * i + 1] = ffma2(ds, hv[k][2 * i + 1], fmul2(dx, f2{bb.z, bb.w}));
-                acc = ffma2(f2{cq.x, cq.y}, hv[k][2 * i], acc);
-                acc = ffma2(f2{cq.z, cq.w}, hv[k][2 * i + 1], acc);
-                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(hv[k][2 * i].x), fabsf(hv[k][2 * i].y)),
-                                         fmaxf(fabsf(hv[k][2 * i + 1].x), fabsf(hv[k][2 * i + 1].y))));
+                hv[2 * i] = ffma2(ds, hv[2 * i], fmul2(dx, f2{bb.x, bb.y}));
+                hv[2 * i + 1] = ffma2(ds, hv[2 * i + 1], fmul2(dx, f2{bb.z, bb.w}));
+                acc = ffma2(f2{cq.x, cq.y}, hv[2 * i], acc);
+                acc = ffma2(f2{cq.z, cq.w}, hv[2 * i + 1], acc);
+                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(hv[2 * i].x), fabsf(hv[2 * i].y)),
+                                         fmaxf(fabsf(hv[2 * i + 1].x), fabsf(hv[2 * i + 1].y))));
             }
             float a = acc.x + acc.y;
 #pragma unroll
@@ -249,7 +251,19 @@ state_update_q8_kernel(int8_t* __restrict__ state_q, float* __restrict__ state_s
         for (int k = 0; k < CH; ++k) {
             if (k * TPB >= nchunks) break;
             const int u = tid + k * TPB;
-            if (u < nchunks) st[u] = pack16(hv[k], inv);
+            if (u >= nchunks) continue;
+            const int cc = u % CPR;
+            const float xv = sx * xq[k];
+            const f2 dx = {dtv * xv, dtv * xv};
+            f2 hv[8];
+            unpack16(sq[s][k][tid], hv);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float4 bb = sb[i * CPR + cc];
+                hv[2 * i] = ffma2(ds, hv[2 * i], fmul2(dx, f2{bb.x, bb.y}));
+                hv[2 * i + 1] = ffma2(ds, hv[2 * i + 1], fmul2(dx, f2{bb.z, bb.w}));
+            }
+            st[u] = pack16(hv, inv);  // the same fp32 values as the max pass (same operations)
         }
         if (tid == 0) state_scale[item] = amax / 127.f;
         if (next >= count) break;
