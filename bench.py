@@ -48,7 +48,7 @@ NOMINAL_HBM_GBS = 7700.0  # B200 HBM3e datasheet bandwidth (HGX), context for th
 # profiles/ncu_fused_chunk_scan_b2_L8192.md.  The traffic grows in proportion to the tokens of a
 # launch, so the bench scales it to the workload.  A changed kernel reports null.
 _CAPTURED_TRAFFIC_PER_TOKEN = {
-    "908438e75786a1238d8443323545ff01890339c19ad4aa2c80502b385ada0975": (342.448384e6 + 118.953984e6) / 16384,
+    "8635a74ee3f87a87ab48cdfa787d4efc669083d79ee870ed455ad88d4e49ce64": (338.766848e6 + 118.679296e6) / 16384,
 }
 
 

@@ -429,9 +429,8 @@ __device__ __noinline__ void store_piece_state(const FusedParams& p, uint32_t tm
                                                float out_scale, int bar_id) {
     const uint32_t lane_base = static_cast<uint32_t>(row & ~31);
     uint32_t hv[2][32];
-    tmem_ld32(tmem_addr(tmem, lane_base, kColH), hv[0]);
-    tmem_ld32(tmem_addr(tmem, lane_base, kColH + 32), hv[1]);
-    tmem_ld_wait();
+    tmem_ld32_sync(tmem_addr(tmem, lane_base, kColH), hv[0]);
+    tmem_ld32_sync(tmem_addr(tmem, lane_base, kColH + 32), hv[1]);
     if (final_piece) {
         if (p.final_state != nullptr && row < p.N) {
             float* dst = p.final_state + ((size_t)seq * p.H + h) * kP * p.N;
@@ -740,9 +739,8 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 float sv[32], dv[32];
                 {
                     uint32_t r0[32], r1[32];
-                    tmem_ld32(tmem_addr(tmem, lane_base, col_acc), r0);
-                    tmem_ld32(tmem_addr(tmem, lane_base, col_acc + 32), r1);
-                    tmem_ld_wait();
+                    tmem_ld32_sync(tmem_addr(tmem, lane_base, col_acc), r0);
+                    tmem_ld32_sync(tmem_addr(tmem, lane_base, col_acc + 32), r1);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const f2 a = {__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1])};
@@ -771,13 +769,16 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
 #pragma unroll 1
                 for (int hq = 0; hq < 2; ++hq) {
                     uint32_t r[32];
-                    tmem_ld32(tmem_addr(tmem, lane_base, col_acc + 32 * hq), r);
-                    tmem_ld_wait();
-                    if (!store) continue;
-                    float v[32];
+                    // (the warp is converged here: the rows past a ragged tail only skip the
+                    // stores below, so every lane reaches the next load together)
+                    tmem_ld32_sync(tmem_addr(tmem, lane_base, col_acc + 32 * hq), r);
+                    if (store) {
+                        float v[32];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-                    store32(v, pv_rho, ybase, hq);
+                        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+                        store32(v, pv_rho, ybase, hq);
+                    }
+                    __syncwarp();
                 }
                 tc_fence_before();
                 wg_sync(bar_id);
@@ -931,8 +932,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
 #pragma unroll 1
                 for (int sc = 0; sc < wq; ++sc) {
                     uint32_t cbv[32], o[16];
-                    tmem_ld32(tmem_addr(tmem, lane_base, col_cb + 32 * sc), cbv);
-                    tmem_ld_wait();
+                    tmem_ld32_sync(tmem_addr(tmem, lane_base, col_cb + 32 * sc), cbv);
                     const float2* cf = reinterpret_cast<const float2*>(cfq + 32 * sc);
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
@@ -945,8 +945,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 // diagonal sub-block: one exponential per entry, s > t masked
                 {
                     uint32_t cbv[32], o[16];
-                    tmem_ld32(tmem_addr(tmem, lane_base, col_cb + 32 * wq), cbv);
-                    tmem_ld_wait();
+                    tmem_ld32_sync(tmem_addr(tmem, lane_base, col_cb + 32 * wq), cbv);
                     const float2* nb = reinterpret_cast<const float2*>(nbeta + 32 * wq);
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
@@ -981,8 +980,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
 #pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
                     uint32_t hv[32];
-                    tmem_ld32(tmem_addr(tmem, lane_base, kColH + 32 * hh), hv);
-                    tmem_ld_wait();
+                    tmem_ld32_sync(tmem_addr(tmem, lane_base, kColH + 32 * hh), hv);
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         uint32_t wq4[4];
@@ -1125,8 +1123,7 @@ chunk_cb_tc_kernel(const __grid_constant__ CUtensorMap map_B, const __grid_const
         const int t = tb * kBlk + tid;
         for (int sc = 0; sc < Q / 32; ++sc) {
             uint32_t r[32];
-            tmem_ld32(tmem_addr(tmem, warp * 32, 32 * sc), r);
-            tmem_ld_wait();
+            tmem_ld32_sync(tmem_addr(tmem, warp * 32, 32 * sc), r);
             if (t < Q) {
 #pragma unroll
                 for (int j = 0; j < 32; ++j) out[(size_t)t * Q + 32 * sc + j] = static_cast<int32_t>(r[j]);
