@@ -125,3 +125,37 @@ def test_prefill_state_hands_over_to_the_int8_cache():
     # the cache holds the oracle's final state to within half a step (+ the scan's tolerance)
     step = s.cpu().numpy()[:, :, None, None]
     assert (np.abs(deq - fr) <= 0.5 * step + 2e-3 * np.abs(fr).max()).all()
+
+
+def test_int8_state_workload_sampled():
+    """The batch-128, Mamba-2-8B-shaped decode at full size on the int8 cached state, in the
+    launch configuration the benchmark times: 64 steps, sampled (batch, head) pairs followed
+    through every step by the oracle with its own cache."""
+    d = W.make_decode_config()
+    steps = 64
+    q, s = ssd_i8.ssd_i8_state_quantize(dev(d.state))
+    codes0, scales0 = q.cpu().numpy(), s.cpu().numpy()
+    pairs = [(0, 0), (127, 127), (64, 3), (5, 90)]
+    ys = {pr: [] for pr in pairs}
+    args = [dev(d.A), dev(d.D), dev(d.x_scale), dev(d.B_scale), dev(d.C_scale)]
+    xs, Bs, Cs, dts = dev(d.x), dev(d.B), dev(d.C), dev(d.dt)
+    for t in range(steps):
+        y = ssd_i8.ssd_i8_state_update_q8(q, s, xs[t], Bs[t], Cs[t], dts[t], *args, y_dtype="f32")
+        for (b, h) in pairs:
+            ys[(b, h)].append(y[b, h].clone())
+    torch.cuda.synchronize()
+    H, G = d.nheads, d.ngroups
+    for (b, h) in pairs:
+        g = h // (H // G)
+        oc = codes0[b:b + 1, h:h + 1]
+        osc = scales0[b:b + 1, h:h + 1].astype(np.float64)
+        refs = []
+        for t in range(steps):
+            yr, oc, osc = oracle.step_q8(oc, osc, d.x[t][b:b + 1, h:h + 1],
+                                         d.B[t][b:b + 1, g:g + 1], d.C[t][b:b + 1, g:g + 1],
+                                         d.dt[t][b:b + 1, h:h + 1], d.A[h:h + 1], d.D[h:h + 1],
+                                         d.x_scale[h:h + 1], d.B_scale[g:g + 1],
+                                         d.C_scale[g:g + 1])
+            refs.append(yr[0, 0])
+        got = torch.stack(ys[(b, h)]).cpu().numpy()
+        check_close(got, np.stack(refs), f"int8-state decode y (b={b}, h={h})")
