@@ -125,6 +125,12 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int K>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(K) : "memory"); }
 
+// (batch, head, group) of an item, and r = head % (heads per group); stepping it by the grid
+// stride needs no integer division (those cost tens of instructions each)
+struct ItemPos {
+    int b, h, g, r;
+};
+
 // Persistent CTAs, each walking the (batch, head) items blockIdx.x, + gridDim.x, ...  Every
 // thread copies its own 16-byte state chunks (and the B or C chunk it stages) of the NEXT item
 // into its private slots of a two-stage shared buffer while it computes the current one, so
@@ -156,10 +162,35 @@ state_update_q8_kernel(int8_t* __restrict__ state_q, float* __restrict__ state_s
     const int nchunks = P * CPR;
     int item = blockIdx.x;
     if (item >= count) return;
+    // the item's position, and the stride's (the only divisions of the kernel)
+    const int HG = H / G;
+    const int Sb = gridDim.x / H, Sh = gridDim.x % H, Sg = Sh / HG, Sr = Sh % HG;
+    ItemPos pos;
+    pos.b = item / H;
+    pos.h = item % H;
+    pos.g = pos.h / HG;
+    pos.r = pos.h % HG;
+    auto step = [&](ItemPos q) {
+        q.r += Sr;
+        q.g += Sg;
+        if (q.r >= HG) {
+            q.r -= HG;
+            ++q.g;
+        }
+        q.h += Sh;
+        q.b += Sb;
+        if (q.h >= H) {
+            q.h -= H;
+            ++q.b;
+            q.g -= G;
+        }
+        return q;
+    };
 
-    // issue the copies of `it`'s chunks into stage `s` (one commit group), and return its x
-    auto prefetch = [&](int it, int s, float (&xq)[CH]) {
-        const int b = it / H, h = it % H, g = h / (H / G);
+    // issue the copies of `it`'s chunks (at position q) into stage `s` (one commit group), and
+    // return its x
+    auto prefetch = [&](int it, const ItemPos& q, int s, float (&xq)[CH]) {
+        const int b = q.b, g = q.g;
         const uint4* st = reinterpret_cast<const uint4*>(state_q + (size_t)it * P * N);
         const int8_t* xrow = x + (size_t)it * P;
 #pragma unroll
@@ -177,21 +208,22 @@ state_update_q8_kernel(int8_t* __restrict__ state_q, float* __restrict__ state_s
     };
 
     float xq[CH], xq_n[CH];
-    prefetch(item, 0, xq);
+    prefetch(item, pos, 0, xq);
     float dtv = dt[item], s_old = state_scale[item];
     for (int it = 0;; ++it) {
         const int s = it & 1;
         const int next = item + gridDim.x;
+        const ItemPos npos = step(pos);
         float dt_n = 0.f, s_old_n = 0.f;
         if (next < count) {
-            prefetch(next, s ^ 1, xq_n);
+            prefetch(next, npos, s ^ 1, xq_n);
             dt_n = dt[next];
             s_old_n = state_scale[next];
             cp_async_wait<1>();  // this item's group has landed (the next one may be in flight)
         } else {
             cp_async_wait<0>();
         }
-        const int h = item % H, g = h / (H / G);
+        const int h = pos.h, g = pos.g;
         const float sx = x_scale[h], Dh = D[h];
         const float decay = __expf(dtv * A[h]);
         float4* sb = sbv[s];
@@ -268,6 +300,7 @@ state_update_q8_kernel(int8_t* __restrict__ state_q, float* __restrict__ state_s
         if (tid == 0) state_scale[item] = amax / 127.f;
         if (next >= count) break;
         item = next;
+        pos = npos;
         dtv = dt_n;
         s_old = s_old_n;
 #pragma unroll
