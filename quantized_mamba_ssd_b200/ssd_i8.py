@@ -7,6 +7,7 @@ is missing or fails to load, the calls raise -- there is no fallback.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import threading
@@ -40,6 +41,7 @@ KERNELS_PER_STATE_UPDATE = 1
 
 _lock = threading.Lock()
 _lib: Optional[ctypes.CDLL] = None
+_tls = threading.local()  # device of the call being marshalled
 
 
 class SSDError(RuntimeError):
@@ -100,6 +102,32 @@ def _check(fn: str, status: int) -> None:
         raise SSDError(fn, status, msg)
 
 
+@contextlib.contextmanager
+def _on_device_of(t: torch.Tensor):
+    """Run one library call with ``t``'s GPU as the current device: the library launches on the
+    current device, and every tensor of the call must live on that one."""
+    if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+        raise ValueError("the library's tensors must be CUDA tensors")
+    prev = getattr(_tls, "device", None)
+    _tls.device = t.device
+    try:
+        with torch.cuda.device(t.device):
+            yield
+    finally:
+        _tls.device = prev
+
+
+def _device_call(fn):
+    """Decorator: the wrapped call marshals and launches on the GPU of its first tensor."""
+    import functools
+
+    @functools.wraps(fn)
+    def wrapper(first, *args, **kwargs):
+        with _on_device_of(first):
+            return fn(first, *args, **kwargs)
+    return wrapper
+
+
 def _ptr(t: Optional[torch.Tensor], name: str, dtype: torch.dtype, shape=None) -> Optional[int]:
     if t is None:
         return None
@@ -107,6 +135,9 @@ def _ptr(t: Optional[torch.Tensor], name: str, dtype: torch.dtype, shape=None) -
         raise TypeError(f"{name} must be a torch.Tensor")
     if t.device.type != "cuda":
         raise ValueError(f"{name} must be a CUDA tensor")
+    dev = getattr(_tls, "device", None)
+    if dev is not None and t.device != dev:
+        raise ValueError(f"{name} is on {t.device}, the call's other tensors on {dev}")
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
@@ -130,6 +161,7 @@ def ssd_i8_chunk_scan_workspace_size(batch: int, seqlen: int, nheads: int, headd
                                                           ngroups, chunk_size))
 
 
+@_device_call
 def ssd_i8_chunk_scan(x: torch.Tensor, B: torch.Tensor, C: torch.Tensor, dt: torch.Tensor,
                       A: torch.Tensor, D: torch.Tensor, x_scale: torch.Tensor,
                       B_scale: torch.Tensor, C_scale: torch.Tensor, chunk_size: int, *,
@@ -204,6 +236,7 @@ def ssd_i8_chunk_scan_varlen_workspace_size(nseq: int) -> int:
     return int(library().ssd_i8_chunk_scan_varlen_workspace_size(int(nseq)))
 
 
+@_device_call
 def ssd_i8_chunk_scan_varlen(x: torch.Tensor, B: torch.Tensor, C: torch.Tensor, dt: torch.Tensor,
                              A: torch.Tensor, D: torch.Tensor, x_scale: torch.Tensor,
                              B_scale: torch.Tensor, C_scale: torch.Tensor, cu_seqlens,
@@ -263,6 +296,7 @@ def ssd_i8_chunk_scan_varlen(x: torch.Tensor, B: torch.Tensor, C: torch.Tensor, 
     return y
 
 
+@_device_call
 def ssd_i8_state_update(state: torch.Tensor, x: torch.Tensor, B: torch.Tensor, C: torch.Tensor,
                         dt: torch.Tensor, A: torch.Tensor, D: torch.Tensor,
                         x_scale: torch.Tensor, B_scale: torch.Tensor, C_scale: torch.Tensor, *,
@@ -296,6 +330,7 @@ def ssd_i8_state_update(state: torch.Tensor, x: torch.Tensor, B: torch.Tensor, C
     return y
 
 
+@_device_call
 def ssd_i8_state_quantize(state: torch.Tensor, state_q: Optional[torch.Tensor] = None,
                           state_scale: Optional[torch.Tensor] = None, stream=None):
     """fp32 state [b,h,p,n] -> (int8 codes [b,h,p,n], float32 scales [b,h]) with scale =
@@ -313,6 +348,7 @@ def ssd_i8_state_quantize(state: torch.Tensor, state_q: Optional[torch.Tensor] =
     return state_q, state_scale
 
 
+@_device_call
 def ssd_i8_state_update_q8(state_q: torch.Tensor, state_scale: torch.Tensor, x: torch.Tensor,
                            B: torch.Tensor, C: torch.Tensor, dt: torch.Tensor, A: torch.Tensor,
                            D: torch.Tensor, x_scale: torch.Tensor, B_scale: torch.Tensor,
@@ -350,6 +386,7 @@ def ssd_i8_state_update_q8(state_q: torch.Tensor, state_scale: torch.Tensor, x: 
     return y
 
 
+@_device_call
 def ssd_i8_chunk_cb(C: torch.Tensor, B: torch.Tensor, chunk_size: int, *,
                     cb: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """ChunkBMM export: int32 [b, ceil(l/Q), g, Q, Q] = Cq Bq^T per chunk and group."""
@@ -374,6 +411,7 @@ def ssd_i8_debug_inject(drop_publish_cta: int, wait_cycles: int) -> None:
     _check("ssd_i8_debug_inject", library().ssd_i8_debug_inject(int(drop_publish_cta), int(wait_cycles)))
 
 
+@_device_call
 def ssd_i8_chunk_scan_status(workspace: torch.Tensor, stream=None) -> None:
     """Raise SSDError (SSD_ERR_TIMEOUT) if the last chunk scan on ``workspace`` reported a
     device-side wait that gave up; synchronises the stream."""
@@ -382,6 +420,7 @@ def ssd_i8_chunk_scan_status(workspace: torch.Tensor, stream=None) -> None:
                                               _stream(stream)))
 
 
+@_device_call
 def ssd_i8_chunk_scan_noalloc(x: torch.Tensor, B: torch.Tensor, C: torch.Tensor,
                               dt: torch.Tensor, A: torch.Tensor, D: torch.Tensor,
                               x_scale: torch.Tensor, B_scale: torch.Tensor,
