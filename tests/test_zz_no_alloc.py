@@ -2,7 +2,7 @@
 
 Such callers (an engine whose memory pool is reserved in full before it serves, code that must
 not risk the device synchronisation of a cudaMalloc, a plug-in whose host owns allocation) call
-``ssd_i8_chunk_scan_noalloc``, which takes its scratch from the library's built-in 16 MiB device
+``ssd_i8_chunk_scan_noalloc``, which takes its scratch from the library's built-in 4 MiB device
 array instead of a workspace.  These tests call it through the C ABI and compare it with the
 workspace-taking ``ssd_i8_chunk_scan`` on the same inputs, with the parity tolerances, on two
 calls in a row (so that the second call runs on scratch the first one left behind).
@@ -67,7 +67,8 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
 
 
 def test_noalloc_refuses_problems_beyond_its_scratch():
-    case = W.make_prefill(4, 2048, 64, 64, 128, 1, 256, seed=43)  # 64 MiB of chunk states
+    # more work items than the scratch has state slots for
+    case = W.make_prefill(4, 2048, 64, 64, 128, 1, 256, seed=43)
     need = ssd_i8.ssd_i8_chunk_scan_workspace_size(4, 2048, 64, 64, 128, 1, 256)
     assert need > ssd_i8.NOALLOC_SCRATCH_BYTES
     ins, _ = _inputs(case)
