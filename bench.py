@@ -6,7 +6,8 @@ shaped long prefill (batch 2 x 16384 tokens, 128 heads x 64, dstate 128, 8 group
 requantizing epilogue.  ``value`` = tokens/s with inputs resident in HBM; ``e2e`` = the same
 through the public call with pinned-host inputs copied in and the int8 output copied back in
 every step.  The decode state update (batch 128, 512 steps) is reported beside it under
-``decode``.
+``decode``; the packed serving prefill (prompts of mixed length as strided views of one
+projection buffer, ``ssd_i8_chunk_scan_varlen``) under ``varlen_strided``.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 For N > 1 launch under torch.distributed.run; every rank scans its own batch (weak scaling,
@@ -237,6 +238,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) leg")
     ap.add_argument("--no-per-tensor", action="store_true",
                     help="skip the per-tensor percentile-clipped workload leg")
+    ap.add_argument("--no-varlen", action="store_true",
+                    help="skip the packed variable-length (strided) serving prefill leg")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="decode batch per rank (default: the workload's 128); smaller batches "
                          "of the same shape serve profiling captures")
@@ -455,6 +458,66 @@ def main():
         }
         del px, pB, pC, pdt, pcase
 
+    # ---- packed serving prefill: the layer's tokens as prompts of mixed length, read as
+    # strided column slices of one projection buffer (ssd_i8_chunk_scan_varlen) ----
+    varlen = None
+    if not args.no_varlen:
+        vcase, cu = W.make_varlen_config(seed=rank_seed(1005, rank),
+                                         **({} if args.seqlen is None and args.batch is None
+                                            else {"total_tokens": bsz * L}))
+        T = int(cu[-1])
+        nseq = len(cu) - 1
+        xw = H * P + 2 * G * N  # one projection row: x | B | C
+        proj = torch.empty((T, xw), dtype=torch.int8, device=dev)
+        proj[:, :H * P] = torch.from_numpy(vcase.x.reshape(T, H * P)).to(dev)
+        proj[:, H * P:H * P + G * N] = torch.from_numpy(vcase.B.reshape(T, G * N)).to(dev)
+        proj[:, H * P + G * N:] = torch.from_numpy(vcase.C.reshape(T, G * N)).to(dev)
+        vx = proj[:, :H * P].view(T, H, P)
+        vB = proj[:, H * P:H * P + G * N].view(T, G, N)
+        vC = proj[:, H * P + G * N:].view(T, G, N)
+        vdt = torch.from_numpy(vcase.dt.reshape(T, H)).to(dev)
+        vA, vD, vsx, vsb, vsc = (torch.from_numpy(a).to(dev) for a in
+                                 (vcase.A, vcase.D, vcase.x_scale, vcase.B_scale, vcase.C_scale))
+        vy = torch.empty((T, H, P), dtype=torch.int8, device=dev)
+        vfs = torch.empty((nseq, H, P, N), dtype=torch.float32, device=dev)
+        vws = torch.empty(ssd_i8.ssd_i8_chunk_scan_varlen_workspace_size(nseq), dtype=torch.uint8,
+                          device=dev)
+
+        def step_vl():
+            ssd_i8.ssd_i8_chunk_scan_varlen(vx, vB, vC, vdt, vA, vD, vsx, vsb, vsc, cu, Q,
+                                            final_state=vfs, y=vy, y_dtype="i8",
+                                            y_scale=y_scale, workspace=vws)
+
+        for _ in range(args.warmup):
+            step_vl()
+        torch.cuda.synchronize()
+        barrier()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step_vl()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        vl_ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dev)
+        vl_bytes = (T * (H * P + 2 * G * N + 4 * H + H * P)  # x, B, C, dt in; y out (int8)
+                    + 4 * nseq * H * P * N)  # final states
+        vl_gbs = vl_bytes / (vl_ms * 1e-3) / 1e9
+        blocks = int(sum(-(-int(n) // 128) for n in (cu[1:] - cu[:-1])))
+        varlen = {
+            "metric": "SSD scan tokens/s (int8 in), packed variable-length sequences read as "
+                      "strided views of one projection buffer, int8 out",
+            "workload": vcase.name, "value": aggregate_tokens_per_s(T, world, vl_ms),
+            "unit": UNIT, "ms_per_step": vl_ms, "sequences": nseq,
+            "length_mix": "log-uniform in [64, 8192] tokens, last cut to fill",
+            "min_len": int((cu[1:] - cu[:-1]).min()), "max_len": int((cu[1:] - cu[:-1]).max()),
+            "token_blocks_of_128": blocks, "padded_token_fraction": 1.0 - T / (128.0 * blocks),
+            "x_token_stride_bytes": xw, "gpu_launches": args.steps * ssd_i8.KERNELS_PER_CHUNK_SCAN,
+            "roofline": {"bound": "hbm", "achieved": vl_gbs, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": vl_gbs / hbm_peak, "traffic": None,
+                         "alg_bytes_per_launch": vl_bytes},
+        }
+        del proj, vx, vB, vC, vdt, vy, vfs, vws, vcase
+
     # ---- roofline of the timed call ----
     alg_bytes = prefill_alg_bytes(case, 1, True)
     alg_ops = prefill_alg_ops(case)
@@ -591,6 +654,7 @@ def main():
             "gpu_launches": args.steps * ssd_i8.KERNELS_PER_CHUNK_SCAN,
             "clocks": clocks.summary(),
             "hadamard_out": hadamard_out, "per_tensor_percentile": per_tensor,
+            "varlen_strided": varlen,
             "decode": decode,
         }
         print(json.dumps(line), flush=True)

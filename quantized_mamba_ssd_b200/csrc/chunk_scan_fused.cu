@@ -181,14 +181,15 @@ struct Range {
         }
     }
     __device__ void seg(const FusedParams& p, int k, Piece& pc) const {
-        const long long u = (k == 0) ? u_last : (k == nseg - 1 ? u_first : u_first + k);
-        const int si = static_cast<int>(u / H);
+        // (unit indices fit in 32 bits: every unit holds at least one of < 2^31 blocks)
+        const int u = static_cast<int>((k == 0) ? u_last : (k == nseg - 1 ? u_first : u_first + k));
+        const int si = u / H;
         const int4 e = seq_entry(p, si);
         pc.seq = e.w;
         pc.tok0 = e.x;
         pc.len = e.y;
         pc.nblk = (e.y + kBlk - 1) / kBlk;
-        pc.h = static_cast<int>(u % H);
+        pc.h = u - si * H;
         pc.cb = u == u_first ? c_first : 0;
         pc.ce = u == u_last ? c_last + 1 : pc.nblk;
     }
@@ -422,9 +423,9 @@ __device__ __forceinline__ void issue_cb(uint32_t d, uint32_t sC, uint32_t sB, i
 
 // Piece end (worker warpgroup, thread = state row n): writes the state of the finished piece,
 // either as the caller's final state or into this CTA's hand-off slot (then publishes the slot).
-// `out_scale` converts TMEM units to units of s_x s_B.  Kept out of line: it runs once or twice
-// per CTA.
-__device__ __noinline__ void store_piece_state(const FusedParams& p, uint32_t tmem, int row,
+// `out_scale` converts TMEM units to units of s_x s_B.  Inlined: a call from the worker loop
+// would save and restore its live registers at every piece switch.
+__device__ __forceinline__ void store_piece_state(const FusedParams& p, uint32_t tmem, int row,
                                                bool final_piece, bool cta_end, int seq, int h,
                                                float out_scale, int bar_id) {
     const uint32_t lane_base = static_cast<uint32_t>(row & ~31);
@@ -456,19 +457,23 @@ __device__ __noinline__ void store_piece_state(const FusedParams& p, uint32_t tm
     }
 }
 
-// Piece start (worker warpgroup): loads the piece's initial state into TMEM in units of s_x s_B:
-// the caller's initial state (or zero) at sequence start, else the predecessor CTA's hand-off
-// slot after a bounded wait for its flag.  Returns max |state| over the piece's state.
-__device__ __noinline__ float load_piece_state(const FusedParams& p, uint32_t tmem, int row,
-                                               float* red, volatile uint32_t* abort_flag, int seq,
-                                               int h, int c_begin, float sigma, int bar_id) {
+// Piece start (worker warpgroup, thread = state row n): the piece's initial state in units of
+// s_x s_B -- the caller's initial state (or zero) at sequence start, else the predecessor CTA's
+// hand-off slot.  piece_state_bound returns its max |.| (for the operand scaling of the piece's
+// first block) without touching tensor memory; for a slot it first waits (bounded) for the
+// predecessor's flag.  write_piece_state later puts the state into TMEM, once the previous
+// piece's last update has been read out.  Both are inlined, like store_piece_state.
+__device__ __forceinline__ const float* piece_state_src(const FusedParams& p, int seq, int h,
+                                                        int c_begin) {
+    if (c_begin != 0) return p.slots + (size_t)(blockIdx.x - 1) * 128 * kP;
+    return p.init_state ? p.init_state + ((size_t)seq * p.H + h) * kP * p.N : nullptr;
+}
+
+__device__ __forceinline__ float piece_state_bound(const FusedParams& p, int row, float* red,
+                                                volatile uint32_t* abort_flag, int seq, int h,
+                                                int c_begin, float sigma, int bar_id) {
     const int warp = row >> 5, lane = row & 31;  // warp within the worker warpgroup
-    const uint32_t lane_base = static_cast<uint32_t>(row & ~31);
-    const float* src = nullptr;
-    bool from_slot = false;
-    if (c_begin == 0) {
-        if (p.init_state) src = p.init_state + ((size_t)seq * p.H + h) * kP * p.N;
-    } else {
+    if (c_begin != 0) {
         if (row == 0) {
             const unsigned long long* f = p.flags + (blockIdx.x - 1);
             const long long t0 = clock64();
@@ -485,31 +490,70 @@ __device__ __noinline__ float load_piece_state(const FusedParams& p, uint32_t tm
             }
         }
         wg_sync(bar_id);
-        src = p.slots + (size_t)(blockIdx.x - 1) * 128 * kP;
-        from_slot = true;
     }
-    const float inv_sigma = 1.f / sigma;
+    const float* src = piece_state_src(p, seq, h, c_begin);
     float m = 0.f;
-#pragma unroll 1
-    for (int half = 0; half < 2; ++half) {
-        uint32_t r[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int jj = 32 * half + i;
-            float v = 0.f;
-            if (src != nullptr && row < p.N)
-                v = from_slot ? __ldcg(src + row * kP + jj) : src[(size_t)jj * p.N + row] * inv_sigma;
-            m = fmaxf(m, fabsf(v));
-            r[i] = __float_as_uint(v);
+    if (src != nullptr && row < p.N) {
+        if (c_begin != 0) {
+            const float4* s4 = reinterpret_cast<const float4*>(src + row * kP);
+#pragma unroll 4
+            for (int q = 0; q < 16; ++q) {
+                const float4 v = __ldcg(s4 + q);
+                m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+            }
+        } else {
+#pragma unroll 8
+            for (int jj = 0; jj < 64; ++jj) m = fmaxf(m, fabsf(src[(size_t)jj * p.N + row]));
+            m /= sigma;
         }
-        tmem_st32(tmem_addr(tmem, lane_base, kColH + 32 * half), r);
     }
-    tmem_st_wait();
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     if (lane == 0) red[8 + warp] = m;
     wg_sync(bar_id);
     return fmaxf(fmaxf(red[8], red[9]), fmaxf(red[10], red[11]));
+}
+
+__device__ __forceinline__ void write_piece_state(const FusedParams& p, uint32_t tmem, int row, int seq,
+                                                  int h, int c_begin, float sigma) {
+    // The branches below are uniform over the worker (tcgen05.st is a warp-collective
+    // instruction: every lane of a warp must execute it together); rows past dstate only read
+    // zeros.
+    const uint32_t lane_base = static_cast<uint32_t>(row & ~31);
+    const float* src = piece_state_src(p, seq, h, c_begin);
+    const bool in = row < p.N;
+    uint32_t r[32];
+    if (src == nullptr) {  // a zero state
+#pragma unroll
+        for (int i = 0; i < 32; ++i) r[i] = 0u;
+        tmem_st32(tmem_addr(tmem, lane_base, kColH), r);
+        tmem_st32(tmem_addr(tmem, lane_base, kColH + 32), r);
+    } else if (c_begin != 0) {  // the predecessor's hand-off slot, already in units of s_x s_B
+        const float4* s4 = reinterpret_cast<const float4*>(src + row * kP);
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float4 v = in ? __ldcg(s4 + 8 * half + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+                r[4 * q] = __float_as_uint(v.x);
+                r[4 * q + 1] = __float_as_uint(v.y);
+                r[4 * q + 2] = __float_as_uint(v.z);
+                r[4 * q + 3] = __float_as_uint(v.w);
+            }
+            tmem_st32(tmem_addr(tmem, lane_base, kColH + 32 * half), r);
+        }
+    } else {  // the caller's initial state [p][n], divided by s_x s_B
+        const float inv_sigma = 1.f / sigma;
+        const float* col = src + (in ? row : 0);
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                r[i] = __float_as_uint(in ? col[(size_t)(32 * half + i) * p.N] * inv_sigma : 0.f);
+            tmem_st32(tmem_addr(tmem, lane_base, kColH + 32 * half), r);
+        }
+    }
+    tmem_st_wait();
 }
 
 // start column of quad q's off-diagonal column factors (q = 1, 2, 3 hold 32 q entries)
@@ -840,18 +884,10 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                                       : make_float4(1.f, 0.f, 1.f, 0.f);
             float hb, U_prev;
             if (pstart) {
-                // piece start: the previous piece (this CTA's previous segment) ends with block
-                // kb - 1; store its state, then load this piece's
-                if (kb >= 1) {
-                    wait_phase(bars + kBarState, (kb - 1) & 1, abort_flag, p);
-                    tc_fence_after();
-                    Piece prev;
-                    rg.seg(p, cur.seg - 1, prev);
-                    store_piece_state(p, tmem, row, prev.ce == prev.nblk, prev.ce != prev.nblk, prev.seq,
-                                      prev.h, sp.z, bar_id);
-                }
-                hb = load_piece_state(p, tmem, row, red, abort_flag, cur.pc.seq, cur.pc.h, cur.pc.cb,
-                                      sigma, bar_id);
+                // piece start: only the bound of its initial state is needed now; the state goes
+                // into TMEM at the hand-over, after the previous piece's last update
+                hb = piece_state_bound(p, row, red, abort_flag, cur.pc.seq, cur.pc.h, cur.pc.cb,
+                                       sigma, bar_id);
                 U_prev = 1.f;
             } else {
                 hb = sp.w * sp.x + 16129.f * sp.y;  // bound after block kb - 1's update
@@ -971,8 +1007,19 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             if (row == 0) mbar_arrive(bars + kBarMp0 + w);
             // (g) state hand-over, after the previous block's update: H' = H U / kappa (f16)
             //     for C'H', then decay + rescale to this block's unit
-            if (!pstart && kb >= 1) wait_phase(bars + kBarState, (kb - 1) & 1, abort_flag, p);
+            if (kb >= 1) wait_phase(bars + kBarState, (kb - 1) & 1, abort_flag, p);
             tc_fence_after();
+            if (pstart) {
+                // the previous piece (this CTA's previous segment) ended with block kb - 1, in
+                // state units sp.z: store its state, then load this piece's
+                if (kb >= 1) {
+                    Piece prev;
+                    rg.seg(p, cur.seg - 1, prev);
+                    store_piece_state(p, tmem, row, prev.ce == prev.nblk, prev.ce != prev.nblk, prev.seq,
+                                      prev.h, sp.z, bar_id);
+                }
+                write_piece_state(p, tmem, row, cur.pc.seq, cur.pc.h, cur.pc.cb, sigma);
+            }
             {
                 const f2 to_hp = {U_prev * invk, U_prev * invk};
                 const float th = e_end * (U_prev * inv_U_new);

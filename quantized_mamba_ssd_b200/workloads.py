@@ -38,6 +38,8 @@ __all__ = [
     "make_prefill_config",
     "make_decode",
     "make_decode_config",
+    "varlen_lengths",
+    "make_varlen_config",
 ]
 
 F32 = np.float32
@@ -323,3 +325,43 @@ def make_decode_config(seed: Optional[int] = None, **overrides) -> DecodeCase:
     if overrides:
         name += " [" + ", ".join(f"{k}={v}" for k, v in sorted(overrides.items())) + "]"
     return make_decode(seed=1004 if seed is None else seed, name=name, **spec)
+
+
+# the packed serving prefill: the 8B layer's 32768 tokens as a batch of prompts of mixed length
+VARLEN_CONFIG = dict(total_tokens=32768, min_len=64, max_len=8192, nheads=128, headdim=64,
+                     dstate=128, ngroups=8, chunk_size=256, law="laplace_outliers_all",
+                     scales="head", out_dtype="i8")
+
+
+def varlen_lengths(total: int, min_len: int, max_len: int, seed: int) -> np.ndarray:
+    """Sequence lengths drawn log-uniformly from [min_len, max_len] until they fill ``total``
+    tokens (the last one is cut to fit); int32."""
+    if total < 0 or min_len < 1 or max_len < min_len:
+        raise ValueError("need total >= 0 and 1 <= min_len <= max_len")
+    rng = np.random.default_rng(seed)
+    out = []
+    left = total
+    while left > 0:
+        n = int(np.exp(rng.uniform(np.log(min_len), np.log(max_len + 1))))
+        n = max(1, min(n, max_len, left))
+        out.append(n)
+        left -= n
+    return np.asarray(out, dtype=np.int32)
+
+
+def make_varlen_config(seed: Optional[int] = None, **overrides):
+    """The packed serving prefill of the Mamba-2-8B layer: one row of ``total_tokens`` tokens
+    (the activation laws of the 8B long prefill), cut into sequences whose lengths are drawn
+    log-uniformly from [min_len, max_len].  Returns (case with batch 1, cu_seqlens int32)."""
+    spec = dict(VARLEN_CONFIG)
+    spec.update(overrides)
+    seed = 1005 if seed is None else seed
+    T = spec.pop("total_tokens")
+    lengths = varlen_lengths(T, spec.pop("min_len"), spec.pop("max_len"), seed + 1)
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    name = (f"mamba2-8b-ssd-packed-serving-prefill T{T} nseq{len(lengths)} "
+            f"h{spec['nheads']} p{spec['headdim']} n{spec['dstate']} g{spec['ngroups']} "
+            f"Q{spec['chunk_size']} int8-out strided")
+    case = make_prefill(1, max(T, 1), spec.pop("nheads"), spec.pop("headdim"), spec.pop("dstate"),
+                        spec.pop("ngroups"), spec.pop("chunk_size"), seed=seed, name=name, **spec)
+    return case, cu

@@ -185,3 +185,46 @@ def test_malformed_sequences_are_rejected():
         ssd_i8.ssd_i8_chunk_scan_varlen(*args, *rest, [0, 100, 50], 256)  # decreasing
     with pytest.raises(ssd_i8.SSDError):
         ssd_i8.ssd_i8_chunk_scan_varlen(*args, *rest, [0, 64, 129], 256)  # past the tokens
+
+
+def test_packed_serving_workload_sampled():
+    """The packed serving prefill the benchmark times, at full size and in its launch
+    configuration: 32768 tokens of the Mamba-2-8B layer as 22 prompts of mixed length, read as
+    strided column slices of one projection buffer, int8 output.  Sampled (sequence, head)
+    pairs (the shortest, the longest and the middle sequence of the list) are checked against the
+    per-sequence oracle: the int8 output within one step, the f32 output of the same call and
+    the final states within the tolerances."""
+    case, cu = W.make_varlen_config()
+    T, H, P, N, G = int(cu[-1]), case.nheads, case.headdim, case.dstate, case.ngroups
+    lens = cu[1:] - cu[:-1]
+    seqs = sorted({int(np.argmin(lens)), int(np.argmax(lens)), len(lens) // 2})
+    heads = [0, 77, 127]
+    refs = {}
+    for s in seqs:
+        a, b = int(cu[s]), int(cu[s + 1])
+        for h in heads:
+            g = h // (H // G)
+            yr, fr, _ = oracle.scan(case.x[:, a:b, h:h + 1], case.B[:, a:b, g:g + 1],
+                                    case.C[:, a:b, g:g + 1], case.dt[:, a:b, h:h + 1],
+                                    case.A[h:h + 1], case.D[h:h + 1], case.x_scale[h:h + 1],
+                                    case.B_scale[g:g + 1], case.C_scale[g:g + 1])
+            refs[(s, h)] = (yr[0, :, 0, :], fr[0, 0])
+    s_y = float(max(np.abs(r[0]).max() for r in refs.values()) / 127.0)
+    xw = H * P + 2 * G * N
+    proj = torch.empty((T, xw), dtype=torch.int8, device=DEV)
+    proj[:, :H * P] = dev(case.x.reshape(T, H * P))
+    proj[:, H * P:H * P + G * N] = dev(case.B.reshape(T, G * N))
+    proj[:, H * P + G * N:] = dev(case.C.reshape(T, G * N))
+    args = [proj[:, :H * P].view(T, H, P), proj[:, H * P:H * P + G * N].view(T, G, N),
+            proj[:, H * P + G * N:].view(T, G, N), dev(case.dt.reshape(T, H)), dev(case.A),
+            dev(case.D), dev(case.x_scale), dev(case.B_scale), dev(case.C_scale), cu, 256]
+    fs = torch.full((len(lens), H, P, N), float("nan"), dtype=torch.float32, device=DEV)
+    yq = ssd_i8.ssd_i8_chunk_scan_varlen(*args, final_state=fs, y_dtype="i8", y_scale=s_y)
+    y32 = ssd_i8.ssd_i8_chunk_scan_varlen(*args, y_dtype="f32")
+    torch.cuda.synchronize()
+    yq, y32, fs = yq.cpu().numpy(), y32.cpu().numpy(), fs.cpu().numpy()
+    for (s, h), (yr, fr) in refs.items():
+        a, b = int(cu[s]), int(cu[s + 1])
+        check_i8(yq[a:b, h, :], oracle.requant(yr, s_y))
+        check_close(y32[a:b, h, :], yr, f"y of sequence {s}, head {h}")
+        check_close(fs[s, h], fr, f"final state of sequence {s}, head {h}")

@@ -66,3 +66,19 @@ def test_generation_is_seeded():
 def test_unknown_scale_recipe_is_rejected():
     with pytest.raises(ValueError):
         W.make_prefill(1, 8, 2, 64, 16, 1, 64, scales="per-channel")
+
+
+def test_varlen_lengths_fill_the_tokens_within_bounds():
+    for seed in range(5):
+        n = W.varlen_lengths(32768, 64, 8192, seed)
+        assert n.sum() == 32768 and n.max() <= 8192 and n.min() >= 1
+        assert (n[:-1] >= 64).all()  # only the last one is cut
+    assert W.varlen_lengths(0, 64, 8192, 0).size == 0
+
+
+def test_varlen_config_is_seeded_and_packed():
+    case, cu = W.make_varlen_config(total_tokens=3000)
+    case2, cu2 = W.make_varlen_config(total_tokens=3000)
+    assert np.array_equal(cu, cu2) and np.array_equal(case.x, case2.x)
+    assert cu[0] == 0 and cu[-1] == 3000 and (np.diff(cu) > 0).all()
+    assert case.batch == 1 and case.seqlen == 3000 and case.x.dtype == np.int8
