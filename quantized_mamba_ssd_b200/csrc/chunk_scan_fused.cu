@@ -79,9 +79,9 @@ constexpr int kOffHp = kOffBp + 2 * 32768;      // H' f16 [128 n][64 p] MN-major
 constexpr int kOffDm = kOffHp + 2 * 16384;      // D s_x / rho on the diagonal of [64][64] f16
 constexpr int kOffColf = kOffDm + 8192;         // off-diagonal column factors [2][192] f32
 constexpr int kOffNb = kOffColf + 2 * 768;      // -beta_s = log2(dt_s / kappa) - a_s [2][128]
-constexpr int kOffA2 = kOffNb + 2 * 512;        // a_t [2][128]
-constexpr int kOffStats = kOffA2 + 2 * 512;     // per-block statistics handed between workers [2][2]
-constexpr int kOffRed = kOffStats + 4 * 16;     // worker scratch [2][16] f32
+constexpr int kOffStats = kOffNb + 2 * 512;     // per-block statistics handed between workers [2][2]
+constexpr int kOffRed = kOffStats + 4 * 16;     // worker scratch [2][16] f32: warp sums, maxima,
+                                                // first-row dt (scan); state bounds (piece start)
 constexpr int kOffBar = kOffRed + 2 * 64;       // mbarriers [32]
 constexpr int kOffMisc = kOffBar + 32 * 8;      // TMEM base, abort flag
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
@@ -705,7 +705,6 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
         uint8_t* hp = smem + kOffHp + w * 16384;
         float* colf = reinterpret_cast<float*>(smem + kOffColf) + w * 192;
         float* nbeta = reinterpret_cast<float*>(smem + kOffNb) + w * 128;
-        float* a2s = reinterpret_cast<float*>(smem + kOffA2) + w * 128;
         float4* stats = reinterpret_cast<float4*>(smem + kOffStats);
         const uint32_t col_cb = kColCB + 128u * w;
         const uint32_t col_acc = kColAcc + 64u * w;
@@ -849,7 +848,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             // (a) output of this worker's previous block
             if (kb >= 2) output(kb - 2);
             // (b) block scan of dt (a_t = log2(e) A cumsum(dt)), with the block's max and sum
-            float incl, tot, dmax, dsum;
+            float incl, tot, dmax, dsum, a32, a64, a96;
             {
                 float v = d, mx = d;
 #pragma unroll
@@ -860,10 +859,14 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
                 if (lane == 31) red[wq] = v;
-                if (lane == 0) red[4 + wq] = mx;
+                if (lane == 0) {
+                    red[4 + wq] = mx;
+                    red[12 + wq] = d;  // the dt of the warp's first row
+                }
                 wg_sync(bar_id);
                 const float4 ws = *reinterpret_cast<const float4*>(red);
                 const float4 wm = *reinterpret_cast<const float4*>(red + 4);
+                const float4 wd = *reinterpret_cast<const float4*>(red + 12);
                 // prefix over warps in a fixed order, so that row 127 carries exactly dsum
                 const float p1 = ws.x, p2 = p1 + ws.y, p3 = p2 + ws.z;
                 const float pre = wq == 0 ? 0.f : (wq == 1 ? p1 : (wq == 2 ? p2 : p3));
@@ -871,9 +874,12 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 dmax = fmaxf(fmaxf(wm.x, wm.y), fmaxf(wm.z, wm.w));
                 incl = A2h * (v + pre);
                 tot = A2h * dsum;
-                a2s[row] = incl;
+                // a_t at rows 32, 64, 96 (the first rows of quarters 1..3): the same operations
+                // as incl in those rows, whose warp prefix is their own dt
+                a32 = A2h * (wd.y + p1);
+                a64 = A2h * (wd.z + p2);
+                a96 = A2h * (wd.w + p3);
             }
-            wg_sync(bar_id);  // a_t of every row written (read by the M' tables below)
             // (c) statistics chained through the workers: the bound hb on |H| / s_x s_B entering
             //     this block and the state unit U of the previous block
             const bool pstart = cur.c == cur.pc.cb;
@@ -948,9 +954,9 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 const float base = d * invk;
                 nbeta[row] = lg2f(base) - incl;  // dt = 0 gives -inf: no contribution
                 if (row < 96) {
-                    colf[colf_off(3) + row] = ex2f(a2s[96] - incl) * base;
-                    if (row < 64) colf[colf_off(2) + row] = ex2f(a2s[64] - incl) * base;
-                    if (row < 32) colf[colf_off(1) + row] = ex2f(a2s[32] - incl) * base;
+                    colf[colf_off(3) + row] = ex2f(a96 - incl) * base;
+                    if (row < 64) colf[colf_off(2) + row] = ex2f(a64 - incl) * base;
+                    if (row < 32) colf[colf_off(1) + row] = ex2f(a32 - incl) * base;
                 }
             }
             wg_sync(bar_id);  // x, B' (for the MMA) and the M' tables complete
@@ -961,7 +967,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             {
                 const float a2t = incl;
                 const f2 a2t2 = {a2t, a2t};
-                const float rowf = wq > 0 ? ex2f(a2t - a2s[32 * wq]) : 0.f;
+                const float rowf = wq > 0 ? ex2f(a2t - (wq == 1 ? a32 : (wq == 2 ? a64 : a96))) : 0.f;
                 const f2 rowf2 = {rowf, rowf};
                 const float* cfq = colf + colf_off(wq);
                 // off the diagonal: 2^(a_t - a_s) = 2^(a_t - a_32q) * 2^(a_32q - a_s), both <= 1
