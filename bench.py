@@ -49,7 +49,7 @@ NOMINAL_HBM_GBS = 7700.0  # B200 HBM3e datasheet bandwidth (HGX), context for th
 # profiles/ncu_fused_chunk_scan_b2_L8192.md.  The traffic grows in proportion to the tokens of a
 # launch, so the bench scales it to the workload.  A changed kernel reports null.
 _CAPTURED_TRAFFIC_PER_TOKEN = {
-    "8635a74ee3f87a87ab48cdfa787d4efc669083d79ee870ed455ad88d4e49ce64": (338.766848e6 + 118.679296e6) / 16384,
+    "ffb35d78bf2216fc860c2cc14870345d8b327bd3a6e18ee814fcd7e347b607af": (334.163968e6 + 117.367296e6) / 16384,
 }
 
 
