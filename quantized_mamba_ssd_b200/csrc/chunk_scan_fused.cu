@@ -123,6 +123,7 @@ struct FusedParams {
     // nseq non-empty sequences; without a table, nseq sequences of L tokens (nblk blocks) each
     const int4* seq_tab;
     int nseq, L, H, G, N, nblk, nctas;
+    int unit_cost;               // cost of a piece start against 4 per block in the range split
     long long dt_stride;         // elements between consecutive tokens of dt
     long long total;             // H * (blocks of all sequences)
     float* slots;                // [nctas][128 n][64 p] handed-off states, units of s_x s_B
@@ -166,11 +167,38 @@ struct Range {
         u = static_cast<long long>(lo) * H + r / nb;
         c = static_cast<int>(r % nb);
     }
+    // First block of CTA i's range.  The flattened list is cut by cost, not by blocks: every
+    // block costs 4 and the first block of each (sequence, head) unit unit_cost more (the
+    // piece switch: a state stored and loaded, bookkeeping), so that CTAs with many short
+    // units get fewer blocks.  Block f's cost starts at 4 f + unit_cost * (units starting
+    // before f); CTA i starts at the first block whose cost starts at or after
+    // floor(Wc i / nctas), Wc the total cost.  (With unit_cost > 0 only when there are at
+    // least two blocks per CTA, every window holds a block start: no range is empty.)
+    __device__ long long boundary(const FusedParams& p, int i) const {
+        if (i >= p.nctas) return p.total;
+        const long long uc = p.unit_cost;
+        const long long Wc = 4 * p.total + uc * p.nseq * static_cast<long long>(H);
+        const long long X = Wc * i / p.nctas;
+        int lo = 0, hi = p.nseq - 1;  // the last sequence whose first block's cost is <= X
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            const long long cs = static_cast<long long>(H) * (4LL * seq_entry(p, mid).z + uc * mid);
+            if (cs <= X) lo = mid;
+            else hi = mid - 1;
+        }
+        const int4 e = seq_entry(p, lo);
+        const long long nb = (e.y + kBlk - 1) / kBlk;
+        const long long r = X - static_cast<long long>(H) * (4LL * e.z + uc * lo);
+        const long long j = r / (4 * nb + uc);  // unit of the sequence
+        const long long rem = r - j * (4 * nb + uc);
+        // inside a unit, block 0's cost starts at 0 and block c >= 1's at uc + 4 c
+        const long long c = rem == 0 ? 0 : max(1LL, (rem - uc + 3) / 4);
+        return static_cast<long long>(H) * e.z + j * nb + c;
+    }
     __device__ void init(const FusedParams& p) {
-        const long long W = p.total;
-        ws = W * blockIdx.x / p.nctas;
-        we = W * (blockIdx.x + 1) / p.nctas;
         H = p.H;
+        ws = boundary(p, blockIdx.x);
+        we = boundary(p, blockIdx.x + 1);
         nseg = 0;
         u_first = u_last = 0;
         c_first = c_last = 0;
@@ -492,8 +520,9 @@ __device__ __forceinline__ float piece_state_bound(const FusedParams& p, int row
         wg_sync(bar_id);
     }
     const float* src = piece_state_src(p, seq, h, c_begin);
+    if (src == nullptr) return 0.f;  // a zero state (uniform over the worker)
     float m = 0.f;
-    if (src != nullptr && row < p.N) {
+    if (row < p.N) {
         if (c_begin != 0) {
             const float4* s4 = reinterpret_cast<const float4*>(src + row * kP);
 #pragma unroll 4
@@ -1346,6 +1375,7 @@ cudaError_t launch_chunk_scan(const ChunkScanArgs& a, cudaStream_t st) {
     const int sms = num_sms();
     if (sms <= 0) return cudaErrorInvalidDevice;
     p.nctas = static_cast<int>(std::min<long long>(std::min(sms, kMaxCtas), p.total));
+    p.unit_cost = p.total >= 2LL * p.nctas ? 1 : 0;
     uint8_t* ws = static_cast<uint8_t*>(a.workspace);
     p.status = reinterpret_cast<unsigned long long*>(ws);
     p.flags = reinterpret_cast<unsigned long long*>(ws + 256);
