@@ -4,12 +4,13 @@
 // Work: units u = (sequence, head), each a run of ceil(len / 128) blocks of 128 tokens; the
 // sequences are either `batch` rows of L tokens or packed variable-length sequences (a table of
 // first token, length and block prefix per sequence; the state starts afresh in each).
-// The flattened (unit, block) list is cut into one contiguous range per CTA, so every SM gets
-// the same number of blocks.  A range holds at most one unit piece that starts mid-sequence
-// (its first) and one that ends mid-sequence (its last).  The CTA runs its last piece first and
-// publishes the state at its end to a workspace slot; it runs its first piece last, after
-// reading the predecessor CTA's slot (a bounded wait).  With at least nblk blocks per CTA the
-// slot is always ready by then.
+// The flattened (unit, block) list is cut into one contiguous range per CTA of equal cost:
+// 4 per block and 1 more per piece start, so a CTA that holds many short units gets fewer
+// blocks.  A range holds at most one unit piece that starts mid-sequence (its first) and one
+// that ends mid-sequence (its last).  The CTA runs its last piece first and publishes the state
+// at its end to a workspace slot; it runs its first piece last, after reading the predecessor
+// CTA's slot (a bounded wait).  With at least nblk blocks per CTA the slot is always ready by
+// then.
 //
 // The chunked scan is evaluated in blocks of 128 tokens (SSDi8 page: ChunkState, state path,
 // ChunkScan, ChunkBMM of Table 5; X_scaled of Figure 3(a)).  This is the same recurrence for
