@@ -49,7 +49,7 @@ NOMINAL_HBM_GBS = 7700.0  # B200 HBM3e datasheet bandwidth (HGX), context for th
 # profiles/ncu_fused_chunk_scan_b2_L8192.md.  The traffic grows in proportion to the tokens of a
 # launch, so the bench scales it to the workload.  A changed kernel reports null.
 _CAPTURED_TRAFFIC_PER_TOKEN = {
-    "ffb35d78bf2216fc860c2cc14870345d8b327bd3a6e18ee814fcd7e347b607af": (334.163968e6 + 117.367296e6) / 16384,
+    "77635acbb725d88e8ff7820df0837e5e61cfb48b8edfc3e471302a80cb6e654d": (330.561024e6 + 116.753152e6) / 16384,
 }
 
 
