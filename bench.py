@@ -53,11 +53,32 @@ _CAPTURED_TRAFFIC_PER_TOKEN = {
 }
 
 
-def captured_traffic(tokens: int):
+# The same for the decode kernels, per (batch, head) item of one step; see
+# profiles/ncu_state_update_decode_b32.md and profiles/ncu_state_update_q8_decode_b128.md.
+_CAPTURED_DECODE_TRAFFIC_PER_ITEM = {
+    "state_update.cu": {
+        "562e8c1b5451d3c1c4461d0695738535cba2ca35b3b7ee7fd354a78db864eb83": (134.587904e6 + 76.073984e6) / (32 * 128),
+    },
+    "state_update_q8.cu": {
+        "ff2801f6675cd1af6669cf61f0875ce58c99cd3ecf6964a44a2f6df0b30a2a13": (135.689216e6 + 77.368832e6) / (128 * 128),
+    },
+}
+
+
+def _source_sha(name: str) -> str:
     import hashlib
-    src = Path(__file__).resolve().parent / "quantized_mamba_ssd_b200" / "csrc" / "chunk_scan_fused.cu"
-    per_token = _CAPTURED_TRAFFIC_PER_TOKEN.get(hashlib.sha256(src.read_bytes()).hexdigest())
+    src = Path(__file__).resolve().parent / "quantized_mamba_ssd_b200" / "csrc" / name
+    return hashlib.sha256(src.read_bytes()).hexdigest()
+
+
+def captured_traffic(tokens: int):
+    per_token = _CAPTURED_TRAFFIC_PER_TOKEN.get(_source_sha("chunk_scan_fused.cu"))
     return None if per_token is None else per_token * tokens
+
+
+def captured_decode_traffic(kernel_source: str, items: int):
+    per_item = _CAPTURED_DECODE_TRAFFIC_PER_ITEM[kernel_source].get(_source_sha(kernel_source))
+    return None if per_item is None else per_item * items
 
 
 def prefill_alg_bytes(c: W.PrefillCase, out_bytes: int, final_state: bool) -> int:
@@ -588,7 +609,8 @@ def main():
             "ms_per_512_steps": dms, "us_per_step": 1e3 * dms / d.steps,
             "workload": d.name, "gpu_launches_per_pass": d.steps,
             "roofline": {"bound": "hbm", "achieved": dgbs, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": dgbs / hbm_peak, "traffic": None,
+                         "frac": dgbs / hbm_peak,
+                         "traffic": captured_decode_traffic("state_update.cu", d.batch * d.nheads),
                          "alg_bytes_per_launch": decode_alg_bytes(d, 2)},
         }
         del graph
@@ -628,7 +650,8 @@ def main():
             "ms_per_512_steps": qms, "us_per_step": 1e3 * qms / d.steps,
             "gpu_launches_per_pass": d.steps,
             "roofline": {"bound": "hbm", "achieved": qgbs, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": qgbs / hbm_peak, "traffic": None,
+                         "frac": qgbs / hbm_peak,
+                         "traffic": captured_decode_traffic("state_update_q8.cu", d.batch * d.nheads),
                          "alg_bytes_per_launch": qstep},
         }
         del graph
