@@ -93,7 +93,8 @@ SSD_API size_t ssd_i8_chunk_scan_workspace_size(int batch, int seqlen, int nhead
  *   y          [batch, seqlen, nheads, headdim] of y_dtype
  *   workspace  device memory of at least ssd_i8_chunk_scan_workspace_size(...) bytes,
  *              256-byte aligned.
- * Supported: headdim == 64; dstate in {16, 32, 64, 128}; seqlen >= 0 (seqlen == 0 only copies
+ * Supported: headdim == 64; dstate in {16, 32, 64, 128}; batch * nheads < 2^31 (larger:
+ * SSD_ERR_UNSUPPORTED); seqlen >= 0 (seqlen == 0 only copies
  * init_state to final_state); batch >= 0; nheads % ngroups == 0; x, B, C and y 16-byte
  * aligned.  Expected ranges: A <= 0 and dt >= 0 (a decaying state); other values are computed
  * but without the range guarantees the f16 operand scaling relies on.
@@ -138,8 +139,9 @@ SSD_API size_t ssd_i8_chunk_scan_varlen_workspace_size(int nseq);
  *   workspace  at least ssd_i8_chunk_scan_varlen_workspace_size(nseq) bytes, 256-byte aligned.
  * The sequence table is uploaded with cudaMemcpyAsync from host memory on `stream` (staged
  * before the call returns), so the call cannot be captured into a CUDA graph.  Shapes, base
- * alignments and error reporting are those of ssd_i8_chunk_scan; SSD_ERR_INVALID_ARG also
- * covers malformed cu_seqlens and strides.
+ * alignments and error reporting are those of ssd_i8_chunk_scan (with the non-empty sequences
+ * in place of batch: their count times nheads < 2^31); SSD_ERR_INVALID_ARG also covers
+ * malformed cu_seqlens and strides.
  */
 SSD_API ssd_status ssd_i8_chunk_scan_varlen(const int8_t *x, long long x_token_stride,
                                             const int8_t *B, const int8_t *C,

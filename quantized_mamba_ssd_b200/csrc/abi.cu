@@ -74,6 +74,8 @@ ssd_status ssd_i8_chunk_scan(const int8_t* x, const int8_t* B, const int8_t* C, 
     if (!A || !D || !x_scale || !B_scale || !C_scale) return SSD_ERR_INVALID_ARG;
     if (headdim != 64 || !chunk_dstate_ok(dstate) || !chunk_size_ok(chunk_size))
         return SSD_ERR_UNSUPPORTED;
+    // the kernel indexes (sequence, head) units with 32-bit integers
+    if ((long long)batch * nheads > 0x7fffffffLL) return SSD_ERR_UNSUPPORTED;
     float inv = 1.f;
     if (!out_scale(y_dtype, y_scale, &inv)) return SSD_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -167,7 +169,8 @@ ssd_status ssd_i8_chunk_scan_varlen(const int8_t* x, long long x_token_stride, c
         blocks += (len + 127) / 128;
     }
     if (tab.empty()) return SSD_OK;
-    if (blocks > 0x7fffffffLL) return SSD_ERR_UNSUPPORTED;
+    if (blocks > 0x7fffffffLL || (long long)(tab.size() / 4) * nheads > 0x7fffffffLL)
+        return SSD_ERR_UNSUPPORTED;
     if (!x || !B || !C || !dt || !y) return SSD_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(B) || !aligned16(C) || !aligned16(y)) return SSD_ERR_INVALID_ARG;
     uint8_t* table = static_cast<uint8_t*>(workspace) + ssd::chunk_scan_varlen_table_offset();

@@ -84,6 +84,7 @@ def _scan_args(**over):
     (dict(P=32), 2),              # headdim not implemented
     (dict(N=48), 2),              # dstate not implemented
     (dict(Q=100), 2),             # chunk size not implemented
+    (dict(batch=1 << 24, H=256), 2),  # 2^32 (sequence, head) units: beyond 32-bit indexing
     (dict(ws=None), 3),           # workspace missing
     (dict(wsb=16), 3),            # workspace too small
     (dict(ws=257), 3),            # workspace misaligned
