@@ -8,7 +8,8 @@ Functions follow the pages' statement of the problem (see ``ssd_oracle.c`` for t
 definitions and their sources):
 
 * :func:`scan` -- sequential fp64 recurrence over a prefill, with optional initial state,
-  final state and an additive per-step state perturbation (for the error-accumulation check).
+  final state and an additive per-step state perturbation (for the error-accumulation check);
+  B and C scales per group, or per group and dstate channel.
 * :func:`step` -- one decode step on an fp64 state.
 * :func:`chunk_cb` -- SSDi8's ChunkBMM matrix CB = Cq Bq^T per chunk and group, int64.
 * :func:`requant` -- static symmetric int8 requantization of an output.
@@ -59,6 +60,8 @@ def load() -> ctypes.CDLL:
             ci = ctypes.c_int
             lib.ssd_oracle_scan.restype = ci
             lib.ssd_oracle_scan.argtypes = [vp] * 9 + [ci] * 6 + [vp] * 4 + [ci]
+            lib.ssd_oracle_scan_pern.restype = ci
+            lib.ssd_oracle_scan_pern.argtypes = [vp] * 9 + [ci] * 6 + [vp] * 4 + [ci]
             lib.ssd_oracle_step.restype = ci
             lib.ssd_oracle_step.argtypes = [vp] * 10 + [ci] * 5 + [vp, ci]
             lib.ssd_oracle_chunk_cb.restype = ci
@@ -83,12 +86,15 @@ def _opt(a, dtype):
 def scan(x, B, C, dt, A, D, x_scale, B_scale, C_scale, *, init_state=None, eps=None,
          want_final_state=True, nthreads: int = 0):
     """fp64 sequential scan.  Shapes: x [b,l,h,p] int8, B/C [b,l,g,n] int8, dt [b,l,h] f32,
-    A/D/x_scale [h] f32, B_scale/C_scale [g] f32, init_state [b,h,p,n] (any float),
-    eps [b,l,h,p,n] (any float).  Returns (y f64 [b,l,h,p], final_state f64 or None,
-    threads used)."""
+    A/D/x_scale [h] f32, B_scale/C_scale [g] f32 -- or both [g, n], one scale per dstate
+    channel --, init_state [b,h,p,n] (any float), eps [b,l,h,p,n] (any float).  Returns
+    (y f64 [b,l,h,p], final_state f64 or None, threads used)."""
     lib = load()
     bsz, L, H, P = x.shape
     G, N = B.shape[2], B.shape[3]
+    per_n = np.ndim(B_scale) == 2
+    if np.shape(B_scale) != ((G, N) if per_n else (G,)) or np.shape(C_scale) != np.shape(B_scale):
+        raise ValueError("B_scale and C_scale must both be [g] or both be [g, n]")
     keep = []
     args = []
     for a, t in ((x, np.int8), (B, np.int8), (C, np.int8), (dt, np.float32), (A, np.float32),
@@ -101,9 +107,10 @@ def scan(x, B, C, dt, A, D, x_scale, B_scale, C_scale, *, init_state=None, eps=N
     ep, peps = _opt(eps, np.float64)
     y = np.zeros((bsz, L, H, P), dtype=np.float64)
     fs = np.zeros((bsz, H, P, N), dtype=np.float64) if want_final_state else None
-    r = lib.ssd_oracle_scan(*args, bsz, L, H, P, N, G, pinit, peps,
-                            None if fs is None else fs.ctypes.data_as(ctypes.c_void_p),
-                            y.ctypes.data_as(ctypes.c_void_p), nthreads)
+    fn = lib.ssd_oracle_scan_pern if per_n else lib.ssd_oracle_scan
+    r = fn(*args, bsz, L, H, P, N, G, pinit, peps,
+           None if fs is None else fs.ctypes.data_as(ctypes.c_void_p),
+           y.ctypes.data_as(ctypes.c_void_p), nthreads)
     if r < 0:
         raise ValueError(f"ssd_oracle_scan failed ({r})")
     del keep, init, ep

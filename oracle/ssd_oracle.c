@@ -9,6 +9,8 @@
  *
  *   dequantize   x_t[p] = s_x[h] * xq[b,t,h,p]
  *                B_t[n] = s_B[g] * Bq[b,t,g,n],  C_t[n] = s_C[g] * Cq[b,t,g,n],  g = h / (H/G)
+ *                (ssd_oracle_scan_pern: s_B[g, n] and s_C[g, n], one scale per dstate channel
+ *                -- the per-N axis of SSDi8's quantization-axis table, Table 10)
  *   recurrence   h_t = Abar_t * h_{t-1} + Bbar_t x_t
  *                ("Ternary Mamba: Grouped QAT of W1.58A16 SSMs", section 1, the SSM recurrence)
  *   discretised  Abar_t = exp(dt_t * A_h),   Bbar_t x_t = dt_t * x_t B_t^T   (Mamba-2 form)
@@ -44,6 +46,7 @@ typedef struct {
     double *y;                /* [b,l,h,p] */
     int next;                 /* next (b,h) work item, taken atomically */
     int status;
+    int bc_per_n;             /* sB, sC are [g, n] (per dstate channel) instead of [g] */
 } scan_job;
 
 static void scan_pair(scan_job *j, int b, int h)
@@ -66,8 +69,10 @@ static void scan_pair(scan_job *j, int b, int h)
         const double dtv = (double)j->dt[bt * H + h];
         const double abar = exp(dtv * (double)j->A[h]);
         for (int n = 0; n < N; ++n) {
-            Bt[n] = (double)j->sB[g] * (double)j->B[(bt * G + g) * N + n];
-            Ct[n] = (double)j->sC[g] * (double)j->C[(bt * G + g) * N + n];
+            const double sb = (double)(j->bc_per_n ? j->sB[g * N + n] : j->sB[g]);
+            const double sc = (double)(j->bc_per_n ? j->sC[g * N + n] : j->sC[g]);
+            Bt[n] = sb * (double)j->B[(bt * G + g) * N + n];
+            Ct[n] = sc * (double)j->C[(bt * G + g) * N + n];
         }
         for (int p = 0; p < P; ++p) {
             const double xv = (double)j->sx[h] * (double)j->x[(bt * H + h) * P + p];
@@ -135,6 +140,26 @@ static int run_pool(void *(*fn)(void *), void *job, int nthreads)
     return 0;
 }
 
+static int scan_impl(const int8_t *x, const int8_t *B, const int8_t *C, const float *dt,
+                     const float *A, const float *D, const float *x_scale, const float *B_scale,
+                     const float *C_scale, int batch, int seqlen, int nheads, int headdim,
+                     int dstate, int ngroups, const double *init_state, const double *eps,
+                     double *final_state, double *y, int nthreads, int bc_per_n)
+{
+    if (batch < 0 || seqlen < 0 || nheads <= 0 || headdim <= 0 || dstate <= 0 || ngroups <= 0 ||
+        nheads % ngroups != 0)
+        return -1;
+    scan_job j = {x, B, C, dt, A, D, x_scale, B_scale, C_scale, batch, seqlen, nheads, headdim,
+                  dstate, ngroups, init_state, eps, final_state, y, 0, 0, bc_per_n};
+    const int items = batch * nheads;
+    if (items == 0)
+        return 0;
+    const int nt = pick_threads(nthreads, items);
+    if (run_pool(scan_worker, &j, nt) != 0 || j.status != 0)
+        return -2;
+    return nt;
+}
+
 /* Sequential fp64 scan over a whole prefill.  Returns the number of threads used, or a
  * negative value on bad arguments / allocation failure. */
 int ssd_oracle_scan(const int8_t *x, const int8_t *B, const int8_t *C, const float *dt,
@@ -143,18 +168,20 @@ int ssd_oracle_scan(const int8_t *x, const int8_t *B, const int8_t *C, const flo
                     int dstate, int ngroups, const double *init_state, const double *eps,
                     double *final_state, double *y, int nthreads)
 {
-    if (batch < 0 || seqlen < 0 || nheads <= 0 || headdim <= 0 || dstate <= 0 || ngroups <= 0 ||
-        nheads % ngroups != 0)
-        return -1;
-    scan_job j = {x, B, C, dt, A, D, x_scale, B_scale, C_scale, batch, seqlen, nheads, headdim,
-                  dstate, ngroups, init_state, eps, final_state, y, 0, 0};
-    const int items = batch * nheads;
-    if (items == 0)
-        return 0;
-    const int nt = pick_threads(nthreads, items);
-    if (run_pool(scan_worker, &j, nt) != 0 || j.status != 0)
-        return -2;
-    return nt;
+    return scan_impl(x, B, C, dt, A, D, x_scale, B_scale, C_scale, batch, seqlen, nheads,
+                     headdim, dstate, ngroups, init_state, eps, final_state, y, nthreads, 0);
+}
+
+/* The same scan with B_scale and C_scale given per group and dstate channel, [g, n]. */
+int ssd_oracle_scan_pern(const int8_t *x, const int8_t *B, const int8_t *C, const float *dt,
+                         const float *A, const float *D, const float *x_scale,
+                         const float *B_scale, const float *C_scale, int batch, int seqlen,
+                         int nheads, int headdim, int dstate, int ngroups,
+                         const double *init_state, const double *eps, double *final_state,
+                         double *y, int nthreads)
+{
+    return scan_impl(x, B, C, dt, A, D, x_scale, B_scale, C_scale, batch, seqlen, nheads,
+                     headdim, dstate, ngroups, init_state, eps, final_state, y, nthreads, 1);
 }
 
 /* One decode step on an fp64 state held by the caller (updated in place). */

@@ -49,12 +49,16 @@ def _run(c, **kw):
 
 
 def _deq(c):
+    """Dequantized x [b,l,h,p] and B, C expanded to heads [b,l,h,n]; B/C scales per group [g]
+    or per group and dstate channel [g, n]."""
     H, G = c.nheads, c.ngroups
     gi = np.arange(H) // (H // G)
     x = c.x.astype(np.float64) * c.x_scale.astype(np.float64)[None, None, :, None]
-    Bf = c.B.astype(np.float64) * c.B_scale.astype(np.float64)[None, None, :, None]
-    Cf = c.C.astype(np.float64) * c.C_scale.astype(np.float64)[None, None, :, None]
-    return x, Bf[:, :, gi, :], Cf[:, :, gi, :]  # B, C expanded to heads: [b,l,h,n]
+    per_group = lambda s: s.astype(np.float64)[None, None, :, None] if s.ndim == 1 else \
+        s.astype(np.float64)[None, None, :, :]
+    Bf = c.B.astype(np.float64) * per_group(c.B_scale)
+    Cf = c.C.astype(np.float64) * per_group(c.C_scale)
+    return x, Bf[:, :, gi, :], Cf[:, :, gi, :]
 
 
 def quadratic_form(c):
@@ -320,6 +324,65 @@ def test_requant_rule():
 
 
 # ----------------------------------------------------------------------------------------
+# B and C scales per dstate channel (the per-N axis of SSDi8's quantization-axis table)
+# ----------------------------------------------------------------------------------------
+def _per_n_case(seed=7, b=1, L=20, H=4, G=2, P=3, N=6):
+    c = _case(b=b, L=L, H=H, G=G, P=P, N=N, seed=seed)
+    rng = np.random.default_rng(seed + 100)
+    c.B_scale = (c.B_scale[:, None] * rng.uniform(0.25, 4.0, size=(G, N))).astype(np.float32)
+    c.C_scale = (c.C_scale[:, None] * rng.uniform(0.25, 4.0, size=(G, N))).astype(np.float32)
+    return c
+
+
+def test_per_n_scales_constant_over_n_equal_per_group():
+    c = _case(seed=5)
+    y, fs, _ = _run(c)
+    N = c.dstate
+    c.B_scale = np.repeat(c.B_scale[:, None], N, axis=1)
+    c.C_scale = np.repeat(c.C_scale[:, None], N, axis=1)
+    y2, fs2, _ = _run(c)
+    assert np.array_equal(y, y2) and np.array_equal(fs, fs2)
+
+
+@pytest.mark.parametrize("seed", [7, 8])
+def test_per_n_duality_quadratic_form(seed):
+    c = _per_n_case(seed=seed)
+    y, fs, _ = _run(c)
+    yq, hq = quadratic_form(c)
+    assert np.abs(y - yq).max() <= 1e-12 * np.abs(yq).max()
+    assert np.abs(fs - hq).max() <= 1e-12 * np.abs(hq).max()
+
+
+def test_per_n_scale_acts_on_its_own_channel():
+    # h_t[p, n] is linear in s_B[g, n] alone and does not involve C: doubling s_B[g, k] (a
+    # power of two, so exactly) doubles column k of the states of group g's heads and nothing
+    # else; doubling s_C[g, k] leaves every state as it was and changes y
+    c = _per_n_case(seed=9)
+    c.init_state = None
+    y, fs, _ = _run(c)
+    H, G = c.nheads, c.ngroups
+    g, k = 1, 4
+    heads = np.arange(H)[np.arange(H) // (H // G) == g]
+    c2 = _per_n_case(seed=9)
+    c2.init_state = None
+    c2.B_scale = c2.B_scale.copy()
+    c2.B_scale[g, k] *= 2
+    y2, fs2, _ = _run(c2)
+    expect = fs.copy()
+    expect[:, heads, :, k] *= 2
+    assert np.array_equal(fs2, expect)
+    c3 = _per_n_case(seed=9)
+    c3.init_state = None
+    c3.C_scale = c3.C_scale.copy()
+    c3.C_scale[g, k] *= 2
+    y3, fs3, _ = _run(c3)
+    assert np.array_equal(fs3, fs)
+    assert not np.array_equal(y3[:, :, heads], y[:, :, heads])
+    others = np.setdiff1d(np.arange(H), heads)
+    assert np.array_equal(y3[:, :, others], y[:, :, others])
+
+
+# ----------------------------------------------------------------------------------------
 # planted mistakes: each broken copy of the oracle must fail at least one pin above
 # ----------------------------------------------------------------------------------------
 MUTANTS = {
@@ -328,7 +391,10 @@ MUTANTS = {
     "flip_decay_sign": ("exp(dtv * (double)j->A[h])", "exp(-dtv * (double)j->A[h])"),
     "drop_dt_on_input": ("row[n] = abar * row[n] + dtv * xv * Bt[n];",
                          "row[n] = abar * row[n] + xv * Bt[n];"),
-    "C_reads_B": ("Ct[n] = (double)j->sC[g] * (double)j->C[", "Ct[n] = (double)j->sC[g] * (double)j->B["),
+    "C_reads_B": ("Ct[n] = sc * (double)j->C[", "Ct[n] = sc * (double)j->B["),
+    "per_n_scale_of_first_channel": ("j->sB[g * N + n] : j->sB[g]", "j->sB[g * N] : j->sB[g]"),
+    "per_n_B_scale_read_from_C": ("(double)(j->bc_per_n ? j->sB[g * N + n]",
+                                  "(double)(j->bc_per_n ? j->sC[g * N + n]"),
     "wrong_group_index": ("const int g = h / (H / G);", "const int g = h % G;"),
     "cb_transposed": ("(int64_t)C[(((size_t)b * L + lt) * G + g) * N + n] *\n                                       (int64_t)B[(((size_t)b * L + ls) * G + g) * N + n]",
                       "(int64_t)C[(((size_t)b * L + ls) * G + g) * N + n] *\n                                       (int64_t)B[(((size_t)b * L + lt) * G + g) * N + n]"),
@@ -346,6 +412,9 @@ def _pins_pass():
         test_chunk_cb_against_python_integers_and_einsum,
         test_requant_rule,
         test_zero_B_leaves_skip_term_only,
+        test_per_n_scales_constant_over_n_equal_per_group,
+        lambda: test_per_n_duality_quadratic_form(7),
+        test_per_n_scale_acts_on_its_own_channel,
     ]
     for chk in checks:
         try:
@@ -370,7 +439,8 @@ def test_pins_reject_planted_mistake(mutant, monkeypatch):
                         "-shared", "-o", so, path, "-lm", "-lpthread"], check=True)
         good = oracle.load()
         lib = ctypes.CDLL(so)
-        for name in ("ssd_oracle_scan", "ssd_oracle_step", "ssd_oracle_chunk_cb", "ssd_oracle_requant"):
+        for name in ("ssd_oracle_scan", "ssd_oracle_scan_pern", "ssd_oracle_step",
+                     "ssd_oracle_chunk_cb", "ssd_oracle_requant"):
             getattr(lib, name).restype = getattr(good, name).restype
             getattr(lib, name).argtypes = getattr(good, name).argtypes
         monkeypatch.setattr(oracle, "_lib", lib)
