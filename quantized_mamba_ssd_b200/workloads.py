@@ -64,8 +64,8 @@ class PrefillCase:
     A: np.ndarray  # f32 [h]
     D: np.ndarray  # f32 [h]
     x_scale: np.ndarray  # f32 [h]
-    B_scale: np.ndarray  # f32 [g]
-    C_scale: np.ndarray  # f32 [g]
+    B_scale: np.ndarray  # f32 [g] (or [g, n] for scales="channel")
+    C_scale: np.ndarray  # f32 [g] (or [g, n] for scales="channel")
     out_dtype: str = "f16"  # "f32" | "f16" | "i8"
     init_state: Optional[np.ndarray] = None  # f32 [b, h, p, n]
 
@@ -127,12 +127,12 @@ DECODE_CONFIG = dict(name="mamba2-8b-ssd-decode b128 x512 steps h128 p64 n128 g8
                      steps=512, nheads=128, headdim=64, dstate=128, ngroups=8, out_dtype="f16")
 
 
-def quantize_symmetric(v: np.ndarray, scale_axis: Optional[int]) -> tuple[np.ndarray, np.ndarray]:
+def quantize_symmetric(v: np.ndarray, scale_axis) -> tuple[np.ndarray, np.ndarray]:
     """Static symmetric int8 quantization: s = absmax / 127, q = clamp(rne(v / s), -127, 127).
 
-    ``scale_axis`` is the axis that keeps its own scale (per head / per group); ``None``
-    gives one per-tensor scale.  Returns (q int8, s f32[...]); s has one entry per index of
-    ``scale_axis`` (or a single entry).
+    ``scale_axis`` is the axis that keeps its own scale (per head / per group), or a tuple of
+    axes (per group and dstate channel); ``None`` gives one per-tensor scale.  Returns
+    (q int8, s f32[...]); s has one entry per index of the kept axes (or a single entry).
     """
     v = np.asarray(v, dtype=F32)
     if v.ndim == 0:
@@ -141,10 +141,12 @@ def quantize_symmetric(v: np.ndarray, scale_axis: Optional[int]) -> tuple[np.nda
     if scale_axis is None:
         amax = np.array([np.abs(v).max() if v.size else 0.0], dtype=np.float64)
     else:
-        axes = tuple(i for i in range(v.ndim) if i != scale_axis)
+        keep = (scale_axis,) if isinstance(scale_axis, int) else tuple(scale_axis)
+        axes = tuple(i for i in range(v.ndim) if i not in keep)
         amax = (np.abs(v).max(axis=axes).astype(np.float64) if v.size
-                else np.zeros(v.shape[scale_axis]))
-        shape[scale_axis] = v.shape[scale_axis]
+                else np.zeros(tuple(v.shape[k] for k in keep)))
+        for k in keep:
+            shape[k] = v.shape[k]
     s = np.where(amax > 0, amax / 127.0, 1.0).astype(F32)
     sb = s.reshape(shape)
     q = np.empty(v.shape, dtype=np.int8)
@@ -215,8 +217,10 @@ def make_prefill(batch: int, seqlen: int, nheads: int, headdim: int, dstate: int
     channels x20 over (h,p); B, C ~ N(0,1)); "laplace_spread" (x, B, C Laplace, x scaled
     per head and B, C per group by U(0.5, 8)); "laplace_outliers_all" (x, B, C Laplace with
     1 % outlier channels x20: x over (h,p), B and C over (g,n)).
-    scales: "tensor" (one scale per tensor, broadcast), "head" (x per head, B/C per group) or
-    "percentile" (per tensor; x clipped at ``clip_percentile`` of |x|, B/C by absmax).
+    scales: "tensor" (one scale per tensor, broadcast), "head" (x per head, B/C per group),
+    "channel" (x per head, B/C per group and dstate channel, [g, n] -- the oracle's per-N
+    scan; the CUDA kernels take per-group scales) or "percentile" (per tensor; x clipped at
+    ``clip_percentile`` of |x|, B/C by absmax).
     """
     if nheads % ngroups:
         raise ValueError("nheads must be a multiple of ngroups")
@@ -269,6 +273,10 @@ def make_prefill(batch: int, seqlen: int, nheads: int, headdim: int, dstate: int
         xq, sx = quantize_symmetric(x, 2)
         Bq, sb = quantize_symmetric(Bf, 2)
         Cq, sc = quantize_symmetric(Cf, 2)
+    elif scales == "channel":  # x per head; B and C per group and dstate channel: [g, n]
+        xq, sx = quantize_symmetric(x, 2)
+        Bq, sb = quantize_symmetric(Bf, (2, 3))
+        Cq, sc = quantize_symmetric(Cf, (2, 3))
     else:
         raise ValueError(f"unknown scales {scales!r}")
     del x, Bf, Cf

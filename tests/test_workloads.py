@@ -82,3 +82,22 @@ def test_varlen_config_is_seeded_and_packed():
     assert np.array_equal(cu, cu2) and np.array_equal(case.x, case2.x)
     assert cu[0] == 0 and cu[-1] == 3000 and (np.diff(cu) > 0).all()
     assert case.batch == 1 and case.seqlen == 3000 and case.x.dtype == np.int8
+
+
+def test_channel_scales_quantize_each_dstate_channel():
+    c = W.make_prefill(2, 50, 4, 8, 6, 2, 64, law="laplace_outliers_all", scales="channel", seed=3)
+    assert c.B_scale.shape == (2, 6) and c.C_scale.shape == (2, 6) and c.x_scale.shape == (4,)
+    # every (group, channel) slice reaches the full code range, so its scale is its own absmax
+    for q in (c.B, c.C):
+        assert (np.abs(q.astype(np.int16)).max(axis=(0, 1)) == 127).all()
+    # the per-head path keeps its scales and codes bit for bit
+    a = W.make_prefill(2, 50, 4, 8, 6, 2, 64, law="laplace_outliers_all", scales="head", seed=3)
+    assert np.array_equal(a.x, c.x) and np.array_equal(a.x_scale, c.x_scale)
+    assert a.B_scale.shape == (2,)
+
+
+def test_oracle_runs_on_channel_scales():
+    import oracle
+    c = W.make_prefill(1, 40, 4, 3, 6, 2, 64, law="normal", scales="channel", seed=4)
+    y, fs, _ = oracle.scan(c.x, c.B, c.C, c.dt, c.A, c.D, c.x_scale, c.B_scale, c.C_scale)
+    assert np.isfinite(y).all() and fs.shape == (1, 4, 3, 6)
