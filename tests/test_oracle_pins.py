@@ -504,6 +504,86 @@ def test_step_q8_with_zero_dt_keeps_the_cache():
     assert np.allclose(y, yref, rtol=1e-12, atol=1e-12)
 
 
+def _golden_step_q8_inputs():
+    with open(os.path.join(GOLDEN, "handworked_step_q8.json")) as f:
+        g = json.load(f)
+    codes = np.array(g["codes"], np.int8)[None, None]
+    scale = np.array([[g["scale"]]], np.float64)
+    ins = dict(x=np.array(g["x_q"], np.int8)[None, None], B=np.array(g["B_q"], np.int8)[None, None],
+               C=np.array(g["C_q"], np.int8)[None, None], dt=np.array([g["dt"]], np.float32),
+               A=np.array(g["A"], np.float32), D=np.array(g["D"], np.float32),
+               x_scale=np.array(g["x_scale"], np.float32),
+               B_scale=np.array(g["B_scale"], np.float32),
+               C_scale=np.array(g["C_scale"], np.float32))
+    return g, codes, scale, ins
+
+
+def test_golden_handworked_step_q8():
+    # a step whose max |h| grows: the fresh scale differs from the incoming one
+    g, codes, scale, ins = _golden_step_q8_inputs()
+    y, c2, s2 = oracle.step_q8(codes, scale, **ins)
+    assert np.allclose(y[0, 0], g["y"], rtol=g["rtol"], atol=0)
+    assert np.array_equal(c2[0, 0], np.array(g["new_codes"], np.int8))
+    assert np.isclose(s2[0, 0], g["new_scale"], rtol=g["rtol"], atol=0)
+    assert not np.isclose(s2[0, 0], g["scale"], rtol=1e-2)
+
+
+def test_step_q8_codes_follow_the_fresh_scale():
+    # random caches and inputs: each new code is within half a fresh step of the fp64 step of
+    # the dequantised cache, the largest element gets code +-127 and the scale is its |h| / 127
+    bsz, H, P, N, G = 2, 4, 8, 16, 2
+    codes, scales = oracle.quantize_state(_random_state(25, (bsz, H, P, N), sd=0.3))
+    rng = np.random.default_rng(26)
+    x = rng.integers(-127, 128, size=(bsz, H, P), dtype=np.int8)
+    B = rng.integers(-127, 128, size=(bsz, G, N), dtype=np.int8)
+    C = rng.integers(-127, 128, size=(bsz, G, N), dtype=np.int8)
+    A = -np.exp(rng.uniform(0, np.log(16), H)).astype(np.float32)
+    D = rng.normal(size=H).astype(np.float32)
+    sx, sB, sC = (np.full(k, v, np.float32) for k, v in ((H, 0.02), (G, 0.03), (G, 0.04)))
+    dt = rng.uniform(0.05, 0.3, size=(bsz, H)).astype(np.float32)
+    y, c2, s2 = oracle.step_q8(codes, scales, x, B, C, dt, A, D, sx, sB, sC)
+    h = np.ascontiguousarray(codes.astype(np.float64) * scales[:, :, None, None])
+    yref = oracle.step(h, x, B, C, dt, A, D, sx, sB, sC)
+    assert np.array_equal(y, yref)
+    m = np.abs(h).reshape(bsz, H, -1).max(axis=2)
+    assert np.allclose(s2, m / 127.0, rtol=1e-15, atol=0)
+    assert (np.abs(c2.astype(np.float64) * s2[:, :, None, None] - h)
+            <= 0.5 * s2[:, :, None, None] * (1 + 1e-12)).all()
+    assert (np.abs(c2).reshape(bsz, H, -1).max(axis=2) == 127).all()
+
+
+def _step_q8_with_incoming_scale(codes, scales, x, B, C, dt, A, D, x_scale, B_scale, C_scale):
+    # planted mistake: requantise the updated state with the scale the cache came in with
+    state = np.ascontiguousarray(codes.astype(np.float64) * scales[:, :, None, None])
+    y = oracle.step(state, x, B, C, dt, A, D, x_scale, B_scale, C_scale)
+    c2 = np.zeros_like(codes)
+    for b in range(codes.shape[0]):
+        for h in range(codes.shape[1]):
+            if scales[b, h] > 0:
+                c2[b, h] = oracle.requant(state[b, h], scales[b, h])
+    return y, c2, np.array(scales, dtype=np.float64)
+
+
+def _step_q8_keeping_codes(codes, scales, x, B, C, dt, A, D, x_scale, B_scale, C_scale):
+    # planted mistake: return the incoming codes and scale
+    state = np.ascontiguousarray(codes.astype(np.float64) * scales[:, :, None, None])
+    y = oracle.step(state, x, B, C, dt, A, D, x_scale, B_scale, C_scale)
+    return y, codes.copy(), np.array(scales, dtype=np.float64)
+
+
+@pytest.mark.parametrize("broken", [_step_q8_with_incoming_scale, _step_q8_keeping_codes])
+def test_step_q8_pins_reject_planted_mistake(broken, monkeypatch):
+    monkeypatch.setattr(oracle, "step_q8", broken)
+    failed = 0
+    for chk in (test_golden_handworked_step_q8, test_step_q8_with_zero_dt_keeps_the_cache,
+                test_step_q8_codes_follow_the_fresh_scale):
+        try:
+            chk()
+        except AssertionError:
+            failed += 1
+    assert failed > 0, f"planted mistake {broken.__name__} passed every step_q8 pin"
+
+
 # ---- Hadamard output transform ----
 
 def test_hadamard_is_an_involution():
