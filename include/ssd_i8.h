@@ -186,8 +186,9 @@ SSD_API ssd_status ssd_i8_debug_inject(int drop_publish_cta, long long wait_cycl
  * every GPU that loads the library holds until the process exits.  The call allocates nothing
  * (no cudaMalloc / cudaFree, no allocating library routine).
  *   - Size limit: problems whose ssd_i8_chunk_scan_workspace_size(...) exceeds 4 MiB
- *     (4194304 bytes; up to 127 batch x head x chunk work items) are rejected with
- *     SSD_ERR_WORKSPACE before anything is launched.
+ *     (4194304 bytes) are rejected with SSD_ERR_WORKSPACE before anything is launched.  The
+ *     kernel works in blocks of 128 tokens whatever chunk_size is, and that size counts them:
+ *     the limit is batch * nheads * ceil(seqlen / 128) <= 127.
  *   - Device: the scratch of the device that is current at the call is used; `stream` must
  *     belong to that device.  The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) and caches it; make that first call before any stream capture.
@@ -205,6 +206,16 @@ SSD_API ssd_status ssd_i8_chunk_scan_noalloc(const int8_t *x, const int8_t *B, c
                                              int chunk_size, const float *init_state,
                                              float *final_state, void *y, int y_dtype,
                                              float y_scale, void *stream);
+
+/*
+ * Status of the last ssd_i8_chunk_scan_noalloc call on the current device -- the counterpart of
+ * ssd_i8_chunk_scan_status for callers that have no workspace to pass: synchronises `stream`,
+ * then returns SSD_ERR_TIMEOUT if a device-side wait of that call gave up (its outputs are then
+ * undefined) and SSD_OK otherwise, also when no allocation-free call has run on the device.
+ * It reads the status words the kernel keeps at the start of the built-in scratch; a later
+ * allocation-free call on the device replaces them.  Allocates nothing.
+ */
+SSD_API ssd_status ssd_i8_chunk_scan_noalloc_status(void *stream);
 
 /*
  * Single-token decode state update, in place (the "SSD update" of the Quamba2 rebuttal's

@@ -19,8 +19,9 @@
 
 namespace {
 
-// Built-in scratch: 4 MiB, the workspace of problems with up to 127 (batch x head x chunk) work
-// items (the chunk scan hands states between CTAs through one 32 KiB slot per CTA).
+// Built-in scratch: 4 MiB, the workspace of problems with up to 127 work items of 128 tokens,
+// batch * nheads * ceil(seqlen / 128) <= 127 whatever the chunk size (the chunk scan hands
+// states between CTAs through one 32 KiB slot per CTA, one CTA per work item at most).
 constexpr size_t kScratchBytes = size_t(4) << 20;
 constexpr int kMaxDevices = 64;
 
@@ -30,12 +31,14 @@ std::mutex g_mutex;
 void* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of g_scratch on the current device; looked up on the first call per device.
-ssd_status scratch_on_current_device(void** out) {
+// With `lookup` false, a device whose address was never looked up (no call ran there) gives
+// *out = nullptr.
+ssd_status scratch_on_current_device(void** out, bool lookup = true) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return SSD_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return SSD_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_mutex);
-    if (g_scratch_ptr[dev] == nullptr) {
+    if (g_scratch_ptr[dev] == nullptr && lookup) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || p == nullptr) return SSD_ERR_CUDA;
         g_scratch_ptr[dev] = p;
@@ -66,4 +69,18 @@ extern "C" ssd_status ssd_i8_chunk_scan_noalloc(
     return ssd_i8_chunk_scan(x, B, C, dt, A, D, x_scale, B_scale, C_scale, batch, seqlen, nheads,
                              headdim, dstate, ngroups, chunk_size, init_state, final_state, y,
                              y_dtype, y_scale, scratch, kScratchBytes, stream);
+}
+
+// The kernel writes its failure words at the start of whatever scratch it ran on, so the
+// workspace status query reads them from the built-in array as well.
+extern "C" ssd_status ssd_i8_chunk_scan_noalloc_status(void* stream) {
+    void* scratch = nullptr;
+    const ssd_status s = scratch_on_current_device(&scratch, false);
+    if (s != SSD_OK) return s;
+    if (scratch == nullptr) {  // no allocation-free call has run on this device
+        if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+            return SSD_ERR_CUDA;
+        return SSD_OK;
+    }
+    return ssd_i8_chunk_scan_status(scratch, stream);
 }

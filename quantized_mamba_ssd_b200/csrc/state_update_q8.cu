@@ -5,9 +5,11 @@
 // h_t with the symmetric per-(batch, head) rule scale = max|h_t| / 127,
 // code = clamp(round_half_even(h_t / scale), -127, 127).
 //
-// One CTA per (batch, head); every thread keeps its 16-byte chunks of the state in registers
-// between the update and the requantisation (the scale needs the maximum over the whole state
-// first).  The state moves once in each direction at one byte per element.
+// Persistent CTAs walk the (batch, head) items.  Each thread stages its 16-byte chunks of the
+// next item's codes (and a B or C chunk) with cp.async while the current item is computed, then
+// runs two passes over the staged codes: the update with y and max|h_t|, and, once the CTA has
+// the maximum, the same update again with the requantisation.  The state moves once in each
+// direction at one byte per element.
 #include <type_traits>
 
 #include "common.cuh"

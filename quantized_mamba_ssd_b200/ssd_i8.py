@@ -29,7 +29,7 @@ EXPORTED = ("ssd_i8_abi_version", "ssd_status_string", "ssd_i8_chunk_scan_worksp
             "ssd_i8_chunk_scan", "ssd_i8_state_update", "ssd_i8_chunk_cb",
             "ssd_i8_chunk_scan_noalloc", "ssd_i8_chunk_scan_status", "ssd_i8_debug_inject",
             "ssd_i8_chunk_scan_varlen_workspace_size", "ssd_i8_chunk_scan_varlen",
-            "ssd_i8_state_quantize", "ssd_i8_state_update_q8")
+            "ssd_i8_state_quantize", "ssd_i8_state_update_q8", "ssd_i8_chunk_scan_noalloc_status")
 
 # built-in scratch of ssd_i8_chunk_scan_noalloc (bytes); larger problems are refused
 NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -92,6 +92,8 @@ def library() -> ctypes.CDLL:
         lib.ssd_i8_state_update_q8.argtypes = [vp] * 11 + [ci] * 5 + [vp, ci, cf, vp]
         lib.ssd_i8_chunk_scan_noalloc.restype = ci
         lib.ssd_i8_chunk_scan_noalloc.argtypes = [vp] * 9 + [ci] * 7 + [vp, vp, vp, ci, cf, vp]
+        lib.ssd_i8_chunk_scan_noalloc_status.restype = ci
+        lib.ssd_i8_chunk_scan_noalloc_status.argtypes = [vp]
         _lib = lib
         return lib
 
@@ -459,3 +461,11 @@ def ssd_i8_chunk_scan_noalloc(x: torch.Tensor, B: torch.Tensor, C: torch.Tensor,
     ]
     _check("ssd_i8_chunk_scan_noalloc", library().ssd_i8_chunk_scan_noalloc(*args))
     return y
+
+
+def ssd_i8_chunk_scan_noalloc_status(stream=None) -> None:
+    """Raise SSDError (SSD_ERR_TIMEOUT) if the last allocation-free chunk scan on the current
+    device reported a device-side wait that gave up; synchronises the stream.  See
+    ``ssd_i8_chunk_scan_noalloc_status`` in include/ssd_i8.h."""
+    _check("ssd_i8_chunk_scan_noalloc_status",
+           library().ssd_i8_chunk_scan_noalloc_status(_stream(stream)))

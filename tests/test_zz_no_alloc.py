@@ -78,3 +78,45 @@ def test_noalloc_refuses_problems_beyond_its_scratch():
     assert ei.value.status == 3  # SSD_ERR_WORKSPACE
     torch.cuda.synchronize()
     assert not y.any()  # refused before anything ran
+
+
+def test_noalloc_limit_falls_at_127_blocks_of_128_tokens():
+    # the built-in scratch holds the hand-off slots of 127 work items of 128 tokens, whatever
+    # the chunk size: one sequence of 127 blocks (every CTA but the first waits for a hand-off)
+    # runs and matches the workspace path; one more block is refused
+    case = W.make_prefill(1, 127 * 128, 1, 64, 128, 1, 256, law="laplace_outliers_all", seed=44,
+                          with_init_state=True)
+    assert ssd_i8.ssd_i8_chunk_scan_workspace_size(1, 127 * 128, 1, 64, 128, 1, 64) <= \
+        ssd_i8.NOALLOC_SCRATCH_BYTES
+    y, fs, y_ref, fs_ref = _both(case, "f32")
+    check_close(y, y_ref, "noalloc y, 127 blocks")
+    check_close(fs, fs_ref, "noalloc final_state, 127 blocks")
+    big = W.make_prefill(1, 127 * 128 + 1, 1, 64, 128, 1, 256, seed=45)
+    assert ssd_i8.ssd_i8_chunk_scan_workspace_size(1, 127 * 128 + 1, 1, 64, 128, 1, 256) > \
+        ssd_i8.NOALLOC_SCRATCH_BYTES
+    ins, _ = _inputs(big)
+    y = torch.zeros((1, 127 * 128 + 1, 1, 64), dtype=torch.float32, device=DEV)
+    with pytest.raises(ssd_i8.SSDError) as ei:
+        ssd_i8.ssd_i8_chunk_scan_noalloc(*ins, 256, y=y, y_dtype="f32")
+    assert ei.value.status == 3  # SSD_ERR_WORKSPACE
+    torch.cuda.synchronize()
+    assert not y.any()
+
+
+def test_noalloc_status_reports_a_device_side_timeout():
+    # a caller without a workspace still learns of a bounded wait that gave up: the hook makes
+    # CTA 0 skip its hand-off for one launch (waits bounded by 2^24 cycles), the allocation-free
+    # status query reports the timeout, and the next clean call is correct and reports none
+    case = W.make_prefill(1, 100 * 128, 1, 64, 128, 1, 128, law="laplace_outliers_all", seed=46)
+    ins, _ = _inputs(case)
+    ssd_i8.ssd_i8_chunk_scan_noalloc_status()  # nothing failed so far
+    y = torch.empty((1, case.seqlen, 1, 64), dtype=torch.float32, device=DEV)
+    ssd_i8.ssd_i8_debug_inject(0, 1 << 24)
+    ssd_i8.ssd_i8_chunk_scan_noalloc(*ins, 128, y=y, y_dtype="f32")
+    with pytest.raises(ssd_i8.SSDError) as ei:
+        ssd_i8.ssd_i8_chunk_scan_noalloc_status()
+    assert ei.value.status == 5  # SSD_ERR_TIMEOUT
+    y, fs, y_ref, fs_ref = _both(case, "f32")
+    ssd_i8.ssd_i8_chunk_scan_noalloc_status()
+    check_close(y, y_ref, "noalloc y after a reported timeout")
+    check_close(fs, fs_ref, "noalloc final_state after a reported timeout")
