@@ -122,6 +122,29 @@ def load_peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+def device_status_field(statuses: dict) -> str:
+    """The line's ``device_status``: "ok" when every timed chunk-scan leg reported SSD_OK
+    after its loop.  A leg whose bounded device-side wait gave up ended early, so its time
+    means nothing: the run stops with a non-zero exit instead of printing a number.
+    ``statuses`` maps a leg name to None (OK) or the failing status code."""
+    bad = {k: v for k, v in statuses.items() if v is not None}
+    if bad:
+        print(json.dumps({"error": "device-side wait gave up in the timed region",
+                          "legs": bad}), file=sys.stderr, flush=True)
+        raise SystemExit(3)
+    return "ok"
+
+
+def scan_status(ssd_i8, workspace):
+    """None if the last chunk scan on ``workspace`` reported no device-side failure, else its
+    status code (the call synchronises the stream)."""
+    try:
+        ssd_i8.ssd_i8_chunk_scan_status(workspace)
+    except ssd_i8.SSDError as e:
+        return e.status
+    return None
+
+
 # ------------------------------------------------------------------------------------------
 # clocks during the timed region (NVML reads only; nothing is changed)
 # ------------------------------------------------------------------------------------------
@@ -247,6 +270,70 @@ def reference_arm(args, case: W.PrefillCase):
 # ------------------------------------------------------------------------------------------
 # our arm
 # ------------------------------------------------------------------------------------------
+def prefill_leg(args, index, rank, world, dev, ssd_i8, barrier, hbm_peak, int8_peak_tops, cpu):
+    """Time ssd_i8_chunk_scan on prefill workload ``index`` in its own output dtype, with the
+    final states written: (report dict, device status of the leg)."""
+    import torch
+    case = W.make_prefill_config(index, seed=rank_seed(1000 + index, rank))
+    x, B, C = (torch.from_numpy(a).to(dev) for a in (case.x, case.B, case.C))
+    dt = torch.from_numpy(case.dt).to(dev)
+    A, Dp, sx, sb, sc = (torch.from_numpy(a).to(dev) for a in
+                         (case.A, case.D, case.x_scale, case.B_scale, case.C_scale))
+    bsz, L, H, P, N, G, Q = (case.batch, case.seqlen, case.nheads, case.headdim, case.dstate,
+                             case.ngroups, case.chunk_size)
+    out = case.out_dtype
+    ob = {"f32": 4, "f16": 2, "i8": 1}[out]
+    y = torch.empty((bsz, L, H, P), dtype=ssd_i8.OUT_DTYPES[out][1], device=dev)
+    fs = torch.empty((bsz, H, P, N), dtype=torch.float32, device=dev)
+    ws = torch.empty(ssd_i8.ssd_i8_chunk_scan_workspace_size(bsz, L, H, P, N, G, Q),
+                     dtype=torch.uint8, device=dev)
+
+    def step():
+        ssd_i8.ssd_i8_chunk_scan(x, B, C, dt, A, Dp, sx, sb, sc, Q, final_state=fs, y=y,
+                                 y_dtype=out, y_scale=0.05, workspace=ws)
+
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clocks:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    status = scan_status(ssd_i8, ws)
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dev)
+    alg_bytes = prefill_alg_bytes(case, ob, True)
+    alg_ops = prefill_alg_ops(case)
+    t_hbm = alg_bytes / (hbm_peak * 1e9)
+    t_ops = alg_ops / (int8_peak_tops * 1e12)
+    gbs = alg_bytes / (ms * 1e-3) / 1e9
+    leg = {
+        "metric": f"SSD scan tokens/s (int8 in), {out} out", "workload": case.name,
+        "value": aggregate_tokens_per_s(bsz * L, world, ms), "unit": UNIT, "ms_per_step": ms,
+        "gpu_launches": args.steps * ssd_i8.KERNELS_PER_CHUNK_SCAN,
+        "roofline": {"bound": "hbm" if t_hbm >= t_ops else "tensor", "achieved": gbs,
+                     "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak, "traffic": None,
+                     "alg_bytes_per_launch": alg_bytes,
+                     "alg_bytes_without_final_state": prefill_alg_bytes(case, ob, False),
+                     "alg_int8_ops_per_launch": alg_ops,
+                     "roofline_us": 1e6 * max(t_hbm, t_ops)},
+        "clocks": clocks.summary(),
+        "cpu_baseline": None,
+    }
+    del x, B, C, dt, y, fs, ws
+    if cpu:
+        v, nt, sample = oracle_tokens_per_s(case, target_s=8.0)
+        leg["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": nt, "kind": "oracle",
+                               "sample": sample}
+    return leg, status
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -261,6 +348,8 @@ def main():
                     help="skip the per-tensor percentile-clipped workload leg")
     ap.add_argument("--no-varlen", action="store_true",
                     help="skip the packed variable-length (strided) serving prefill leg")
+    ap.add_argument("--no-smaller", action="store_true",
+                    help="skip the 1.3B- and 2.7B-shaped prefill legs")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="decode batch per rank (default: the workload's 128); smaller batches "
                          "of the same shape serve profiling captures")
@@ -343,6 +432,7 @@ def main():
         ev1.record(stream)
         torch.cuda.synchronize()
     barrier()
+    statuses = {"main": scan_status(ssd_i8, ws)}
     ms = ev0.elapsed_time(ev1) / args.steps
     ms_max = max_over_ranks(ms, dev)
     tokens_all = bsz * L * world
@@ -363,6 +453,7 @@ def main():
     ev1.record(stream)
     torch.cuda.synchronize()
     barrier()
+    statuses["hadamard_out"] = scan_status(ssd_i8, ws)
     had_ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dev)
 
     # ---- end to end: pinned host inputs in, int8 output back, every step ----
@@ -393,6 +484,7 @@ def main():
         ev1.record(stream)
         torch.cuda.synchronize()
         barrier()
+        statuses["e2e_serial"] = scan_status(ssd_i8, ws)
         serial_ms = max_over_ranks(ev0.elapsed_time(ev1) / e2e_steps, dev)
         # pipelined: step i's inputs go up on one copy stream while step i - 1 computes and step
         # i - 2's output comes down on another (two device buffer sets, two host output buffers)
@@ -433,6 +525,7 @@ def main():
         ev1.record(stream)
         torch.cuda.synchronize()
         barrier()
+        statuses["e2e_pipelined"] = scan_status(ssd_i8, ws)
         e2e_ms = max_over_ranks(ev0.elapsed_time(ev1) / e2e_steps, dev)
         e2e = {"value": aggregate_tokens_per_s(bsz * L, world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -466,6 +559,7 @@ def main():
         ev1.record(stream)
         torch.cuda.synchronize()
         barrier()
+        statuses["per_tensor_percentile"] = scan_status(ssd_i8, ws)
         pt_ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dev)
         pt_gbs = prefill_alg_bytes(pcase, 1, True) / (pt_ms * 1e-3) / 1e9
         per_tensor = {
@@ -519,6 +613,7 @@ def main():
         ev1.record(stream)
         torch.cuda.synchronize()
         barrier()
+        statuses["varlen_strided"] = scan_status(ssd_i8, vws)
         vl_ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dev)
         vl_bytes = (T * (H * P + 2 * G * N + 4 * H + H * P)  # x, B, C, dt in; y out (int8)
                     + 4 * nseq * H * P * N)  # final states
@@ -538,6 +633,14 @@ def main():
                          "alg_bytes_per_launch": vl_bytes},
         }
         del proj, vx, vB, vC, vdt, vy, vfs, vws, vcase
+
+    # ---- the 1.3B- and 2.7B-shaped prefills (f16 out, final states written) ----
+    smaller = {}
+    if not args.no_smaller:
+        for idx, key in ((1, "prefill_1p3b"), (2, "prefill_2p7b")):
+            smaller[key], statuses[key] = prefill_leg(
+                args, idx, rank, world, dev, ssd_i8, barrier, hbm_peak, int8_peak_tops,
+                cpu=(rank == 0 and world == 1 and not args.no_cpu_baseline))
 
     # ---- roofline of the timed call ----
     alg_bytes = prefill_alg_bytes(case, 1, True)
@@ -661,6 +764,8 @@ def main():
         v, nt, sample = oracle_tokens_per_s(case)
         cpu = {"value": v, "unit": UNIT, "cores": nt, "kind": "oracle", "sample": sample}
 
+    if rank != 0:
+        device_status_field(statuses)
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -678,7 +783,10 @@ def main():
             "clocks": clocks.summary(),
             "hadamard_out": hadamard_out, "per_tensor_percentile": per_tensor,
             "varlen_strided": varlen,
+            "prefill_1p3b": smaller.get("prefill_1p3b"),
+            "prefill_2p7b": smaller.get("prefill_2p7b"),
             "decode": decode,
+            "device_status": device_status_field(statuses),
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -157,11 +157,13 @@ SSD_API ssd_status ssd_i8_chunk_scan_varlen(const int8_t *x, long long x_token_s
                                             size_t workspace_bytes, void *stream);
 
 /*
- * Status of the last ssd_i8_chunk_scan call that ran on `workspace`: synchronises `stream`,
- * then returns SSD_ERR_TIMEOUT if a device-side wait of that call gave up (a CTA waiting for its
- * predecessor's state hand-off, or for a tensor-core / TMA completion) and SSD_OK otherwise.
+ * Status of the chunk-scan calls (ssd_i8_chunk_scan or _varlen) that ran on `workspace` since
+ * the previous status query on it (or, with none, since the first call): synchronises `stream`,
+ * then returns SSD_ERR_TIMEOUT if a device-side wait of any of them gave up (a CTA waiting for
+ * its predecessor's state hand-off, or for a tensor-core / TMA completion) and SSD_OK otherwise.
  * Every wait inside the kernels is bounded (about one second), so a failed call still
- * terminates; its outputs are then undefined.
+ * terminates; its outputs are then undefined.  Calls on one workspace are assumed to come from
+ * one host thread at a time (they may not overlap anyway).
  */
 SSD_API ssd_status ssd_i8_chunk_scan_status(const void *workspace, void *stream);
 
@@ -208,12 +210,12 @@ SSD_API ssd_status ssd_i8_chunk_scan_noalloc(const int8_t *x, const int8_t *B, c
                                              float y_scale, void *stream);
 
 /*
- * Status of the last ssd_i8_chunk_scan_noalloc call on the current device -- the counterpart of
- * ssd_i8_chunk_scan_status for callers that have no workspace to pass: synchronises `stream`,
- * then returns SSD_ERR_TIMEOUT if a device-side wait of that call gave up (its outputs are then
- * undefined) and SSD_OK otherwise, also when no allocation-free call has run on the device.
- * It reads the status words the kernel keeps at the start of the built-in scratch; a later
- * allocation-free call on the device replaces them.  Allocates nothing.
+ * Status of the ssd_i8_chunk_scan_noalloc calls on the current device since the previous query
+ * -- the counterpart of ssd_i8_chunk_scan_status for callers that have no workspace to pass:
+ * synchronises `stream`, then returns SSD_ERR_TIMEOUT if a device-side wait of one of them gave
+ * up (its outputs are then undefined) and SSD_OK otherwise, also when no allocation-free call
+ * has run on the device.  It reads the status words the kernel keeps at the start of the
+ * built-in scratch.  Allocates nothing.
  */
 SSD_API ssd_status ssd_i8_chunk_scan_noalloc_status(void *stream);
 

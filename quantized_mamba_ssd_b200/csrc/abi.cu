@@ -282,9 +282,13 @@ ssd_status ssd_i8_chunk_scan_status(const void* workspace, void* stream) {
     unsigned long long w[3] = {0, 0, 0};
     if (cudaMemcpy(w, workspace, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess)
         return SSD_ERR_CUDA;
-    // w[0]: epoch of the call that recorded a failure, w[1]: failure code, w[2]: epoch of the
-    // last call that ran on this workspace
-    if (w[1] != 0 && w[0] == w[2]) return SSD_ERR_TIMEOUT;
+    // w[0]: epoch of the last call that recorded a failure, w[1]: failure code, w[2]: epoch of
+    // the last call that ran on this workspace.  Epochs grow by one per launch in a process, so
+    // the calls since the previous query are those from `first` to w[2].
+    unsigned long long first = 0;
+    const bool since = ssd::take_first_epoch(workspace, &first);
+    if (w[1] != 0 && (since ? (w[0] >= first && w[0] <= w[2]) : w[0] == w[2]))
+        return SSD_ERR_TIMEOUT;
     return SSD_OK;
 }
 

@@ -43,6 +43,7 @@
 #include <atomic>
 #include <mutex>
 #include <random>
+#include <unordered_map>
 
 #include "common.cuh"
 #include "sm100.cuh"
@@ -1311,6 +1312,11 @@ bool g_inject_armed = false;
 int g_inject_cta = -1;
 long long g_inject_wait = kWaitCycles;
 
+// epoch of the first launch on each workspace since its last status query (status queries
+// report a failure of any launch from there on)
+std::mutex g_epoch_mutex;
+std::unordered_map<const void*, unsigned long long> g_first_epoch;
+
 long long total_blocks(int batch, int seqlen, int nheads) {
     return (long long)batch * nheads * ceil_div(seqlen, kBlk);
 }
@@ -1382,6 +1388,10 @@ cudaError_t launch_chunk_scan(const ChunkScanArgs& a, cudaStream_t st) {
     p.flags = reinterpret_cast<unsigned long long*>(ws + 256);
     p.slots = reinterpret_cast<float*>(ws + 256 + kMaxCtas * 8);
     p.epoch = ++epoch_counter();
+    {
+        std::lock_guard<std::mutex> lock(g_epoch_mutex);
+        g_first_epoch.emplace(a.workspace, p.epoch);  // kept if an earlier launch is unqueried
+    }
     p.wait_limit = kWaitCycles;
     p.drop_publish = -1;
     {
@@ -1401,6 +1411,15 @@ cudaError_t launch_chunk_scan(const ChunkScanArgs& a, cudaStream_t st) {
         case SSD_OUT_I8 | SSD_OUT_HADAMARD: return launch_fused<SSD_OUT_I8, true>(mx, mB, mC, p, st);
         default: return cudaErrorInvalidValue;
     }
+}
+
+bool take_first_epoch(const void* workspace, unsigned long long* epoch) {
+    std::lock_guard<std::mutex> lock(g_epoch_mutex);
+    const auto it = g_first_epoch.find(workspace);
+    if (it == g_first_epoch.end()) return false;
+    *epoch = it->second;
+    g_first_epoch.erase(it);
+    return true;
 }
 
 void arm_fault_injection(int drop_publish_cta, long long wait_cycles) {

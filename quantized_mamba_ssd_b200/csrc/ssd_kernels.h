@@ -85,5 +85,8 @@ cudaError_t launch_state_update_q8(const StateUpdateQ8Args& a, cudaStream_t stre
 cudaError_t launch_state_quantize(const float* state, int8_t* q, float* scale, int count,
                                   int headdim, int dstate, cudaStream_t stream);
 void arm_fault_injection(int drop_publish_cta, long long wait_cycles);
+// Epoch of the first chunk-scan launch on `workspace` since the last call of this function for
+// it (false: none launched since); the entry is removed.
+bool take_first_epoch(const void* workspace, unsigned long long* epoch);
 
 }  // namespace ssd

@@ -47,3 +47,33 @@ def test_captured_traffic_scales_with_the_work():
         v = bench.captured_decode_traffic(src, 128 * 128)
         if v is not None:
             assert abs(bench.captured_decode_traffic(src, 64 * 128) * 2 - v) < 1e-6 * v
+
+
+def test_algorithmic_bytes_of_the_smaller_prefills():
+    # x + B + C + dt + f16 y (SURVEY's roofline table: 104.9 MB and 522.2 MB), and with the
+    # final states the legs write
+    c1 = W.PrefillCase("shape-only", 4, 2048, 64, 64, 128, 1, 256, *([None] * 9))
+    c2 = W.PrefillCase("shape-only", 8, 4096, 80, 64, 128, 1, 256, *([None] * 9))
+    assert bench.prefill_alg_bytes(c1, 2, False) == 104857600
+    assert bench.prefill_alg_bytes(c2, 2, False) == 522190848
+    assert bench.prefill_alg_bytes(c1, 2, True) == 104857600 + 4 * 4 * 64 * 64 * 128
+    assert bench.prefill_alg_bytes(c2, 2, True) == 522190848 + 4 * 8 * 80 * 64 * 128
+
+
+def test_device_status_field_reports_ok_and_stops_on_a_timeout():
+    # every timed chunk-scan leg reports its device status; a leg whose bounded wait gave up
+    # ended early, so the run exits non-zero instead of printing its time
+    assert bench.device_status_field({"main": None, "varlen_strided": None}) == "ok"
+    import pytest
+    with pytest.raises(SystemExit) as ei:
+        bench.device_status_field({"main": None, "hadamard_out": 5})
+    assert ei.value.code != 0
+
+
+def test_bench_line_carries_the_device_status():
+    # the field is part of the printed line, computed from the statuses of every timed leg
+    src = open(bench.__file__).read()
+    assert '"device_status": device_status_field(statuses)' in src
+    for leg in ("main", "hadamard_out", "e2e_serial", "e2e_pipelined", "per_tensor_percentile",
+                "varlen_strided"):
+        assert f'statuses["{leg}"]' in src or f'"{leg}": scan_status' in src
