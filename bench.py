@@ -270,11 +270,13 @@ def reference_arm(args, case: W.PrefillCase):
 # ------------------------------------------------------------------------------------------
 # our arm
 # ------------------------------------------------------------------------------------------
-def prefill_leg(args, index, rank, world, dev, ssd_i8, barrier, hbm_peak, int8_peak_tops, cpu):
-    """Time ssd_i8_chunk_scan on prefill workload ``index`` in its own output dtype, with the
-    final states written: (report dict, device status of the leg)."""
+def prefill_leg(args, index, rank, world, dev, ssd_i8, barrier, hbm_peak, int8_peak_tops, cpu,
+                **overrides):
+    """Time ssd_i8_chunk_scan on prefill workload ``index`` (with ``overrides`` of its recipe,
+    e.g. per-channel B/C scales) in its own output dtype, with the final states written:
+    (report dict, device status of the leg)."""
     import torch
-    case = W.make_prefill_config(index, seed=rank_seed(1000 + index, rank))
+    case = W.make_prefill_config(index, seed=rank_seed(1000 + index, rank), **overrides)
     x, B, C = (torch.from_numpy(a).to(dev) for a in (case.x, case.B, case.C))
     dt = torch.from_numpy(case.dt).to(dev)
     A, Dp, sx, sb, sc = (torch.from_numpy(a).to(dev) for a in
@@ -313,8 +315,10 @@ def prefill_leg(args, index, rank, world, dev, ssd_i8, barrier, hbm_peak, int8_p
     t_hbm = alg_bytes / (hbm_peak * 1e9)
     t_ops = alg_ops / (int8_peak_tops * 1e12)
     gbs = alg_bytes / (ms * 1e-3) / 1e9
+    per_n = case.B_scale.ndim == 2
     leg = {
-        "metric": f"SSD scan tokens/s (int8 in), {out} out", "workload": case.name,
+        "metric": f"SSD scan tokens/s (int8 in), {out} out"
+                  + (", B/C scales per dstate channel" if per_n else ""), "workload": case.name,
         "value": aggregate_tokens_per_s(bsz * L, world, ms), "unit": UNIT, "ms_per_step": ms,
         "gpu_launches": args.steps * ssd_i8.KERNELS_PER_CHUNK_SCAN,
         "roofline": {"bound": "hbm" if t_hbm >= t_ops else "tensor", "achieved": gbs,
@@ -350,6 +354,8 @@ def main():
                     help="skip the packed variable-length (strided) serving prefill leg")
     ap.add_argument("--no-smaller", action="store_true",
                     help="skip the 1.3B- and 2.7B-shaped prefill legs")
+    ap.add_argument("--no-per-channel", action="store_true",
+                    help="skip the per-dstate-channel B/C scale leg")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="decode batch per rank (default: the workload's 128); smaller batches "
                          "of the same shape serve profiling captures")
@@ -642,6 +648,13 @@ def main():
                 args, idx, rank, world, dev, ssd_i8, barrier, hbm_peak, int8_peak_tops,
                 cpu=(rank == 0 and world == 1 and not args.no_cpu_baseline))
 
+    # ---- the 8B-shaped long prefill with B and C scales per dstate channel ([g, n]) ----
+    per_channel = None
+    if not args.no_per_channel:
+        per_channel, statuses["per_channel_scales"] = prefill_leg(
+            args, PREFILL_CFG, rank, world, dev, ssd_i8, barrier, hbm_peak, int8_peak_tops,
+            cpu=False, scales="channel", **overrides)
+
     # ---- roofline of the timed call ----
     alg_bytes = prefill_alg_bytes(case, 1, True)
     alg_ops = prefill_alg_ops(case)
@@ -785,6 +798,7 @@ def main():
             "varlen_strided": varlen,
             "prefill_1p3b": smaller.get("prefill_1p3b"),
             "prefill_2p7b": smaller.get("prefill_2p7b"),
+            "per_channel_scales": per_channel,
             "decode": decode,
             "device_status": device_status_field(statuses),
         }

@@ -62,6 +62,18 @@ typedef enum ssd_out_dtype { SSD_OUT_F32 = 0, SSD_OUT_F16 = 1, SSD_OUT_I8 = 2 } 
  */
 #define SSD_OUT_HADAMARD 16
 
+/*
+ * Flag OR-ed into the y_dtype of ssd_i8_chunk_scan / _varlen / _noalloc and of the decode steps
+ * ssd_i8_state_update / _q8: B_scale and C_scale are per group AND dstate channel, float
+ * [ngroups, dstate] (row-major), instead of per group -- the per-P(N) quantization axis of the
+ * SSDi8 page, Table 10: B_t[n] = s_B[g, n] Bq[t, g, n] and C_t[n] = s_C[g, n] Cq[t, g, n].  In
+ * the chunk scan the products s_C[g, n] s_B[g, n] then sit inside ChunkBMM, which runs on f16
+ * tensor cores (Cq exact, Bq s_C s_B / max_n(s_C s_B) rounded to f16) instead of exact int8;
+ * the chunk state and C H take the channel scales exactly.  The states (init_state,
+ * final_state, the cached decode state) are the true states, as without the flag.
+ */
+#define SSD_SCALES_PER_N 32
+
 /* Version of this ABI; bumped when a signature or a layout changes. */
 SSD_API int ssd_i8_abi_version(void);
 
@@ -86,11 +98,13 @@ SSD_API size_t ssd_i8_chunk_scan_workspace_size(int batch, int seqlen, int nhead
  *   B, C       int8  [batch, seqlen, ngroups, dstate]
  *   dt         float [batch, seqlen, nheads]   (already discretised / softplus'ed, >= 0)
  *   A, D       float [nheads]                   (A <= 0)
- *   x_scale    float [nheads];  B_scale, C_scale float [ngroups]   (static scales)
+ *   x_scale    float [nheads];  B_scale, C_scale float [ngroups]   (static scales; float
+ *              [ngroups, dstate] with SSD_SCALES_PER_N in y_dtype)
  *   chunk_size Q: 64, 128 or 256.  The result does not depend on Q beyond rounding.
  *   init_state float [batch, nheads, headdim, dstate] or NULL (zero initial state)
  *   final_state float [batch, nheads, headdim, dstate] or NULL (not written)
- *   y          [batch, seqlen, nheads, headdim] of y_dtype
+ *   y          [batch, seqlen, nheads, headdim] of y_dtype (an SSD_OUT_* code, optionally
+ *              OR-ed with SSD_OUT_HADAMARD and SSD_SCALES_PER_N)
  *   workspace  device memory of at least ssd_i8_chunk_scan_workspace_size(...) bytes,
  *              256-byte aligned.
  * Supported: headdim == 64; dstate in {16, 32, 64, 128}; batch * nheads < 2^31 (larger:
@@ -227,7 +241,8 @@ SSD_API ssd_status ssd_i8_chunk_scan_noalloc_status(void *stream);
  *   x          int8  [batch, nheads, headdim]
  *   B, C       int8  [batch, ngroups, dstate]
  *   dt         float [batch, nheads]
- *   A, D, x_scale float [nheads]; B_scale, C_scale float [ngroups]
+ *   A, D, x_scale float [nheads]; B_scale, C_scale float [ngroups] ([ngroups, dstate] with
+ *              SSD_SCALES_PER_N in y_dtype)
  *   y          [batch, nheads, headdim] of y_dtype
  * Supported: dstate in {16, 32, 64, 128, 256}; 1 <= headdim <= 256; nheads % ngroups == 0.
  */

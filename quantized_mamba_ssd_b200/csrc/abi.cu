@@ -14,8 +14,8 @@ constexpr size_t kWorkspaceAlign = 256;
 
 bool valid_out_dtype(int d) { return d == SSD_OUT_F32 || d == SSD_OUT_F16 || d == SSD_OUT_I8; }
 
-// chunk-scan outputs may also carry the Hadamard flag
-bool valid_scan_out(int d) { return valid_out_dtype(d & ~SSD_OUT_HADAMARD); }
+// chunk-scan and decode outputs may also carry the Hadamard and per-channel-scale flags
+bool valid_scan_out(int d) { return valid_out_dtype(d & ~(SSD_OUT_HADAMARD | SSD_SCALES_PER_N)); }
 
 bool chunk_dstate_ok(int n) { return n == 16 || n == 32 || n == 64 || n == 128; }
 
@@ -27,7 +27,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // kernels multiply by its fp32 reciprocal.
 bool out_scale(int y_dtype, float y_scale, float* inv) {
     *inv = 1.f;
-    if ((y_dtype & ~SSD_OUT_HADAMARD) != SSD_OUT_I8) return true;
+    if ((y_dtype & ~(SSD_OUT_HADAMARD | SSD_SCALES_PER_N)) != SSD_OUT_I8) return true;
     if (!(y_scale > 0.f) || !std::isfinite(y_scale)) return false;
     *inv = 1.f / y_scale;
     return std::isfinite(*inv);
@@ -208,8 +208,10 @@ ssd_status ssd_i8_state_update(float* state, const int8_t* x, const int8_t* B, c
     if (!state || !x || !B || !C || !dt || !A || !D || !x_scale || !B_scale || !C_scale || !y)
         return SSD_ERR_INVALID_ARG;
     ssd::StateUpdateArgs a{state, x, B, C, dt, A, D, x_scale, B_scale, C_scale, batch, nheads,
-                           headdim, dstate, ngroups, y, y_dtype & ~SSD_OUT_HADAMARD, inv,
-                           (y_dtype & SSD_OUT_HADAMARD) ? 1 : 0};
+                           headdim, dstate, ngroups, y,
+                           y_dtype & ~(SSD_OUT_HADAMARD | SSD_SCALES_PER_N), inv,
+                           (y_dtype & SSD_OUT_HADAMARD) ? 1 : 0,
+                           (y_dtype & SSD_SCALES_PER_N) ? 1 : 0};
     return ssd::launch_state_update(a, static_cast<cudaStream_t>(stream)) == cudaSuccess
                ? SSD_OK
                : SSD_ERR_CUDA;
@@ -249,7 +251,9 @@ ssd_status ssd_i8_state_update_q8(int8_t* state_q, float* state_scale, const int
     if (!aligned16(state_q) || !aligned16(B) || !aligned16(C)) return SSD_ERR_INVALID_ARG;
     ssd::StateUpdateQ8Args a{state_q, state_scale, x, B, C, dt, A, D, x_scale, B_scale,
                              C_scale, batch, nheads, headdim, dstate, ngroups, y,
-                             y_dtype & ~SSD_OUT_HADAMARD, inv, (y_dtype & SSD_OUT_HADAMARD) ? 1 : 0};
+                             y_dtype & ~(SSD_OUT_HADAMARD | SSD_SCALES_PER_N), inv,
+                             (y_dtype & SSD_OUT_HADAMARD) ? 1 : 0,
+                             (y_dtype & SSD_SCALES_PER_N) ? 1 : 0};
     return ssd::launch_state_update_q8(a, static_cast<cudaStream_t>(stream)) == cudaSuccess
                ? SSD_OK
                : SSD_ERR_CUDA;

@@ -17,9 +17,10 @@
 // any chunk length, so the result depends on the caller's chunk size only through rounding.
 // Per block and head, with a_t = log2(e) * sum_{k<=t} dt_k A_h inside the block:
 //   CB    = Cq Bq^T                                   tcgen05 kind::i8, exact int32 in TMEM
-//   M'    = CB * 2^(a_t - a_s) * dt_s / kappa  (s <= t), f16, written over CB in TMEM; off the
-//           32 x 32 diagonal sub-blocks as a product of a row and a column factor (both <= 1)
-//   acc   = C' H'^T + x (D s_x / rho) + M' x          tcgen05 kind::f16
+//   M'    = CB * 2^(a_t - a_s) * dt_s / kappa  (s <= t), plus D s_x / rho on the diagonal (the
+//           skip term D x), f16, written over CB in TMEM; off the 32 x 32 diagonal sub-blocks as
+//           a product of a row and a column factor (both <= 1)
+//   acc   = M' x + C' H'^T                             tcgen05 kind::f16
 //           C'[t,n] = Cq[t,n] 2^a_t,  H' = (H / s_x s_B) / kappa
 //   y     = rho * acc,  rho = s_C s_x s_B kappa (a power of two)
 //   H    <- 2^a_end H + B'^T x,  B'[t,n] = Bq[t,n] dt_t 2^(a_end - a_t) / U
@@ -28,15 +29,23 @@
 // needed.  Only the non-int8 operands (M', C', B', H', D s_x / rho) are rounded, once each,
 // to f16.
 //
+// B and C scales per dstate channel n (SSDi8 page, Table 10, the per-P(N) axis): with
+// u_n = s_C[g,n] s_B[g,n] and u~_n = u_n / max_n u_n, CB = max u * C B~^T with B~ = Bq u~_n is
+// no longer an integer product; it runs on kind::f16 (Cq and Bq u~_n in f16, the C copy in the
+// worker's free accumulator columns, B~ in its B' buffer before B' is written).  The state and
+// C'H'^T take the channel scales as per-lane (TMEM lane = n) factors: H is kept in units of
+// s_x s_B[g,n], and H' carries u~_n.
+//
 // Warp roles, coupled only through mbarriers (buffers alternate with the block parity j):
 //   warp 8      TMA: x, B, C tiles of block k into stage j
 //   warp 9      MMA issue: CB(k+1); M'x(k); state(k); C'H'(k) + x D(k)
 //   warps 0-3   block worker for even blocks, warps 4-7 for odd blocks: both run the same
 //               compact loop (the kernel is limited by instruction fetch, and two warps on an
-//               SM sub-partition that run the same code share it): output of the worker's
-//               previous block, block scan of dt, block statistics chained through the
-//               workers (bound on |H|, state unit), x and B' conversions, M' from CB(k), then
-//               the serial part, the state hand-over (H', decay) and C', D.
+//               SM sub-partition that run the same code share it): block scan of dt, block
+//               statistics chained through the workers (bound on |H|, state unit), output of
+//               the worker's previous block (its accumulator completes meanwhile), x and B'
+//               conversions, M' from CB(k), then the serial part, the state hand-over (H',
+//               decay) and C'.
 // Every wait is bounded; a timeout sets a status word and turns the remaining waits into
 // no-ops so that the kernel still ends (its outputs are then undefined).
 #include <algorithm>
@@ -78,17 +87,16 @@ constexpr int kStC = 0, kStB = 16384, kStX = 32768;
 constexpr int kOffXf = 2 * kStageBytes;         // x f16 [128 t][64 p], 128B swizzle, 2 buffers
 constexpr int kOffBp = kOffXf + 2 * 16384;      // B' f16 2 x [128 t][64 n] MN-major, 2 buffers
 constexpr int kOffHp = kOffBp + 2 * 32768;      // H' f16 [128 n][64 p] MN-major, 2 buffers
-constexpr int kOffDm = kOffHp + 2 * 16384;      // D s_x / rho on the diagonal of [64][64] f16
-constexpr int kOffColf = kOffDm + 8192;         // off-diagonal column factors [2][192] f32
+constexpr int kOffColf = kOffHp + 2 * 16384;    // off-diagonal column factors [2][192] f32
 constexpr int kOffNb = kOffColf + 2 * 768;      // -beta_s = log2(dt_s / kappa) - a_s [2][128]
 constexpr int kOffStats = kOffNb + 2 * 512;     // per-block statistics handed between workers [2][2]
 constexpr int kOffRed = kOffStats + 4 * 16;     // worker scratch [2][16] f32: warp sums, maxima,
                                                 // first-row dt (scan); state bounds (piece start)
-constexpr int kOffBar = kOffRed + 2 * 64;       // mbarriers [32]
+constexpr int kOffUt = kOffRed + 2 * 64;        // per-channel u~_n, f16 [2][128] (per-N scales)
+constexpr int kOffBar = kOffUt + 2 * 256;       // mbarriers [32]
 constexpr int kOffMisc = kOffBar + 32 * 8;      // TMEM base, abort flag
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
-static_assert(kOffXf % 1024 == 0 && kOffBp % 1024 == 0 && kOffHp % 1024 == 0 &&
-                  kOffDm % 1024 == 0, "alignment");
+static_assert(kOffXf % 1024 == 0 && kOffBp % 1024 == 0 && kOffHp % 1024 == 0, "alignment");
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 enum {
@@ -99,12 +107,13 @@ enum {
     kBarXb0, kBarXb1,              // x f16 and B' of block k ready
     kBarMp0, kBarMp1,              // M'(k) in TMEM buffer j
     kBarPh0, kBarPh1,              // H' written and H decayed for block k
-    kBarPc0, kBarPc1,              // C' and D of block k written
+    kBarPc0, kBarPc1,              // C' of block k written
     kBarMx0, kBarMx1,              // M'x(k) done (CB buffer j free)
     kBarAcc0, kBarAcc1,            // accumulator j complete
     kBarAccFree0, kBarAccFree1,    // accumulator j read out
     kBarState,                     // state update of the last issued block done
-    kBarCh,                        // C'H' + xD of the last issued block done (C', D free)
+    kBarCh,                        // C'H' of the last issued block done (C' free)
+    kBarCbIn0, kBarCbIn1,          // per-N scales: C and B~ of block k in place for ChunkBMM
     kNumBars
 };
 static_assert(kNumBars <= 32, "barrier space");
@@ -455,9 +464,10 @@ __device__ __forceinline__ void issue_cb(uint32_t d, uint32_t sC, uint32_t sB, i
 // either as the caller's final state or into this CTA's hand-off slot (then publishes the slot).
 // `out_scale` converts TMEM units to units of s_x s_B.  Inlined: a call from the worker loop
 // would save and restore its live registers at every piece switch.
+// With `per_n`, the B scales are per dstate channel ([g, n]) and row n's own one applies.
 __device__ __forceinline__ void store_piece_state(const FusedParams& p, uint32_t tmem, int row,
                                                bool final_piece, bool cta_end, int seq, int h,
-                                               float out_scale, int bar_id) {
+                                               float out_scale, bool per_n, int bar_id) {
     const uint32_t lane_base = static_cast<uint32_t>(row & ~31);
     uint32_t hv[2][32];
     tmem_ld32_sync(tmem_addr(tmem, lane_base, kColH), hv[0]);
@@ -465,7 +475,9 @@ __device__ __forceinline__ void store_piece_state(const FusedParams& p, uint32_t
     if (final_piece) {
         if (p.final_state != nullptr && row < p.N) {
             float* dst = p.final_state + ((size_t)seq * p.H + h) * kP * p.N;
-            const float s = out_scale * p.x_scale[h] * p.B_scale[h / (p.H / p.G)];
+            const int g = h / (p.H / p.G);
+            const float sB = per_n ? p.B_scale[(size_t)g * p.N + row] : p.B_scale[g];
+            const float s = out_scale * p.x_scale[h] * sB;
 #pragma unroll
             for (int jj = 0; jj < 64; ++jj)
                 dst[(size_t)jj * p.N + row] = s * __uint_as_float(hv[jj / 32][jj % 32]);
@@ -488,7 +500,8 @@ __device__ __forceinline__ void store_piece_state(const FusedParams& p, uint32_t
 }
 
 // Piece start (worker warpgroup, thread = state row n): the piece's initial state in units of
-// s_x s_B -- the caller's initial state (or zero) at sequence start, else the predecessor CTA's
+// s_x s_B (sigma = s_x s_B of row n) -- the caller's initial state (or zero) at sequence start,
+// else the predecessor CTA's
 // hand-off slot.  piece_state_bound returns its max |.| (for the operand scaling of the piece's
 // first block) without touching tensor memory; for a slot it first waits (bounded) for the
 // predecessor's flag.  write_piece_state later puts the state into TMEM, once the previous
@@ -590,7 +603,7 @@ __device__ __forceinline__ void write_piece_state(const FusedParams& p, uint32_t
 // start column of quad q's off-diagonal column factors (q = 1, 2, 3 hold 32 q entries)
 __host__ __device__ constexpr int colf_off(int q) { return 16 * q * (q - 1); }
 
-template <int YT, bool HAD>
+template <int YT, bool HAD, bool PERN>
 __global__ void __launch_bounds__(kThreads, 1)
 fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                         const __grid_constant__ CUtensorMap map_B,
@@ -614,10 +627,6 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
         *abort_flag = 0;
         if (blockIdx.x == 0) p.status[2] = p.epoch;  // the call the status word refers to
     }
-    // the D matrix is zero off its diagonal
-    for (int i = tid; i < 8192 / 16; i += kThreads)
-        reinterpret_cast<uint4*>(smem + kOffDm)[i] = make_uint4(0u, 0u, 0u, 0u);
-    fence_proxy_async_smem();
     if (warp == kWarpMma) {
         tmem_alloc(misc, kTmemCols);
         tmem_relinquish();
@@ -637,6 +646,9 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             tma_prefetch_map(&map_x);
             tma_prefetch_map(&map_B);
             tma_prefetch_map(&map_C);
+            // L2 priorities: B and C tiles are read again by the other heads of their group
+            // (kept), x tiles only once (evicted first)
+            const uint64_t pol_x = l2_policy_evict_first(), pol_bc = l2_policy_evict_last();
             int kb = 0;
             for (int k = 0; k < rg.nseg && !*abort_flag; ++k) {
                 Piece pc;
@@ -650,9 +662,9 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                     uint64_t* bar = bars + kBarFull0 + s;
                     mbar_arrive_expect_tx(bar, kStageBytes);
                     const int t0 = pc.tok0 + c * kBlk;  // packed token of the block's first row
-                    tma_load_3d(stage + kStX, &map_x, 0, h, t0, bar);
-                    tma_load_3d(stage + kStB, &map_B, 0, g, t0, bar);
-                    tma_load_3d(stage + kStC, &map_C, 0, g, t0, bar);
+                    tma_load_3d(stage + kStX, &map_x, 0, h, t0, bar, pol_x);
+                    tma_load_3d(stage + kStB, &map_B, 0, g, t0, bar, pol_bc);
+                    tma_load_3d(stage + kStC, &map_C, 0, g, t0, bar, pol_bc);
                 }
             }
             // drain: both stages' last loads must have landed before the CTA exits
@@ -664,21 +676,31 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
         if (lane == 0 && nb_total > 0) {
             const uint32_t id_st = idesc_f16(kBlk, kP, true, true);   // B'^T (MN) x xf (MN)
             const uint32_t id_y = idesc_f16(kBlk, kP, false, true);   // C' / M' (TMEM) x hp / xf
-            const uint32_t id_d = idesc_f16(kBlk, kP, false, false);  // xf (K-major) x D (K-major)
             const uint32_t sbase = smem_u32(smem);
             const uint64_t d_bp = smem_desc(sbase + kOffBp, 16384, 1024, kSwizzle128B);
             const uint64_t d_xf = smem_desc(sbase + kOffXf, 16, 1024, kSwizzle128B);
             const uint64_t d_hp = smem_desc(sbase + kOffHp, 16, 1024, kSwizzle128B);
-            const uint64_t d_dm = smem_desc(sbase + kOffDm, 16, 1024, kSwizzle128B);
+            const uint32_t id_cb16 = idesc_f16(kBlk, kBlk, false, false);  // C (TMEM) x B~ (K-major)
             auto issue_cb_block = [&](int kb) {
                 const int j = kb & 1;
-                wait_phase(bars + kBarFull0 + j, (kb >> 1) & 1, abort_flag, p);
+                // per-N scales: the worker has put C and B~ in place (after the tiles landed)
+                wait_phase(bars + (PERN ? kBarCbIn0 : kBarFull0) + j, (kb >> 1) & 1, abort_flag, p);
                 // CB buffer j held M'(kb - 2), read by M'x(kb - 2)
                 if (kb >= 2) wait_phase(bars + kBarMx0 + j, ((kb >> 1) - 1) & 1, abort_flag, p);
                 tc_fence_after();
-                uint8_t* stage = smem + j * kStageBytes;
-                issue_cb(tmem + kColCB + 128u * j, smem_u32(stage + kStC), smem_u32(stage + kStB),
-                         0, kBlk);
+                if constexpr (PERN) {
+                    // CB / max u = C B~^T: A = C f16 in the accumulator columns of buffer j, B = B~
+                    // [s][n] K-major in the B' buffer (two 64-channel halves, 128-byte swizzle)
+                    const uint64_t bt = smem_desc(sbase + kOffBp + j * 32768, 16, 1024, kSwizzle128B);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_f16_ts(tmem + kColCB + 128u * j, tmem + kColAcc + 64u * j + 8 * kk,
+                                   bt + (kk >> 2) * (16384 >> 4) + 2 * (kk & 3), id_cb16, kk > 0);
+                } else {
+                    uint8_t* stage = smem + j * kStageBytes;
+                    issue_cb(tmem + kColCB + 128u * j, smem_u32(stage + kStC), smem_u32(stage + kStB),
+                             0, kBlk);
+                }
                 tc_commit(bars + kBarCb0 + j);
                 tc_commit(bars + kBarEmpty0 + j);
             };
@@ -690,7 +712,8 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 const uint64_t xf = d_xf + static_cast<uint64_t>((j * 16384) >> 4);
                 const uint64_t hp = d_hp + static_cast<uint64_t>((j * 16384) >> 4);
                 const uint32_t acc = tmem + kColAcc + 64u * j;
-                if (kb + 1 < nb_total) issue_cb_block(kb + 1);
+                // (per-N scales: later, once the next block's worker has its operands in place)
+                if (!PERN && kb + 1 < nb_total) issue_cb_block(kb + 1);
                 // acc = M' x   (A = M' from TMEM, K = 128 s): opens the accumulator
                 wait_phase(bars + kBarMp0 + j, ph, abort_flag, p);
                 wait_phase(bars + kBarXb0 + j, ph, abort_flag, p);
@@ -707,14 +730,13 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 for (int kk = 0; kk < kBlk / 16; ++kk)
                     mma_f16_ss(tmem + kColH, bp + 128 * kk, xf + 128 * kk, id_st, 1);
                 tc_commit(bars + kBarState);
-                // acc += C' H'^T (A = C' from TMEM, K = 128 n) + x D (K = 64 p)
+                if (PERN && kb + 1 < nb_total) issue_cb_block(kb + 1);
+                // acc += C' H'^T (A = C' from TMEM, K = 128 n)
                 wait_phase(bars + kBarPc0 + j, ph, abort_flag, p);
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_f16_ts(acc, tmem + kColC + 8 * kk, hp + 128 * kk, id_y, 1);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) mma_f16_ss(acc, xf + 2 * kk, d_dm + 2 * kk, id_d, 1);
                 tc_commit(bars + kBarCh);
                 ++n_ch;
                 tc_commit(bars + kBarAcc0 + j);
@@ -754,6 +776,10 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
         // per-piece constants
         int const_seg = -1;
         float sx = 1.f, sBg = 1.f, sCg = 1.f, A2h = 0.f, D_h = 0.f, d_bound = 0.f;
+        // scale of the B C products (s_B s_C, or max_n u_n with per-channel scales), and this
+        // thread's state row n: its B scale and u~_n
+        float uscale = 1.f, sB_row = 1.f, ut_row = 1.f;
+        __half* ut_s = reinterpret_cast<__half*>(smem + kOffUt) + 128 * w;
         float d = w < nb_total ? dt_at(cur) : 0.f;  // dt of this token, this block
         // this worker's previous block, whose output is pending
         int pv_tok = 0, pv_h = 0, pv_valid = 0;  // first packed token of the block
@@ -775,8 +801,8 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                     wv[q] = __byte_perm(lo, hi, 0x5410);
                 }
                 uint4* yo = reinterpret_cast<uint4*>(static_cast<int8_t*>(p.y) + ybase) + 2 * hq;
-                yo[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-                yo[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+                __stcs(yo, make_uint4(wv[0], wv[1], wv[2], wv[3]));  // streamed (evict first)
+                __stcs(yo + 1, make_uint4(wv[4], wv[5], wv[6], wv[7]));
             } else if constexpr (YT == SSD_OUT_F16) {
                 const f2 s2 = {s, s};
                 uint4* yo = reinterpret_cast<uint4*>(static_cast<__half*>(p.y) + ybase) + 4 * hq;
@@ -788,7 +814,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                         const f2 t = fmul2(f2{v[8 * q + 2 * i], v[8 * q + 2 * i + 1]}, s2);
                         wq4[i] = pack_f16x2(t.x, t.y);
                     }
-                    yo[q] = make_uint4(wq4[0], wq4[1], wq4[2], wq4[3]);
+                    __stcs(yo + q, make_uint4(wq4[0], wq4[1], wq4[2], wq4[3]));
                 }
             } else {
                 const f2 s2 = {s, s};
@@ -797,7 +823,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 for (int q = 0; q < 8; ++q) {
                     const f2 t0 = fmul2(f2{v[4 * q], v[4 * q + 1]}, s2);
                     const f2 t1 = fmul2(f2{v[4 * q + 2], v[4 * q + 3]}, s2);
-                    yo[q] = make_float4(t0.x, t0.y, t1.x, t1.y);
+                    __stcs(yo + q, make_float4(t0.x, t0.y, t1.x, t1.y));
                 }
             }
         };
@@ -870,15 +896,32 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 sCg = p.C_scale[g];
                 A2h = p.A[cur.pc.h] * kLog2e;
                 D_h = p.D[cur.pc.h];
-                d_bound = fabsf(D_h) / (sCg * sBg);  // |D s_x / rho| <= 2^14 needs kappa >= this / 2^14
+                if constexpr (PERN) {
+                    // u_n = s_C[g,n] s_B[g,n], its maximum over the channels, u~_n = u_n / max u
+                    const float* sBv = p.B_scale + (size_t)g * p.N;
+                    const float* sCv = p.C_scale + (size_t)g * p.N;
+                    const float u = row < p.N ? sCv[row] * sBv[row] : 0.f;
+                    sB_row = row < p.N ? sBv[row] : 0.f;
+                    float m = fabsf(u);
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                    if (tl == 0) red[8 + wq] = m;
+                    wg_sync(bar_id);
+                    const float umax = fmaxf(fmaxf(red[8], red[9]), fmaxf(red[10], red[11]));
+                    uscale = umax > 0.f ? umax : 1.f;
+                    ut_row = u / uscale;
+                    ut_s[row] = __float2half_rn(ut_row);  // read by the whole worker after the scan's barrier
+                } else {
+                    sB_row = sBg;
+                    uscale = sCg * sBg;
+                }
+                d_bound = fabsf(D_h) / uscale;  // |D s_x / rho| <= 2^14 needs kappa >= this / 2^14
             }
-            const float sigma = sx * sBg;
+            const float sigma_row = sx * sB_row;  // units of state row n
             const int valid = min(kBlk, cur.pc.len - cur.c * kBlk);
             // dt of this worker's next block, in flight during this block
             const float d_next = kb + 2 < nb_total ? dt_at(nxt) : 0.f;
-            // (a) output of this worker's previous block
-            if (kb >= 2) output(kb - 2);
-            // (b) block scan of dt (a_t = log2(e) A cumsum(dt)), with the block's max and sum
+            // (a) block scan of dt (a_t = log2(e) A cumsum(dt)), with the block's max and sum
             float incl, tot, dmax, dsum, a32, a64, a96;
             {
                 float v = d, mx = d;
@@ -911,7 +954,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 a64 = A2h * (wd.z + p2);
                 a96 = A2h * (wd.w + p3);
             }
-            // (c) statistics chained through the workers: the bound hb on |H| / s_x s_B entering
+            // (b) statistics chained through the workers: the bound hb on |H| / s_x s_B entering
             //     this block and the state unit U of the previous block
             const bool pstart = cur.c == cur.pc.cb;
             if (kb >= 1) wait_phase(bars + kBarSt0 + (w ^ 1), ((kb - 1) >> 1) & 1, abort_flag, p);
@@ -924,7 +967,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 // piece start: only the bound of its initial state is needed now; the state goes
                 // into TMEM at the hand-over, after the previous piece's last update
                 hb = piece_state_bound(p, row, red, abort_flag, cur.pc.seq, cur.pc.h, cur.pc.cb,
-                                       sigma, bar_id);
+                                       sigma_row, bar_id);
                 U_prev = 1.f;
             } else {
                 hb = sp.w * sp.x + 16129.f * sp.y;  // bound after block kb - 1's update
@@ -937,8 +980,69 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 stats[2 * w + ph] = make_float4(e_end, dsum, U_new, hb);
                 mbar_arrive(bars + kBarSt0 + w);
             }
-            // (d) x -> f16 and B row scaled by w_t / U -> B'
+            // (c) output of this worker's previous block; its accumulator (C'H' issued at the
+            //     end of that block) completed while the scan and statistics ran.  The wait for
+            //     it also frees x f16 and B' (read by the MMAs of that block) for step (d).
+            if (kb >= 2) output(kb - 2);
+            // (d) x -> f16 and B row scaled by w_t / U -> B' (with per-channel scales first
+            //     ChunkBMM's operands, and B' once ChunkBMM has read B~ from the same buffer)
             wait_phase(bars + kBarFull0 + w, ph, abort_flag, p);
+            auto convert_bp = [&]() {
+                const __half2 w2 = __float2half2_rn(d * ex2f(tot - incl) * inv_U_new);
+                uint4 wv = *reinterpret_cast<const uint4*>(stage + kStB + sw128(row, 0));
+#pragma unroll 2
+                for (int q = 0; q < 8; ++q) {
+                    uint4 nw = wv;
+                    if (q < 7) nw = *reinterpret_cast<const uint4*>(stage + kStB + sw128(row, 16 * (q + 1)));
+                    uint4 o0, o1;
+                    cvt16_scaled(wv, w2, o0, o1);
+                    uint8_t* blk = bp + (q >> 2) * 16384;
+                    *reinterpret_cast<uint4*>(blk + sw128(row, 32 * (q & 3))) = o0;
+                    *reinterpret_cast<uint4*>(blk + sw128(row, 32 * (q & 3) + 16)) = o1;
+                    wv = nw;
+                }
+            };
+            if constexpr (PERN) {
+                // C (f16, exact) into this buffer's accumulator columns -- free since the output
+                // step read them -- and B~ = Bq u~_n into the B' buffer: the operands of CB / max u
+                uint4 wv = *reinterpret_cast<const uint4*>(stage + kStC + sw128(row, 0));
+#pragma unroll 2
+                for (int q = 0; q < 8; ++q) {
+                    uint4 nw = wv;
+                    if (q < 7) nw = *reinterpret_cast<const uint4*>(stage + kStC + sw128(row, 16 * (q + 1)));
+                    uint4 o0, o1;
+                    cvt16(wv, o0, o1);
+                    tmem_st8(tmem_addr(tmem, lane_base, col_acc + 8 * q), o0, o1);
+                    wv = nw;
+                }
+                const uint4* ut4 = reinterpret_cast<const uint4*>(ut_s);
+                wv = *reinterpret_cast<const uint4*>(stage + kStB + sw128(row, 0));
+#pragma unroll 2
+                for (int q = 0; q < 8; ++q) {
+                    uint4 nw = wv;
+                    if (q < 7) nw = *reinterpret_cast<const uint4*>(stage + kStB + sw128(row, 16 * (q + 1)));
+                    uint4 o0, o1;
+                    cvt16(wv, o0, o1);
+                    const uint4 u0 = ut4[2 * q], u1 = ut4[2 * q + 1];
+                    o0 = make_uint4(hmul2_u32(o0.x, *reinterpret_cast<const __half2*>(&u0.x)),
+                                    hmul2_u32(o0.y, *reinterpret_cast<const __half2*>(&u0.y)),
+                                    hmul2_u32(o0.z, *reinterpret_cast<const __half2*>(&u0.z)),
+                                    hmul2_u32(o0.w, *reinterpret_cast<const __half2*>(&u0.w)));
+                    o1 = make_uint4(hmul2_u32(o1.x, *reinterpret_cast<const __half2*>(&u1.x)),
+                                    hmul2_u32(o1.y, *reinterpret_cast<const __half2*>(&u1.y)),
+                                    hmul2_u32(o1.z, *reinterpret_cast<const __half2*>(&u1.z)),
+                                    hmul2_u32(o1.w, *reinterpret_cast<const __half2*>(&u1.w)));
+                    uint8_t* blk = bp + (q >> 2) * 16384;
+                    *reinterpret_cast<uint4*>(blk + sw128(row, 32 * (q & 3))) = o0;
+                    *reinterpret_cast<uint4*>(blk + sw128(row, 32 * (q & 3) + 16)) = o1;
+                    wv = nw;
+                }
+                fence_proxy_async_smem();
+                tmem_st_wait();
+                tc_fence_before();
+                wg_sync(bar_id);
+                if (row == 0) mbar_arrive(bars + kBarCbIn0 + w);
+            }
             {
                 const int lt = row;
                 uint4 wv = *reinterpret_cast<const uint4*>(stage + kStX + (lt >> 2) * 64 + 16 * (lt & 3));
@@ -958,29 +1062,15 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                     wv = nw;
                 }
             }
-            {
-                const __half2 w2 = __float2half2_rn(d * ex2f(tot - incl) * inv_U_new);
-                uint4 wv = *reinterpret_cast<const uint4*>(stage + kStB + sw128(row, 0));
-#pragma unroll 2
-                for (int q = 0; q < 8; ++q) {
-                    uint4 nw = wv;
-                    if (q < 7) nw = *reinterpret_cast<const uint4*>(stage + kStB + sw128(row, 16 * (q + 1)));
-                    uint4 o0, o1;
-                    cvt16_scaled(wv, w2, o0, o1);
-                    uint8_t* blk = bp + (q >> 2) * 16384;
-                    *reinterpret_cast<uint4*>(blk + sw128(row, 32 * (q & 3))) = o0;
-                    *reinterpret_cast<uint4*>(blk + sw128(row, 32 * (q & 3) + 16)) = o1;
-                    wv = nw;
-                }
-            }
+            if constexpr (!PERN) convert_bp();
             fence_proxy_async_smem();
             // (e) scales and M' tables of this block
             float need = fmaxf(fmaxf(hb, 16129.f * static_cast<float>(p.N) * dmax), d_bound) *
                          (1.f / kF16Range);
             need = (need > 1e-30f && need < 1e30f) ? need : 1.f;  // also catches NaN / inf
-            const float rho = pow2_ceil(fmaxf(sCg * sigma * need, 1e-30f));
+            const float rho = pow2_ceil(fmaxf(uscale * sx * need, 1e-30f));
             const float inv_rho = inv_pow2(rho);
-            const float invk = sCg * sigma * inv_rho;  // 1 / kappa
+            const float invk = uscale * sx * inv_rho;  // 1 / kappa
             {
                 const float base = d * invk;
                 nbeta[row] = lg2f(base) - incl;  // dt = 0 gives -inf: no contribution
@@ -991,13 +1081,30 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 }
             }
             wg_sync(bar_id);  // x, B' (for the MMA) and the M' tables complete
-            if (row == 0) mbar_arrive(bars + kBarXb0 + w);
+            if (row == 0 && !PERN) mbar_arrive(bars + kBarXb0 + w);
             // (f) M' in place over CB, one 32-column chunk at a time (increasing order)
             wait_phase(bars + kBarCb0 + w, ph, abort_flag, p);
             tc_fence_after();
+            if constexpr (PERN) {  // ChunkBMM has read B~: B' in its place
+                convert_bp();
+                fence_proxy_async_smem();
+                wg_sync(bar_id);
+                if (row == 0) mbar_arrive(bars + kBarXb0 + w);
+            }
+            // ChunkBMM entries as exact fp32: int32 from the int8 products, or the f32 of the
+            // f16 products (per-channel scales)
+            auto cb2f = [&](uint32_t v0, uint32_t v1) -> f2 {
+                if constexpr (PERN) return f2{__uint_as_float(v0), __uint_as_float(v1)};
+                else return cb_pair(v0, v1);
+            };
             {
                 const float a2t = incl;
                 const f2 a2t2 = {a2t, a2t};
+                // the skip term D x as D s_x / rho on M's diagonal (entry tl of this row's
+                // diagonal sub-block)
+                const float dterm = D_h * sx * inv_rho;
+                const int ediag = tl >> 1;
+                const f2 dd2 = (tl & 1) ? f2{0.f, dterm} : f2{dterm, 0.f};
                 const float rowf = wq > 0 ? ex2f(a2t - (wq == 1 ? a32 : (wq == 2 ? a64 : a96))) : 0.f;
                 const f2 rowf2 = {rowf, rowf};
                 const float* cfq = colf + colf_off(wq);
@@ -1010,7 +1117,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
                         const float2 c2 = cf[e];
-                        const f2 v = fmul2(fmul2(cb_pair(cbv[2 * e], cbv[2 * e + 1]), f2{c2.x, c2.y}), rowf2);
+                        const f2 v = fmul2(fmul2(cb2f(cbv[2 * e], cbv[2 * e + 1]), f2{c2.x, c2.y}), rowf2);
                         o[e] = pack_f16x2(v.x, v.y);
                     }
                     tmem_st16(tmem_addr(tmem, lane_base, col_cb + 16 * sc), o);
@@ -1024,7 +1131,8 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                     for (int e = 0; e < 16; ++e) {
                         const float2 n2 = nb[e];
                         const f2 arg = fadd2(a2t2, f2{n2.x, n2.y});
-                        const f2 v = fmul2(cb_pair(cbv[2 * e], cbv[2 * e + 1]), f2{ex2f(arg.x), ex2f(arg.y)});
+                        f2 v = fmul2(cb2f(cbv[2 * e], cbv[2 * e + 1]), f2{ex2f(arg.x), ex2f(arg.y)});
+                        if (e == ediag) v = fadd2(v, dd2);
                         o[e] = pack_f16x2(2 * e <= tl ? v.x : 0.f, 2 * e + 1 <= tl ? v.y : 0.f);
                     }
                     tmem_st16(tmem_addr(tmem, lane_base, col_cb + 16 * wq), o);
@@ -1053,12 +1161,14 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                     Piece prev;
                     rg.seg(p, cur.seg - 1, prev);
                     store_piece_state(p, tmem, row, prev.ce == prev.nblk, prev.ce != prev.nblk, prev.seq,
-                                      prev.h, sp.z, bar_id);
+                                      prev.h, sp.z, PERN, bar_id);
                 }
-                write_piece_state(p, tmem, row, cur.pc.seq, cur.pc.h, cur.pc.cb, sigma);
+                write_piece_state(p, tmem, row, cur.pc.seq, cur.pc.h, cur.pc.cb, sigma_row);
             }
             {
-                const f2 to_hp = {U_prev * invk, U_prev * invk};
+                // H' = H U / kappa, times u~_n of this row with per-channel scales
+                const float hps = U_prev * invk * ut_row;
+                const f2 to_hp = {hps, hps};
                 const float th = e_end * (U_prev * inv_U_new);
                 const f2 to_h = {th, th};
 #pragma unroll 1
@@ -1091,7 +1201,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             tc_fence_before();
             wg_sync(bar_id);
             if (row == 0) mbar_arrive(bars + kBarPh0 + w);
-            // (h) C row scaled by 2^a_t -> C' in TMEM, and D, once the previous C'H' is done
+            // (h) C row scaled by 2^a_t -> C' in TMEM, once the previous C'H' is done
             if (kb >= 1) wait_phase(bars + kBarCh, (kb - 1) & 1, abort_flag, p);
             tc_fence_after();
             {
@@ -1106,14 +1216,10 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                     tmem_st8(tmem_addr(tmem, lane_base, kColC + 8 * q), o0, o1);
                     wv = nw;
                 }
-                if (row < kP)
-                    *reinterpret_cast<__half*>(smem + kOffDm + sw128(row, 2 * row)) =
-                        __float2half_rn(D_h * sx * inv_rho);
             }
-            fence_proxy_async_smem();
             tmem_st_wait();
             tc_fence_before();
-            wg_sync(bar_id);  // every thread is done with the stage, C' and D are written
+            wg_sync(bar_id);  // every thread is done with the stage, C' is written
             if (row == 0) {
                 mbar_arrive(bars + kBarPc0 + w);
                 mbar_arrive(bars + kBarEmpty0 + w);
@@ -1138,7 +1244,7 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             Piece last;
             rg.seg(p, rg.nseg - 1, last);
             store_piece_state(p, tmem, row, last.ce == last.nblk, last.ce != last.nblk, last.seq, last.h,
-                              last_U, bar_id);
+                              last_U, PERN, bar_id);
         }
     }
 
@@ -1321,14 +1427,21 @@ long long total_blocks(int batch, int seqlen, int nheads) {
     return (long long)batch * nheads * ceil_div(seqlen, kBlk);
 }
 
-template <int YT, bool HAD>
+template <int YT, bool HAD, bool PERN>
 cudaError_t launch_fused(const CUtensorMap& mx, const CUtensorMap& mB, const CUtensorMap& mC,
                          const FusedParams& p, cudaStream_t st) {
-    cudaError_t e = cudaFuncSetAttribute(fused_chunk_scan_kernel<YT, HAD>,
+    cudaError_t e = cudaFuncSetAttribute(fused_chunk_scan_kernel<YT, HAD, PERN>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    fused_chunk_scan_kernel<YT, HAD><<<p.nctas, kThreads, kSmemBytes, st>>>(mx, mB, mC, p);
+    fused_chunk_scan_kernel<YT, HAD, PERN><<<p.nctas, kThreads, kSmemBytes, st>>>(mx, mB, mC, p);
     return cudaGetLastError();
+}
+
+template <int YT, bool HAD>
+cudaError_t launch_fused(const CUtensorMap& mx, const CUtensorMap& mB, const CUtensorMap& mC,
+                         const FusedParams& p, bool per_n, cudaStream_t st) {
+    return per_n ? launch_fused<YT, HAD, true>(mx, mB, mC, p, st)
+                 : launch_fused<YT, HAD, false>(mx, mB, mC, p, st);
 }
 
 }  // namespace
@@ -1402,13 +1515,14 @@ cudaError_t launch_chunk_scan(const ChunkScanArgs& a, cudaStream_t st) {
             g_inject_armed = false;
         }
     }
-    switch (a.y_dtype) {
-        case SSD_OUT_F32: return launch_fused<SSD_OUT_F32, false>(mx, mB, mC, p, st);
-        case SSD_OUT_F16: return launch_fused<SSD_OUT_F16, false>(mx, mB, mC, p, st);
-        case SSD_OUT_I8: return launch_fused<SSD_OUT_I8, false>(mx, mB, mC, p, st);
-        case SSD_OUT_F32 | SSD_OUT_HADAMARD: return launch_fused<SSD_OUT_F32, true>(mx, mB, mC, p, st);
-        case SSD_OUT_F16 | SSD_OUT_HADAMARD: return launch_fused<SSD_OUT_F16, true>(mx, mB, mC, p, st);
-        case SSD_OUT_I8 | SSD_OUT_HADAMARD: return launch_fused<SSD_OUT_I8, true>(mx, mB, mC, p, st);
+    const bool per_n = (a.y_dtype & SSD_SCALES_PER_N) != 0;
+    switch (a.y_dtype & ~SSD_SCALES_PER_N) {
+        case SSD_OUT_F32: return launch_fused<SSD_OUT_F32, false>(mx, mB, mC, p, per_n, st);
+        case SSD_OUT_F16: return launch_fused<SSD_OUT_F16, false>(mx, mB, mC, p, per_n, st);
+        case SSD_OUT_I8: return launch_fused<SSD_OUT_I8, false>(mx, mB, mC, p, per_n, st);
+        case SSD_OUT_F32 | SSD_OUT_HADAMARD: return launch_fused<SSD_OUT_F32, true>(mx, mB, mC, p, per_n, st);
+        case SSD_OUT_F16 | SSD_OUT_HADAMARD: return launch_fused<SSD_OUT_F16, true>(mx, mB, mC, p, per_n, st);
+        case SSD_OUT_I8 | SSD_OUT_HADAMARD: return launch_fused<SSD_OUT_I8, true>(mx, mB, mC, p, per_n, st);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -21,7 +21,7 @@ struct ChunkScanArgs {
     const float* init_state;
     float* final_state;
     void* y;
-    int y_dtype;
+    int y_dtype;  // SSD_OUT_* code with the SSD_OUT_HADAMARD / SSD_SCALES_PER_N flags
     float inv_y_scale;
     void* workspace;
     // packed variable-length sequences (seq_tab == null: `batch` contiguous rows of `seqlen`)
@@ -50,6 +50,7 @@ struct StateUpdateArgs {
     int y_dtype;  // SSD_OUT_* without the Hadamard flag
     float inv_y_scale;
     int hadamard;  // 1: y' = H y / 8 over headdim (64) before the conversion
+    int per_n;     // 1: B_scale / C_scale are [ngroups, dstate]
 };
 
 struct StateUpdateQ8Args {
@@ -69,6 +70,7 @@ struct StateUpdateQ8Args {
     int y_dtype;  // SSD_OUT_* without the Hadamard flag
     float inv_y_scale;
     int hadamard;  // 1: y' = H y / 8 over headdim (64) before the conversion
+    int per_n;     // 1: B_scale / C_scale are [ngroups, dstate]
 };
 
 size_t chunk_scan_workspace_bytes(int batch, int seqlen, int nheads, int headdim, int dstate,

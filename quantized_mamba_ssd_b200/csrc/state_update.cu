@@ -21,7 +21,8 @@ state_update_kernel(float* __restrict__ state, const int8_t* __restrict__ x,
                     const float* __restrict__ dt, const float* __restrict__ A,
                     const float* __restrict__ D, const float* __restrict__ x_scale,
                     const float* __restrict__ B_scale, const float* __restrict__ C_scale,
-                    int H, int P, int G, void* __restrict__ y, int y_dtype, float inv_y_scale) {
+                    int H, int P, int G, int per_n, void* __restrict__ y, int y_dtype,
+                    float inv_y_scale) {
     __shared__ float ys[HAD ? 64 : 1];  // y of this (batch, head) to be transformed (P = 64)
     constexpr int VEC = N / 4;                          // float4 per state row
     constexpr int LPR = VEC < kWarp ? VEC : kWarp;      // lanes per row
@@ -34,7 +35,11 @@ state_update_kernel(float* __restrict__ state, const int8_t* __restrict__ x,
 
     const float dtv = dt[(size_t)b * H + h];
     const float decay = __expf(dtv * A[h]);
-    const float sx = x_scale[h], sB = B_scale[g], sC = C_scale[g], Dh = D[h];
+    const float sx = x_scale[h], Dh = D[h];
+    // B and C scales: per group, or per group and dstate channel (SSDi8 Table 10, per-P(N))
+    const float* sBv = B_scale + (per_n ? (size_t)g * N : g);
+    const float* sCv = C_scale + (per_n ? (size_t)g * N : g);
+    const int sn = per_n ? 1 : 0;
     float bv[VPL][4], cv[VPL][4];
     const int8_t* brow = Bq + ((size_t)b * G + g) * N;
     const int8_t* crow = Cq + ((size_t)b * G + g) * N;
@@ -43,8 +48,11 @@ state_update_kernel(float* __restrict__ state, const int8_t* __restrict__ x,
         const int n0 = (sub + k * LPR) * 4;
         const char4 b4 = *reinterpret_cast<const char4*>(brow + n0);
         const char4 c4 = *reinterpret_cast<const char4*>(crow + n0);
-        bv[k][0] = sB * b4.x; bv[k][1] = sB * b4.y; bv[k][2] = sB * b4.z; bv[k][3] = sB * b4.w;
-        cv[k][0] = sC * c4.x; cv[k][1] = sC * c4.y; cv[k][2] = sC * c4.z; cv[k][3] = sC * c4.w;
+        const int i0 = sn * n0;
+        bv[k][0] = sBv[i0] * b4.x; bv[k][1] = sBv[i0 + sn] * b4.y;
+        bv[k][2] = sBv[i0 + 2 * sn] * b4.z; bv[k][3] = sBv[i0 + 3 * sn] * b4.w;
+        cv[k][0] = sCv[i0] * c4.x; cv[k][1] = sCv[i0 + sn] * c4.y;
+        cv[k][2] = sCv[i0 + 2 * sn] * c4.z; cv[k][3] = sCv[i0 + 3 * sn] * c4.w;
     }
     float4* st = reinterpret_cast<float4*>(state + ((size_t)b * H + h) * P * N);
     const int8_t* xrow = x + ((size_t)b * H + h) * P;
@@ -100,8 +108,8 @@ cudaError_t launch_n(const StateUpdateArgs& a, cudaStream_t st) {
     dim3 grid(a.nheads, a.batch);
     auto kernel = a.hadamard ? state_update_kernel<N, true> : state_update_kernel<N, false>;
     kernel<<<grid, kThreads, 0, st>>>(a.state, a.x, a.B, a.C, a.dt, a.A, a.D, a.x_scale, a.B_scale,
-                                      a.C_scale, a.nheads, a.headdim, a.ngroups, a.y, a.y_dtype,
-                                      a.inv_y_scale);
+                                      a.C_scale, a.nheads, a.headdim, a.ngroups, a.per_n, a.y,
+                                      a.y_dtype, a.inv_y_scale);
     return cudaGetLastError();
 }
 

@@ -148,7 +148,7 @@ state_update_q8_kernel(int8_t* __restrict__ state_q, float* __restrict__ state_s
                        const float* __restrict__ A, const float* __restrict__ D,
                        const float* __restrict__ x_scale, const float* __restrict__ B_scale,
                        const float* __restrict__ C_scale, int count, int H, int P, int G,
-                       void* __restrict__ y, int y_dtype, float inv_y_scale) {
+                       int per_n, void* __restrict__ y, int y_dtype, float inv_y_scale) {
     constexpr int CPR = N / 16;  // 16-byte chunks per state row (lanes per row, <= 16)
     __shared__ float scratch[TPB / kWarp];
     // s_B B_n and s_C C_n (double-buffered), float4 j of chunk cc at [j * CPR + cc]: the lanes
@@ -233,11 +233,23 @@ state_update_q8_kernel(int8_t* __restrict__ state_q, float* __restrict__ state_s
         if (tid < 2 * CPR) {
             f2 v[8];
             unpack16(sbc[s][tid], v);
-            const float sv = tid < CPR ? B_scale[g] : C_scale[g];
+            // scales per group, or per group and dstate channel (SSDi8 Table 10, per-P(N)):
+            // this chunk holds channels 16 (tid % CPR) .. + 15
+            const float* sp = tid < CPR ? B_scale : C_scale;
             float4* dst = (tid < CPR ? sb : sc) + tid % CPR;
+            if (per_n) {
+                const float* sv = sp + (size_t)g * N + 16 * (tid % CPR);
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                dst[i * CPR] = make_float4(sv * v[2 * i].x, sv * v[2 * i].y, sv * v[2 * i + 1].x, sv * v[2 * i + 1].y);
+                for (int i = 0; i < 4; ++i)
+                    dst[i * CPR] = make_float4(sv[4 * i] * v[2 * i].x, sv[4 * i + 1] * v[2 * i].y,
+                                               sv[4 * i + 2] * v[2 * i + 1].x,
+                                               sv[4 * i + 3] * v[2 * i + 1].y);
+            } else {
+                const float sv = sp[g];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    dst[i * CPR] = make_float4(sv * v[2 * i].x, sv * v[2 * i].y, sv * v[2 * i + 1].x, sv * v[2 * i + 1].y);
+            }
         }
         __syncthreads();
 
@@ -387,7 +399,8 @@ cudaError_t launch_q8_nh(const StateUpdateQ8Args& a, cudaStream_t st) {
         const int grid = count < resident ? count : resident;
         state_update_q8_kernel<N, TPB, CH, HAD><<<grid, TPB, 0, st>>>(
             a.state_q, a.state_scale, a.x, a.B, a.C, a.dt, a.A, a.D, a.x_scale, a.B_scale,
-            a.C_scale, count, a.nheads, a.headdim, a.ngroups, a.y, a.y_dtype, a.inv_y_scale);
+            a.C_scale, count, a.nheads, a.headdim, a.ngroups, a.per_n, a.y, a.y_dtype,
+            a.inv_y_scale);
         return cudaGetLastError();
     });
 }

@@ -23,6 +23,7 @@ STATUS_NAMES = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED",
                 3: "SSD_ERR_WORKSPACE", 4: "SSD_ERR_CUDA", 5: "SSD_ERR_TIMEOUT"}
 OUT_DTYPES = {"f32": (0, torch.float32), "f16": (1, torch.float16), "i8": (2, torch.int8)}
 OUT_HADAMARD = 16  # flag: y' = H y / 8 over headdim before the conversion (include/ssd_i8.h)
+SCALES_PER_N = 32  # flag: B_scale / C_scale are [ngroups, dstate] (include/ssd_i8.h)
 
 # names of every extern "C" symbol include/ssd_i8.h declares
 EXPORTED = ("ssd_i8_abi_version", "ssd_status_string", "ssd_i8_chunk_scan_workspace_size",
@@ -149,6 +150,16 @@ def _ptr(t: Optional[torch.Tensor], name: str, dtype: torch.dtype, shape=None) -
     return t.data_ptr() if t.numel() else None
 
 
+def _bc_scales(B_scale: torch.Tensor, C_scale: torch.Tensor, G: int, N: int) -> tuple:
+    """Pointers of the B and C scales, [G] per group or [G, N] per group and dstate channel,
+    and the y_dtype flag that says which."""
+    per_n = isinstance(B_scale, torch.Tensor) and B_scale.dim() == 2
+    shape = (G, N) if per_n else (G,)
+    return (_ptr(B_scale, "B_scale", torch.float32, shape),
+            _ptr(C_scale, "C_scale", torch.float32, shape),
+            SCALES_PER_N if per_n else 0)
+
+
 def _stream(stream) -> Optional[int]:
     if stream is None:
         return torch.cuda.current_stream().cuda_stream
@@ -176,7 +187,8 @@ def ssd_i8_chunk_scan(x: torch.Tensor, B: torch.Tensor, C: torch.Tensor, dt: tor
     applies the output transform y' = H y / 8 over headdim (``SSD_OUT_HADAMARD``).
 
     x int8 [b,l,h,p]; B, C int8 [b,l,g,n]; dt f32 [b,l,h]; A, D, x_scale f32 [h];
-    B_scale, C_scale f32 [g]; optional init_state / final_state f32 [b,h,p,n]; returns y
+    B_scale, C_scale f32 [g] (or [g, n]: per dstate channel, ``SSD_SCALES_PER_N``); optional
+    init_state / final_state f32 [b,h,p,n]; returns y
     [b,l,h,p] of ``y_dtype`` ("f32", "f16" or "i8"; "i8" uses ``y_scale``).  ``workspace`` is
     a uint8 CUDA tensor of at least ``ssd_i8_chunk_scan_workspace_size`` bytes; one is
     allocated through torch when omitted.
@@ -191,6 +203,7 @@ def ssd_i8_chunk_scan(x: torch.Tensor, B: torch.Tensor, C: torch.Tensor, dt: tor
     need = ssd_i8_chunk_scan_workspace_size(bsz, L, H, P, N, G, chunk_size)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    pb, pc, flag = _bc_scales(B_scale, C_scale, G, N)
     args = [
         _ptr(x, "x", torch.int8, (bsz, L, H, P)),
         _ptr(B, "B", torch.int8, (bsz, L, G, N)),
@@ -199,13 +212,12 @@ def ssd_i8_chunk_scan(x: torch.Tensor, B: torch.Tensor, C: torch.Tensor, dt: tor
         _ptr(A, "A", torch.float32, (H,)),
         _ptr(D, "D", torch.float32, (H,)),
         _ptr(x_scale, "x_scale", torch.float32, (H,)),
-        _ptr(B_scale, "B_scale", torch.float32, (G,)),
-        _ptr(C_scale, "C_scale", torch.float32, (G,)),
+        pb, pc,
         bsz, L, H, P, N, G, int(chunk_size),
         _ptr(init_state, "init_state", torch.float32, (bsz, H, P, N)),
         _ptr(final_state, "final_state", torch.float32, (bsz, H, P, N)),
         _ptr(y, "y", tdt, (bsz, L, H, P)),
-        code | (OUT_HADAMARD if hadamard else 0), float(y_scale),
+        code | (OUT_HADAMARD if hadamard else 0) | flag, float(y_scale),
         _ptr(workspace, "workspace", torch.uint8),
         workspace.numel(),
         _stream(stream),
@@ -278,18 +290,18 @@ def ssd_i8_chunk_scan_varlen(x: torch.Tensor, B: torch.Tensor, C: torch.Tensor, 
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
     cu_arr = (ctypes.c_int32 * len(cu))(*cu)
+    pbs, pcs, flag = _bc_scales(B_scale, C_scale, G, N)
     args = [
         xp, xs, bp, cp, bs, dp, ds,
         _ptr(A, "A", torch.float32, (H,)),
         _ptr(D, "D", torch.float32, (H,)),
         _ptr(x_scale, "x_scale", torch.float32, (H,)),
-        _ptr(B_scale, "B_scale", torch.float32, (G,)),
-        _ptr(C_scale, "C_scale", torch.float32, (G,)),
+        pbs, pcs,
         ctypes.cast(cu_arr, ctypes.c_void_p), nseq, T, H, P, N, G, int(chunk_size),
         _ptr(init_state, "init_state", torch.float32, (nseq, H, P, N)),
         _ptr(final_state, "final_state", torch.float32, (nseq, H, P, N)),
         _ptr(y, "y", tdt, (T, H, P)),
-        code | (OUT_HADAMARD if hadamard else 0), float(y_scale),
+        code | (OUT_HADAMARD if hadamard else 0) | flag, float(y_scale),
         _ptr(workspace, "workspace", torch.uint8),
         workspace.numel(),
         _stream(stream),
@@ -312,6 +324,7 @@ def ssd_i8_state_update(state: torch.Tensor, x: torch.Tensor, B: torch.Tensor, C
     code, tdt = OUT_DTYPES[y_dtype]
     if y is None:
         y = torch.empty((bsz, H, P), dtype=tdt, device=state.device)
+    pb, pc, flag = _bc_scales(B_scale, C_scale, G, N)
     args = [
         _ptr(state, "state", torch.float32, (bsz, H, P, N)),
         _ptr(x, "x", torch.int8, (bsz, H, P)),
@@ -321,11 +334,10 @@ def ssd_i8_state_update(state: torch.Tensor, x: torch.Tensor, B: torch.Tensor, C
         _ptr(A, "A", torch.float32, (H,)),
         _ptr(D, "D", torch.float32, (H,)),
         _ptr(x_scale, "x_scale", torch.float32, (H,)),
-        _ptr(B_scale, "B_scale", torch.float32, (G,)),
-        _ptr(C_scale, "C_scale", torch.float32, (G,)),
+        pb, pc,
         bsz, H, P, N, G,
         _ptr(y, "y", tdt, (bsz, H, P)),
-        code | (OUT_HADAMARD if hadamard else 0), float(y_scale),
+        code | (OUT_HADAMARD if hadamard else 0) | flag, float(y_scale),
         _stream(stream),
     ]
     _check("ssd_i8_state_update", library().ssd_i8_state_update(*args))
@@ -367,6 +379,7 @@ def ssd_i8_state_update_q8(state_q: torch.Tensor, state_scale: torch.Tensor, x: 
     code, tdt = OUT_DTYPES[y_dtype]
     if y is None:
         y = torch.empty((bsz, H, P), dtype=tdt, device=state_q.device)
+    pb, pc, flag = _bc_scales(B_scale, C_scale, G, N)
     args = [
         _ptr(state_q, "state_q", torch.int8, (bsz, H, P, N)),
         _ptr(state_scale, "state_scale", torch.float32, (bsz, H)),
@@ -377,11 +390,10 @@ def ssd_i8_state_update_q8(state_q: torch.Tensor, state_scale: torch.Tensor, x: 
         _ptr(A, "A", torch.float32, (H,)),
         _ptr(D, "D", torch.float32, (H,)),
         _ptr(x_scale, "x_scale", torch.float32, (H,)),
-        _ptr(B_scale, "B_scale", torch.float32, (G,)),
-        _ptr(C_scale, "C_scale", torch.float32, (G,)),
+        pb, pc,
         bsz, H, P, N, G,
         _ptr(y, "y", tdt, (bsz, H, P)),
-        code | (OUT_HADAMARD if hadamard else 0), float(y_scale),
+        code | (OUT_HADAMARD if hadamard else 0) | flag, float(y_scale),
         _stream(stream),
     ]
     _check("ssd_i8_state_update_q8", library().ssd_i8_state_update_q8(*args))
@@ -450,13 +462,12 @@ def ssd_i8_chunk_scan_noalloc(x: torch.Tensor, B: torch.Tensor, C: torch.Tensor,
         _ptr(A, "A", torch.float32, (H,)),
         _ptr(D, "D", torch.float32, (H,)),
         _ptr(x_scale, "x_scale", torch.float32, (H,)),
-        _ptr(B_scale, "B_scale", torch.float32, (G,)),
-        _ptr(C_scale, "C_scale", torch.float32, (G,)),
+        *_bc_scales(B_scale, C_scale, G, N)[:2],
         bsz, L, H, P, N, G, int(chunk_size),
         _ptr(init_state, "init_state", torch.float32, (bsz, H, P, N)),
         _ptr(final_state, "final_state", torch.float32, (bsz, H, P, N)),
         _ptr(y, "y", tdt, (bsz, L, H, P)),
-        code, float(y_scale),
+        code | _bc_scales(B_scale, C_scale, G, N)[2], float(y_scale),
         _stream(stream),
     ]
     _check("ssd_i8_chunk_scan_noalloc", library().ssd_i8_chunk_scan_noalloc(*args))

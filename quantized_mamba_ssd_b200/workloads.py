@@ -218,8 +218,8 @@ def make_prefill(batch: int, seqlen: int, nheads: int, headdim: int, dstate: int
     per head and B, C per group by U(0.5, 8)); "laplace_outliers_all" (x, B, C Laplace with
     1 % outlier channels x20: x over (h,p), B and C over (g,n)).
     scales: "tensor" (one scale per tensor, broadcast), "head" (x per head, B/C per group),
-    "channel" (x per head, B/C per group and dstate channel, [g, n] -- the oracle's per-N
-    scan; the CUDA kernels take per-group scales) or "percentile" (per tensor; x clipped at
+    "channel" (x per head, B/C per group and dstate channel, [g, n]: the per-P(N) axis, taken
+    by the kernels with SSD_SCALES_PER_N) or "percentile" (per tensor; x clipped at
     ``clip_percentile`` of |x|, B/C by absmax).
     """
     if nheads % ngroups:
@@ -301,11 +301,13 @@ def make_prefill_config(index: int, seed: Optional[int] = None, **overrides) -> 
 
 
 def make_decode(batch: int, steps: int, nheads: int, headdim: int, dstate: int, ngroups: int, *,
-                out_dtype: str = "f16", seed: int = 0, name: Optional[str] = None) -> DecodeCase:
+                out_dtype: str = "f16", seed: int = 0, name: Optional[str] = None,
+                scales: str = "head") -> DecodeCase:
     """Draw a seeded decode run: an fp32 state ~ N(0, 0.1^2) and ``steps`` fresh tokens.
 
-    Per step x, B, C ~ N(0, 1), quantized with static scales (x per head, B/C per group)
-    calibrated over all steps; dt, A, D as in the prefill workloads.
+    Per step x, B, C ~ N(0, 1), quantized with static scales (x per head, B/C per group, or
+    with ``scales="channel"`` per group and dstate channel, [g, n]) calibrated over all steps;
+    dt, A, D as in the prefill workloads.
     """
     if nheads % ngroups:
         raise ValueError("nheads must be a multiple of ngroups")
@@ -316,8 +318,14 @@ def make_decode(batch: int, steps: int, nheads: int, headdim: int, dstate: int, 
     Cf = _normal(rng, (steps, batch, ngroups, dstate))
     state = (0.1 * _normal(rng, (batch, nheads, headdim, dstate))).astype(F32)
     xq, sx = quantize_symmetric(x, 2)
-    Bq, sb = quantize_symmetric(Bf, 2)
-    Cq, sc = quantize_symmetric(Cf, 2)
+    if scales == "head":
+        Bq, sb = quantize_symmetric(Bf, 2)
+        Cq, sc = quantize_symmetric(Cf, 2)
+    elif scales == "channel":
+        Bq, sb = quantize_symmetric(Bf, (2, 3))
+        Cq, sc = quantize_symmetric(Cf, (2, 3))
+    else:
+        raise ValueError(f"unknown scales {scales!r}")
     return DecodeCase(
         name=name or f"decode b{batch} x{steps} h{nheads} p{headdim} n{dstate} g{ngroups}",
         batch=batch, steps=steps, nheads=nheads, headdim=headdim, dstate=dstate,

@@ -80,6 +80,9 @@ def _scan_args(**over):
     (dict(H=6, G=4), 1),          # H % G != 0
     (dict(yd=7), 1),              # bad dtype code
     (dict(yd=2, ys=0.0), 1),      # int8 output needs y_scale > 0
+    (dict(yd=2 | 32, ys=0.0), 1),  # the same with per-channel B/C scales (flag parsed)
+    (dict(yd=64), 1),             # unknown flag bit
+    (dict(yd=7 | 32), 1),         # bad dtype code under the per-channel flag
     (dict(A=None), 1),            # null pointer
     (dict(P=32), 2),              # headdim not implemented
     (dict(N=48), 2),              # dstate not implemented
@@ -108,6 +111,15 @@ def test_state_update_rejects_bad_arguments_on_host(lib):
     null_state = list(base)
     null_state[0] = None
     assert f(*null_state) == 1
+
+
+def test_per_channel_flag_reaches_the_decode_checks(lib):
+    f = lib.ssd_i8_state_update
+    base = [1] * 10 + [1, 4, 64, 16, 1, 1, 2 | 32, 0.0, None]  # int8 out with per-channel scales
+    assert f(*base) == 1  # y_scale 0 refused: the flag combination is understood
+    q8 = lib.ssd_i8_state_update_q8
+    base = [1] * 11 + [1, 4, 64, 16, 1, 1, 7 | 32, 1.0, None]
+    assert q8(*base) == 1  # a bad dtype code under the flag
 
 
 def test_chunk_cb_rejects_bad_arguments_on_host(lib):
