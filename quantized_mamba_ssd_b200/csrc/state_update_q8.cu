@@ -57,6 +57,13 @@ __device__ __forceinline__ f2 ffma2(f2 a, f2 b, f2 c) {
     return r;
 }
 
+// max(m, |a.x|, |a.y|): one three-input maximum
+__device__ __forceinline__ float amax3(float m, f2 a) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(m), "f"(fabsf(a.x)), "f"(fabsf(a.y)));
+    return r;
+}
+
 // 16 int8 codes (one 16-byte chunk) -> 8 pairs of floats, exactly: the byte (sign bit flipped)
 // becomes the low mantissa byte of 2^23, and 2^23 + 128 comes off again (one packed subtract
 // per pair)
@@ -83,6 +90,20 @@ __device__ __forceinline__ uint4 pack16(const f2 (&v)[8], float inv) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const f2 a = fadd2(fmul2(v[2 * i], i2), rnd), b = fadd2(fmul2(v[2 * i + 1], i2), rnd);
+        ww[i] = __byte_perm(__byte_perm(__float_as_uint(a.x), __float_as_uint(a.y), 0x0040),
+                            __byte_perm(__float_as_uint(b.x), __float_as_uint(b.y), 0x0040), 0x5410);
+    }
+    return make_uint4(ww[0], ww[1], ww[2], ww[3]);
+}
+
+// pack16 with the rounding in one step: q = rne(v * inv) of the exact product (an FMA with the
+// rounding constant); the same bound |v * inv| < 127.5 makes a clamp unnecessary
+__device__ __forceinline__ uint4 pack16_fma(const f2 (&v)[8], float inv) {
+    const f2 i2 = {inv, inv}, rnd = {12582912.f, 12582912.f};
+    uint32_t ww[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const f2 a = ffma2(v[2 * i], i2, rnd), b = ffma2(v[2 * i + 1], i2, rnd);
         ww[i] = __byte_perm(__byte_perm(__float_as_uint(a.x), __float_as_uint(a.y), 0x0040),
                             __byte_perm(__float_as_uint(b.x), __float_as_uint(b.y), 0x0040), 0x5410);
     }
@@ -276,8 +297,7 @@ state_update_q8_kernel(int8_t* __restrict__ state_q, float* __restrict__ state_s
                 hv[2 * i + 1] = ffma2(ds, hv[2 * i + 1], fmul2(dx, f2{bb.z, bb.w}));
                 acc = ffma2(f2{cq.x, cq.y}, hv[2 * i], acc);
                 acc = ffma2(f2{cq.z, cq.w}, hv[2 * i + 1], acc);
-                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(hv[2 * i].x), fabsf(hv[2 * i].y)),
-                                         fmaxf(fabsf(hv[2 * i + 1].x), fabsf(hv[2 * i + 1].y))));
+                amax = amax3(amax3(amax, hv[2 * i]), hv[2 * i + 1]);
             }
             float a = acc.x + acc.y;
 #pragma unroll
@@ -309,7 +329,7 @@ state_update_q8_kernel(int8_t* __restrict__ state_q, float* __restrict__ state_s
                 hv[2 * i] = ffma2(ds, hv[2 * i], fmul2(dx, f2{bb.x, bb.y}));
                 hv[2 * i + 1] = ffma2(ds, hv[2 * i + 1], fmul2(dx, f2{bb.z, bb.w}));
             }
-            st[u] = pack16(hv, inv);  // the same fp32 values as the max pass (same operations)
+            st[u] = pack16_fma(hv, inv);  // the same fp32 values as the max pass (same operations)
         }
         if (tid == 0) state_scale[item] = amax / 127.f;
         if (next >= count) break;

@@ -7,11 +7,25 @@ Tolerances are the ones the target states for the int8 SSD scan:
 """
 from __future__ import annotations
 
+import json
+import os
+
 import numpy as np
 
 MAXABS_REL = 2e-3
 REL_L2 = 1e-3
 I8_LSB_FRACTION = 0.9999
+
+
+def _log_margin(record: dict) -> None:
+    """With SSD_PARITY_LOG set to a file path, append the check's achieved error as a fraction
+    of its tolerance (one JSON line per check, tagged with the running test)."""
+    path = os.environ.get("SSD_PARITY_LOG")
+    if not path:
+        return
+    record["test"] = os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0]
+    with open(path, "a") as f:
+        f.write(json.dumps(record) + "\n")
 
 
 def check_close(got, ref, what: str = "y"):
@@ -24,6 +38,8 @@ def check_close(got, ref, what: str = "y"):
     maxabs = err.max() if err.size else 0.0
     nrm = np.linalg.norm(ref)
     rel = np.linalg.norm(got - ref) / nrm if nrm > 0 else np.linalg.norm(got - ref)
+    _log_margin({"what": what, "maxabs_of_tol": float(maxabs / (MAXABS_REL * scale)) if scale > 0
+                 else 0.0, "relL2_of_tol": float(rel / REL_L2)})
     assert maxabs <= MAXABS_REL * scale + 1e-30, \
         f"{what}: max-abs err {maxabs:.3e} > {MAXABS_REL} * max|ref| ({scale:.3e})"
     assert rel <= REL_L2, f"{what}: rel-L2 err {rel:.3e} > {REL_L2}"
@@ -37,6 +53,8 @@ def check_i8(got, ref_q):
     assert got.min() >= -127 and got.max() <= 127, "int8 output outside the symmetric range"
     d = np.abs(got - ref_q)
     within = (d <= 1).mean() if d.size else 1.0
+    _log_margin({"what": "int8", "differ_fraction": float((d != 0).mean()) if d.size else 0.0,
+                 "max_lsb": int(d.max()) if d.size else 0})
     assert within >= I8_LSB_FRACTION, f"only {within:.6f} of int8 outputs within +-1 LSB"
     return within, int(d.max()) if d.size else 0
 
