@@ -80,24 +80,10 @@ __device__ __forceinline__ void unpack16(const uint4 w, f2 (&v)[8]) {
     }
 }
 
-// q = rne(fp32(v * inv)) of 16 values -> one 16-byte chunk, for inv = 127 / max|v| taken over the
-// same fp32 values: then |v * inv| <= 127 (1 + 2^-22) < 127.5, so no clamp is needed.  Adding
+// q = rne(v * inv) of 16 values -> one 16-byte chunk, for inv = 127 / max|v| taken over the same
+// fp32 values: then |v * inv| <= 127 (1 + 2^-22) < 127.5, so no clamp is needed.  Adding
 // 1.5 * 2^23 rounds to an integer (half to even) in the low mantissa bits, whose low byte is then
-// the code.  The multiply and the add are separate roundings (no contraction).
-__device__ __forceinline__ uint4 pack16(const f2 (&v)[8], float inv) {
-    const f2 i2 = {inv, inv}, rnd = {12582912.f, 12582912.f};
-    uint32_t ww[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const f2 a = fadd2(fmul2(v[2 * i], i2), rnd), b = fadd2(fmul2(v[2 * i + 1], i2), rnd);
-        ww[i] = __byte_perm(__byte_perm(__float_as_uint(a.x), __float_as_uint(a.y), 0x0040),
-                            __byte_perm(__float_as_uint(b.x), __float_as_uint(b.y), 0x0040), 0x5410);
-    }
-    return make_uint4(ww[0], ww[1], ww[2], ww[3]);
-}
-
-// pack16 with the rounding in one step: q = rne(v * inv) of the exact product (an FMA with the
-// rounding constant); the same bound |v * inv| < 127.5 makes a clamp unnecessary
+// the code; the multiply and the add are one FMA (one rounding, of the exact product).
 __device__ __forceinline__ uint4 pack16_fma(const f2 (&v)[8], float inv) {
     const f2 i2 = {inv, inv}, rnd = {12582912.f, 12582912.f};
     uint32_t ww[4];
@@ -110,7 +96,8 @@ __device__ __forceinline__ uint4 pack16_fma(const f2 (&v)[8], float inv) {
     return make_uint4(ww[0], ww[1], ww[2], ww[3]);
 }
 
-// scalar form of pack16 for the fp32 quantiser
+// the same rule for the fp32 quantiser, with the multiply and the add rounded separately (the
+// documented rule: rne of the fp32 product)
 __device__ __forceinline__ uint4 pack16(const float (&v)[16], float inv) {
     constexpr float kRound = 12582912.f;
     uint32_t ww[4];
