@@ -49,7 +49,7 @@ NOMINAL_HBM_GBS = 7700.0  # B200 HBM3e datasheet bandwidth (HGX), context for th
 # profiles/ncu_fused_chunk_scan_b2_L8192.md.  The traffic grows in proportion to the tokens of a
 # launch, so the bench scales it to the workload.  A changed kernel reports null.
 _CAPTURED_TRAFFIC_PER_TOKEN = {
-    "77635acbb725d88e8ff7820df0837e5e61cfb48b8edfc3e471302a80cb6e654d": (330.561024e6 + 116.753152e6) / 16384,
+    "82da36d30a3b33808cff01661fd1091f433c59f7488d8f645071cff230a5d608": (329.368576e6 + 108.555520e6) / 16384,
 }
 
 
@@ -60,7 +60,8 @@ _CAPTURED_DECODE_TRAFFIC_PER_ITEM = {
         "562e8c1b5451d3c1c4461d0695738535cba2ca35b3b7ee7fd354a78db864eb83": (134.587904e6 + 76.073984e6) / (32 * 128),
     },
     "state_update_q8.cu": {
-        "ff2801f6675cd1af6669cf61f0875ce58c99cd3ecf6964a44a2f6df0b30a2a13": (135.689216e6 + 77.368832e6) / (128 * 128),
+        # captured on the source 5b540318...; this one differs by comments and an unused helper
+        "163058fc1d5ec17c0f39aa41cbe624d32d1f0c9b841046783ff8da9fefcc7881": (135.700480e6 + 77.127680e6) / (128 * 128),
     },
 }
 
