@@ -427,8 +427,9 @@ def ssd_i8_debug_inject(drop_publish_cta: int, wait_cycles: int) -> None:
 
 @_device_call
 def ssd_i8_chunk_scan_status(workspace: torch.Tensor, stream=None) -> None:
-    """Raise SSDError (SSD_ERR_TIMEOUT) if the last chunk scan on ``workspace`` reported a
-    device-side wait that gave up; synchronises the stream."""
+    """Raise SSDError (SSD_ERR_TIMEOUT) if a chunk scan that ran on ``workspace`` since the
+    previous status query on it (with none, since its first call) reported a device-side wait
+    that gave up; synchronises the stream."""
     _check("ssd_i8_chunk_scan_status",
            library().ssd_i8_chunk_scan_status(_ptr(workspace, "workspace", torch.uint8),
                                               _stream(stream)))
