@@ -290,6 +290,42 @@ def make_prefill(batch: int, seqlen: int, nheads: int, headdim: int, dstate: int
         x_scale=sx, B_scale=sb, C_scale=sc, out_dtype=out_dtype, init_state=init)
 
 
+def make_exact_readout(batch: int, seqlen: int, ngroups: int, dstate: int, chunk_size: int = 256,
+                       seed: int = 0, dt_log2: int = -3, headdim: int = 64) -> PrefillCase:
+    """A prefill whose every intermediate is exactly representable, so that y reads out the
+    ChunkBMM products one by one.
+
+    B and C codes are drawn uniformly from {-1, 0, 1}; x is one-hot: head j of a group (there
+    are ceil(seqlen / headdim) heads per group) carries a 1 at token headdim * j + p in column p
+    and 0 elsewhere.  dt is 2^dt_log2 everywhere, A = D = 0 (no decay, no skip term), and the
+    scales are powers of two (s_x = 1/2, s_B = 1/4, s_C = 1/2).  With the state starting at
+    zero, the SSM recurrence then gives
+        y[b, t, h, p] = dt s_x s_B s_C (C_t . B_s),  s = headdim * j + p <= t  (0 for s > t)
+    for head h = j of group g, an integer times a power of two."""
+    if seqlen < 1 or headdim < 1:
+        raise ValueError("need seqlen >= 1 and headdim >= 1")
+    rng = np.random.default_rng(seed)
+    per_group = -(-seqlen // headdim)
+    H = ngroups * per_group
+    x = np.zeros((batch, seqlen, H, headdim), dtype=np.int8)
+    for h in range(H):
+        j = h % per_group
+        for p in range(headdim):
+            s = headdim * j + p
+            if s < seqlen:
+                x[:, s, h, p] = 1
+    B = rng.integers(-1, 2, size=(batch, seqlen, ngroups, dstate)).astype(np.int8)
+    C = rng.integers(-1, 2, size=(batch, seqlen, ngroups, dstate)).astype(np.int8)
+    dt = np.full((batch, seqlen, H), 2.0 ** dt_log2, dtype=np.float32)
+    zeros_h = np.zeros(H, dtype=np.float32)
+    return PrefillCase(
+        name=f"exact readout b{batch} L{seqlen} h{H} p{headdim} n{dstate} g{ngroups} Q{chunk_size}",
+        batch=batch, seqlen=seqlen, nheads=H, headdim=headdim, dstate=dstate, ngroups=ngroups,
+        chunk_size=chunk_size, x=x, B=B, C=C, dt=dt, A=zeros_h, D=zeros_h.copy(),
+        x_scale=np.full(H, 0.5, dtype=np.float32), B_scale=np.full(ngroups, 0.25, dtype=np.float32),
+        C_scale=np.full(ngroups, 0.5, dtype=np.float32), out_dtype="f32")
+
+
 def make_prefill_config(index: int, seed: Optional[int] = None, **overrides) -> PrefillCase:
     """The prefill workload ``index`` (0..4) with its default seed 1000 + index."""
     spec = dict(PREFILL_CONFIGS[index])
