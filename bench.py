@@ -57,7 +57,7 @@ _CAPTURED_TRAFFIC_PER_TOKEN = {
 # profiles/ncu_state_update_decode_b32.md and profiles/ncu_state_update_q8_decode_b128.md.
 _CAPTURED_DECODE_TRAFFIC_PER_ITEM = {
     "state_update.cu": {
-        "562e8c1b5451d3c1c4461d0695738535cba2ca35b3b7ee7fd354a78db864eb83": (134.587904e6 + 76.073984e6) / (32 * 128),
+        "dbcc58a871c5d4171d5134d6be749c7661410af95c3498b2f3f5b0a99ad2ffdc": (134.594304e6 + 75.850496e6) / (32 * 128),
     },
     "state_update_q8.cu": {
         # captured on the source 5b540318...; this one differs by comments and an unused helper
