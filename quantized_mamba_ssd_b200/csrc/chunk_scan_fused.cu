@@ -38,7 +38,8 @@
 //
 // Warp roles, coupled only through mbarriers (buffers alternate with the block parity j):
 //   warp 8      TMA: x, B, C tiles of block k into stage j
-//   warp 9      MMA issue: CB(k+1); M'x(k); state(k); C'H'(k) + x D(k)
+//   warp 9      MMA issue: CB(k+1); M'x(k) (the skip term rides on M's diagonal); state(k);
+//               C'H'(k)
 //   warps 0-3   block worker for even blocks, warps 4-7 for odd blocks: both run the same
 //               compact loop (the kernel is limited by instruction fetch, and two warps on an
 //               SM sub-partition that run the same code share it): block scan of dt, block
