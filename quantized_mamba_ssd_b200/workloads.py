@@ -326,6 +326,41 @@ def make_exact_readout(batch: int, seqlen: int, ngroups: int, dstate: int, chunk
         C_scale=np.full(ngroups, 0.5, dtype=np.float32), out_dtype="f32")
 
 
+def make_exact_readout_varlen(lengths, ngroups: int, dstate: int, chunk_size: int = 256,
+                              seed: int = 0, headdim: int = 64):
+    """The exact-readout family (``make_exact_readout``) over packed sequences of the given
+    lengths: one row of sum(lengths) tokens, and in sequence i head j of a group carries a 1 at
+    the sequence's token headdim * j + p in column p.  Every sequence shares the head count
+    ngroups * ceil(max length / headdim).  Returns (case with batch 1, cu_seqlens int32)."""
+    lengths = np.asarray(lengths, dtype=np.int64)
+    if lengths.ndim != 1 or (lengths < 0).any():
+        raise ValueError("lengths must be a 1-D sequence of non-negative integers")
+    T = int(lengths.sum())
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    per_group = max(1, -(-int(lengths.max(initial=0)) // headdim))
+    H = ngroups * per_group
+    rng = np.random.default_rng(seed)
+    x = np.zeros((1, max(T, 1), H, headdim), dtype=np.int8)
+    for i, L in enumerate(lengths):
+        for h in range(H):
+            j = h % per_group
+            for p in range(headdim):
+                t = headdim * j + p
+                if t < L:
+                    x[0, cu[i] + t, h, p] = 1
+    B = rng.integers(-1, 2, size=(1, max(T, 1), ngroups, dstate)).astype(np.int8)
+    C = rng.integers(-1, 2, size=(1, max(T, 1), ngroups, dstate)).astype(np.int8)
+    dt = np.full((1, max(T, 1), H), 0.125, dtype=np.float32)
+    zeros_h = np.zeros(H, dtype=np.float32)
+    case = PrefillCase(
+        name=f"exact readout packed T{T} nseq{len(lengths)} h{H} p{headdim} n{dstate} g{ngroups}",
+        batch=1, seqlen=max(T, 1), nheads=H, headdim=headdim, dstate=dstate, ngroups=ngroups,
+        chunk_size=chunk_size, x=x, B=B, C=C, dt=dt, A=zeros_h, D=zeros_h.copy(),
+        x_scale=np.full(H, 0.5, dtype=np.float32), B_scale=np.full(ngroups, 0.25, dtype=np.float32),
+        C_scale=np.full(ngroups, 0.5, dtype=np.float32), out_dtype="f32")
+    return case, cu
+
+
 def make_prefill_config(index: int, seed: Optional[int] = None, **overrides) -> PrefillCase:
     """The prefill workload ``index`` (0..4) with its default seed 1000 + index."""
     spec = dict(PREFILL_CONFIGS[index])

@@ -139,3 +139,83 @@ def test_fused_scan_is_exact_on_the_readout_family(_lib, b, L, G, N, Q, init):
     # Hadamard-transformed output H y / 8: butterflies of small dyadic values, exact too
     yh, _ = _gpu(case, h0, "f32", hadamard=True)
     assert np.array_equal(yh.numpy().astype(np.float64), oracle.hadamard(y_ref))
+
+
+# ---------------------------------------------------------------------------------------------
+# The same family on the other entry points: packed sequences (the state restarts in each
+# sequence, the sequence table, empty and one-token sequences), B and C scales per dstate
+# channel (ChunkBMM on f16; power-of-two channel scales keep every operand exact), and the
+# fp32-state decode step.
+# ---------------------------------------------------------------------------------------------
+@pytest.mark.gpu
+def test_packed_sequences_are_exact_on_the_readout_family(_lib):
+    lengths = [320, 1, 0, 200, 700, 130]
+    case, cu = W.make_exact_readout_varlen(lengths, 2, 128, seed=11)
+    H, P, N = case.nheads, case.headdim, case.dstate
+    nseq = len(lengths)
+    T = int(cu[-1])
+    fs = torch.full((nseq, H, P, N), float("nan"), dtype=torch.float32, device=DEV)
+    y = ssd_i8.ssd_i8_chunk_scan_varlen(
+        _dev(case.x[0, :T]), _dev(case.B[0, :T]), _dev(case.C[0, :T]), _dev(case.dt[0, :T]),
+        _dev(case.A), _dev(case.D), _dev(case.x_scale), _dev(case.B_scale), _dev(case.C_scale),
+        cu, case.chunk_size, final_state=fs, y_dtype="f32")
+    torch.cuda.synchronize()
+    y = y.cpu().numpy().astype(np.float64)
+    fs = fs.cpu().numpy().astype(np.float64)
+    for i in range(nseq):
+        a, b = int(cu[i]), int(cu[i + 1])
+        if b > a:
+            yr, fr = oracle.scan(case.x[:, a:b], case.B[:, a:b], case.C[:, a:b], case.dt[:, a:b],
+                                 case.A, case.D, case.x_scale, case.B_scale, case.C_scale)[:2]
+            assert np.array_equal(y[a:b], yr[0]), f"sequence {i}: y differs"
+            assert np.array_equal(fs[i], fr[0]), f"sequence {i}: final state differs"
+        else:
+            assert np.array_equal(fs[i], np.zeros_like(fs[i])), "empty sequence: state not zero"
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("N", [64, 128])
+def test_per_channel_scales_are_exact_on_the_readout_family(_lib, N):
+    case = W.make_exact_readout(2, 300, 2, N, 256, seed=N)
+    rng = np.random.default_rng(N + 1)
+    G = case.ngroups
+    # s_B[g, n] in {1/4, 1/8}, s_C = 1/2: u = s_B s_C in {1/8, 1/16}, u / max u in {1, 1/2}, so
+    # C . (B u / max u) is a multiple of 1/2 below 2^8 in magnitude: exact in f16 and fp32
+    case.B_scale = (2.0 ** -rng.integers(2, 4, size=(G, N))).astype(np.float32)
+    case.C_scale = np.full((G, N), 0.5, dtype=np.float32)
+    y_ref, fs_ref = oracle.scan(case.x, case.B, case.C, case.dt, case.A, case.D, case.x_scale,
+                                case.B_scale, case.C_scale)[:2]
+    y, fs = _gpu(case, None, "f32")
+    assert np.array_equal(y.numpy().astype(np.float64), y_ref)
+    assert np.array_equal(fs.astype(np.float64), fs_ref)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("N,hadamard", [(128, False), (16, False), (128, True)])
+def test_decode_steps_are_exact_on_the_readout_family(_lib, N, hadamard):
+    """Five fp32-state decode steps with A = D = 0, dt and scales powers of two, x, B, C codes
+    in {-1, 0, 1} and a state of multiples of 1/8: every update and every y is exact."""
+    b, H, P, G = 3, 4, 64, 2
+    rng = np.random.default_rng(N + 7)
+    state = (rng.integers(-2, 3, size=(b, H, P, N)) / 8.0).astype(np.float32)
+    ref = state.astype(np.float64)
+    A = np.zeros(H, dtype=np.float32)
+    D = np.zeros(H, dtype=np.float32)
+    sx = np.full(H, 0.5, dtype=np.float32)
+    sb = np.full(G, 0.25, dtype=np.float32)
+    sc = np.full(G, 0.5, dtype=np.float32)
+    st = _dev(state)
+    for step in range(5):
+        x = rng.integers(-1, 2, size=(b, H, P)).astype(np.int8)
+        B = rng.integers(-1, 2, size=(b, G, N)).astype(np.int8)
+        C = rng.integers(-1, 2, size=(b, G, N)).astype(np.int8)
+        dt = np.full((b, H), 0.125, dtype=np.float32)
+        y_ref = oracle.step(ref, x, B, C, dt, A, D, sx, sb, sc)
+        if hadamard:
+            y_ref = oracle.hadamard(y_ref)
+        y = ssd_i8.ssd_i8_state_update(st, _dev(x), _dev(B), _dev(C), _dev(dt), _dev(A), _dev(D),
+                                       _dev(sx), _dev(sb), _dev(sc), y_dtype="f32",
+                                       hadamard=hadamard)
+        torch.cuda.synchronize()
+        assert np.array_equal(y.cpu().numpy().astype(np.float64), y_ref), f"step {step}: y differs"
+    assert np.array_equal(st.cpu().numpy().astype(np.float64), ref)
