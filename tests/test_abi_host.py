@@ -7,6 +7,7 @@ import ctypes
 import glob
 import os
 import re
+from pathlib import Path
 
 import pytest
 
@@ -145,3 +146,21 @@ def test_binding_refuses_cpu_tensors(lib):
         ssd_i8.ssd_i8_chunk_scan(x, B, B, torch.zeros(1, 8, 4), f, f, f, torch.zeros(1),
                                  torch.zeros(1), 64, y=torch.zeros(1, 8, 4, 64, dtype=torch.float16),
                                  workspace=torch.zeros(1 << 20, dtype=torch.uint8))
+
+
+def test_missing_library_fails_loudly():
+    """Without libssd_i8.so the binding raises; there is no CPU or library fallback.  (A fresh
+    interpreter: the loaded library is cached per process.)"""
+    import subprocess
+    import sys
+    code = ("import quantized_mamba_ssd_b200.ssd_i8 as m\n"
+            "m.LIB_PATH = '/nonexistent/libssd_i8.so'\n"
+            "try:\n"
+            "    m.library()\n"
+            "except RuntimeError as e:\n"
+            "    print('raised:', e)\n")
+    root = Path(__file__).resolve().parent.parent
+    out = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True,
+                         timeout=300)
+    assert out.returncode == 0, out.stderr
+    assert "raised:" in out.stdout and "no fallback" in out.stdout
