@@ -49,8 +49,7 @@ NOMINAL_HBM_GBS = 7700.0  # B200 HBM3e datasheet bandwidth (HGX), context for th
 # profiles/ncu_fused_chunk_scan_b2_L8192.md.  The traffic grows in proportion to the tokens of a
 # launch, so the bench scales it to the workload.  A changed kernel reports null.
 _CAPTURED_TRAFFIC_PER_TOKEN = {
-    # captured on the source 82da36d3...; this one differs by a comment
-    "c4c8f1a4dcb13646de7b09276d7be90bae294ae997e70e596ceb8241428e3849": (329.368576e6 + 108.555520e6) / 16384,
+    "efe4e564dc6a982169aa468427b2678cf7e8abde933c2a76fb103dccab37e53b": (328.967424e6 + 107.602688e6) / 16384,
 }
 
 

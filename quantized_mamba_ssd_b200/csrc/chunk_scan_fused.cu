@@ -46,7 +46,11 @@
 //               statistics chained through the workers (bound on |H|, state unit), output of
 //               the worker's previous block (its accumulator completes meanwhile), x and B'
 //               conversions, M' from CB(k), then the serial part, the state hand-over (H',
-//               decay) and C'.
+//               decay) and C'.  Only the dt scan and the M' tables need a barrier across the
+//               worker's four warps; the steps whose results only the MMA warp reads (the
+//               accumulator read-out, M', the hand-over, C' and the stage release) end with one
+//               mbarrier arrival per warp, so a warp with a lighter part (the causal M' work
+//               grows with the token quarter) goes on to its next step without waiting.
 // Every wait is bounded; a timeout sets a status word and turns the remaining waits into
 // no-ops so that the kernel still ends (its outputs are then undefined).
 #include <algorithm>
@@ -623,7 +627,11 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
 
     if (tid == 0) {
         for (int i = 0; i < kNumBars; ++i)
-            mbar_init(bars + i, (i == kBarEmpty0 || i == kBarEmpty1) ? 2 : 1);
+            mbar_init(bars + i, (i == kBarEmpty0 || i == kBarEmpty1) ? 5
+                                : (i == kBarMp0 || i == kBarMp1 || i == kBarPh0 || i == kBarPh1 ||
+                                   i == kBarPc0 || i == kBarPc1 || i == kBarAccFree0 ||
+                                   i == kBarAccFree1 || i == kBarXb0 || i == kBarXb1 ||
+                                   i == kBarCbIn0 || i == kBarCbIn1) ? 4 : 1);
         fence_mbar_init();
         *abort_flag = 0;
         if (blockIdx.x == 0) p.status[2] = p.epoch;  // the call the status word refers to
@@ -854,8 +862,8 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                     }
                 }
                 tc_fence_before();
-                wg_sync(bar_id);
-                if (row == 0) mbar_arrive(bars + kBarAccFree0 + w);
+                __syncwarp();
+                if (tl == 0) mbar_arrive(bars + kBarAccFree0 + w);  // one arrival per warp
                 if (!store) return;
                 const float rs = pv_rho * 0.125f;
 #pragma unroll 1
@@ -882,8 +890,8 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                     __syncwarp();
                 }
                 tc_fence_before();
-                wg_sync(bar_id);
-                if (row == 0) mbar_arrive(bars + kBarAccFree0 + w);
+                __syncwarp();
+                if (tl == 0) mbar_arrive(bars + kBarAccFree0 + w);  // one arrival per warp
             }
         };
         int kb_last = -1;
@@ -1041,8 +1049,8 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 fence_proxy_async_smem();
                 tmem_st_wait();
                 tc_fence_before();
-                wg_sync(bar_id);
-                if (row == 0) mbar_arrive(bars + kBarCbIn0 + w);
+                __syncwarp();
+                if (tl == 0) mbar_arrive(bars + kBarCbIn0 + w);  // one arrival per warp
             }
             {
                 const int lt = row;
@@ -1082,15 +1090,15 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 }
             }
             wg_sync(bar_id);  // x, B' (for the MMA) and the M' tables complete
-            if (row == 0 && !PERN) mbar_arrive(bars + kBarXb0 + w);
+            if (tl == 0 && !PERN) mbar_arrive(bars + kBarXb0 + w);  // one arrival per warp
             // (f) M' in place over CB, one 32-column chunk at a time (increasing order)
             wait_phase(bars + kBarCb0 + w, ph, abort_flag, p);
             tc_fence_after();
             if constexpr (PERN) {  // ChunkBMM has read B~: B' in its place
                 convert_bp();
                 fence_proxy_async_smem();
-                wg_sync(bar_id);
-                if (row == 0) mbar_arrive(bars + kBarXb0 + w);
+                __syncwarp();
+                if (tl == 0) mbar_arrive(bars + kBarXb0 + w);  // one arrival per warp
             }
             // ChunkBMM entries as exact fp32: int32 from the int8 products, or the f32 of the
             // f16 products (per-channel scales)
@@ -1149,8 +1157,8 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
                 tmem_st_wait();
             }
             tc_fence_before();
-            wg_sync(bar_id);
-            if (row == 0) mbar_arrive(bars + kBarMp0 + w);
+            __syncwarp();
+            if (tl == 0) mbar_arrive(bars + kBarMp0 + w);  // one arrival per warp
             // (g) state hand-over, after the previous block's update: H' = H U / kappa (f16)
             //     for C'H', then decay + rescale to this block's unit
             if (kb >= 1) wait_phase(bars + kBarState, (kb - 1) & 1, abort_flag, p);
@@ -1200,8 +1208,8 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             fence_proxy_async_smem();
             tmem_st_wait();
             tc_fence_before();
-            wg_sync(bar_id);
-            if (row == 0) mbar_arrive(bars + kBarPh0 + w);
+            __syncwarp();
+            if (tl == 0) mbar_arrive(bars + kBarPh0 + w);  // one arrival per warp
             // (h) C row scaled by 2^a_t -> C' in TMEM, once the previous C'H' is done
             if (kb >= 1) wait_phase(bars + kBarCh, (kb - 1) & 1, abort_flag, p);
             tc_fence_after();
@@ -1220,8 +1228,8 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
             }
             tmem_st_wait();
             tc_fence_before();
-            wg_sync(bar_id);  // every thread is done with the stage, C' is written
-            if (row == 0) {
+            __syncwarp();  // the warp is done with the stage, its C' rows are written
+            if (tl == 0) {
                 mbar_arrive(bars + kBarPc0 + w);
                 mbar_arrive(bars + kBarEmpty0 + w);
             }
