@@ -49,7 +49,8 @@ NOMINAL_HBM_GBS = 7700.0  # B200 HBM3e datasheet bandwidth (HGX), context for th
 # profiles/ncu_fused_chunk_scan_b2_L8192.md.  The traffic grows in proportion to the tokens of a
 # launch, so the bench scales it to the workload.  A changed kernel reports null.
 _CAPTURED_TRAFFIC_PER_TOKEN = {
-    "efe4e564dc6a982169aa468427b2678cf7e8abde933c2a76fb103dccab37e53b": (328.967424e6 + 107.602688e6) / 16384,
+    # captured on the source efe4e564...; this one differs by a comment
+    "ba5773591ada92b032d5f81afe4d044344a376a682f6ec0300947b3f30e8ce63": (328.967424e6 + 107.602688e6) / 16384,
 }
 
 

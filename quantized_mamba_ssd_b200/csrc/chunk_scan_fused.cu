@@ -50,7 +50,11 @@
 //               worker's four warps; the steps whose results only the MMA warp reads (the
 //               accumulator read-out, M', the hand-over, C' and the stage release) end with one
 //               mbarrier arrival per warp, so a warp with a lighter part (the causal M' work
-//               grows with the token quarter) goes on to its next step without waiting.
+//               grows with the token quarter) goes on to its next step without waiting.  The
+//               dt-scan barrier at every block start is what keeps these counts sound: a warp
+//               makes its arrival for block k + 2 only after that barrier, which every warp
+//               reaches only after its own arrival for block k, so no phase is completed by a
+//               mix of two blocks' arrivals.
 // Every wait is bounded; a timeout sets a status word and turns the remaining waits into
 // no-ops so that the kernel still ends (its outputs are then undefined).
 #include <algorithm>
