@@ -49,8 +49,7 @@ NOMINAL_HBM_GBS = 7700.0  # B200 HBM3e datasheet bandwidth (HGX), context for th
 # profiles/ncu_fused_chunk_scan_b2_L8192.md.  The traffic grows in proportion to the tokens of a
 # launch, so the bench scales it to the workload.  A changed kernel reports null.
 _CAPTURED_TRAFFIC_PER_TOKEN = {
-    # captured on the source efe4e564...; this one differs by a comment
-    "ba5773591ada92b032d5f81afe4d044344a376a682f6ec0300947b3f30e8ce63": (328.967424e6 + 107.602688e6) / 16384,
+    "d0ae31f7d1c82131495dfc905ac9833d6cd97c6b7fe9a63ed92414a83e90d084": (179.526656e6 + 108.476160e6) / 16384,
 }
 
 

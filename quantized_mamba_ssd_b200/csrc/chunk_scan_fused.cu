@@ -1365,7 +1365,8 @@ EncodeTiledFn encode_fn() {
 // 3-D int8 map over packed tokens: [T][rows2][inner] with `tok_stride` bytes between tokens and
 // `inner` bytes between rows2 entries; box {box0, 1, rows}.
 bool make_map3(CUtensorMap* m, const void* base, int inner, int rows2, long long T,
-               long long tok_stride, int box0, int rows, CUtensorMapSwizzle sw) {
+               long long tok_stride, int box0, int rows, CUtensorMapSwizzle sw,
+               CUtensorMapL2promotion promo = CU_TENSOR_MAP_L2_PROMOTION_L2_256B) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows2, (cuuint64_t)T};
@@ -1373,7 +1374,7 @@ bool make_map3(CUtensorMap* m, const void* base, int inner, int rows2, long long
     cuuint32_t box[3] = {(cuuint32_t)box0, 1, (cuuint32_t)rows};
     cuuint32_t es[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, promo,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -1480,7 +1481,12 @@ cudaError_t launch_chunk_scan(const ChunkScanArgs& a, cudaStream_t st) {
     const long long xs = varlen ? a.x_token_stride : (long long)a.nheads * kP;
     const long long bcs = varlen ? a.bc_token_stride : (long long)a.ngroups * a.dstate;
     CUtensorMap mx, mB, mC;
-    if (!make_map3(&mx, a.x, kP, a.nheads, T, xs, kP, kBlk, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+    // x with 64-byte L2 promotion: a tile row is one head's 64 bytes of a token, and the next
+    // head's row is 64 bytes on.  With 256-byte promotion every row fetched three other heads'
+    // rows into L2, which the evict-first policy of x then dropped before those heads ran:
+    // 1.9x the input bytes read from DRAM, against 1.02x now (same kernel time).
+    if (!make_map3(&mx, a.x, kP, a.nheads, T, xs, kP, kBlk, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_64B) ||
         !make_map3(&mB, a.B, a.dstate, a.ngroups, T, bcs, 128, kBlk, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map3(&mC, a.C, a.dstate, a.ngroups, T, bcs, 128, kBlk, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
