@@ -21,7 +21,8 @@
  *     Argument errors are detected on the host and returned before anything is launched;
  *     launch failures return SSD_ERR_CUDA.  No entry point throws or aborts.
  *   - Output dtype codes: SSD_OUT_F32 (float), SSD_OUT_F16 (IEEE half), SSD_OUT_I8 (int8,
- *     q = clamp(round_half_even(y / y_scale), -127, 127); y_scale > 0 is used only for I8).
+ *     q = clamp(round_half_even(y * fp32(1 / y_scale)), -127, 127), the product taken exactly
+ *     and rounded once; y_scale > 0 is used only for I8).
  */
 #ifndef SSD_I8_H
 #define SSD_I8_H

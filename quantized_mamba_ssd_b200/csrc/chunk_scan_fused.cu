@@ -291,6 +291,16 @@ __device__ __forceinline__ f2 fadd2(f2 a, f2 b) {
     return r;
 }
 
+// a * b + c with one rounding
+__device__ __forceinline__ f2 ffma2(f2 a, f2 b, f2 c) {
+    f2 r;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return r;
+}
+
 __device__ __forceinline__ f2 fsub2(f2 a, f2 b) {
     f2 r;
     asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
@@ -801,14 +811,17 @@ fused_chunk_scan_kernel(const __grid_constant__ CUtensorMap map_x,
         // output dtype
         auto store32 = [&](const float (&v)[32], float s, size_t ybase, int hq) {
             if constexpr (YT == SSD_OUT_I8) {
-                // q = clamp(rint(fp32(acc * s / s_y))): the same rounding as the fp32 output
+                // q = clamp(rint(acc * s / s_y)) with the product rounded once: an FMA with the
+                // rounding constant 1.5 * 2^23 rounds the exact product to an integer, half to
+                // even.  s and s / s_y differ by the power of two rho, so this is the exact
+                // product of the fp32 output y and fp32(1 / s_y), rounded once.
                 const float sc = s * p.inv_y_scale;
                 const f2 s2 = {sc, sc}, rnd = {kRound, kRound};
                 uint32_t wv[8];
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
-                    const f2 v0 = fadd2(fmul2(f2{v[4 * q], v[4 * q + 1]}, s2), rnd);
-                    const f2 v1 = fadd2(fmul2(f2{v[4 * q + 2], v[4 * q + 3]}, s2), rnd);
+                    const f2 v0 = ffma2(f2{v[4 * q], v[4 * q + 1]}, s2, rnd);
+                    const f2 v1 = ffma2(f2{v[4 * q + 2], v[4 * q + 3]}, s2, rnd);
                     const uint32_t lo = __byte_perm(clamp_code(v0.x), clamp_code(v0.y), 0x0040);
                     const uint32_t hi = __byte_perm(clamp_code(v1.x), clamp_code(v1.y), 0x0040);
                     wv[q] = __byte_perm(lo, hi, 0x5410);

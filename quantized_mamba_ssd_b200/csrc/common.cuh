@@ -14,14 +14,18 @@ constexpr int kWarp = 32;
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 // Output store in the requested dtype.  I8 applies q = clamp(rne(y * inv_scale), -127, 127)
-// with inv_scale = 1 / y_scale computed once in fp32 on the host.
+// with inv_scale = 1 / y_scale computed once in fp32 on the host and the product rounded once
+// (as in the chunk scan's epilogue).
 __device__ __forceinline__ void store_out(void* y, size_t idx, float v, int dtype, float inv_scale) {
     if (dtype == SSD_OUT_F32) {
         static_cast<float*>(y)[idx] = v;
     } else if (dtype == SSD_OUT_F16) {
         static_cast<__half*>(y)[idx] = __float2half_rn(v);
     } else {
-        float r = rintf(v * inv_scale);
+        // an FMA with 1.5 * 2^23 rounds the exact product to an integer, half to even
+        // (|v * inv_scale| >= 2^22 lands outside +-127 either way and is clamped)
+        constexpr float kRoundI = 12582912.f;
+        float r = __fmaf_rn(v, inv_scale, kRoundI) - kRoundI;
         r = fminf(fmaxf(r, -127.f), 127.f);
         static_cast<int8_t*>(y)[idx] = static_cast<int8_t>(static_cast<int>(r));
     }

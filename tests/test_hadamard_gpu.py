@@ -98,9 +98,10 @@ def test_int8_hadamard_is_the_fp32_hadamard_requantized():
     s_y = np.float32(np.abs(y32).max() / 100.0)
     yq, _ = run(case, y_dtype="i8", y_scale=float(s_y))
     # the per-block scale and the 1/8 are powers of two, so scaling commutes with rounding and
-    # the int8 output is exactly the f32 output requantized with fp32(1 / s_y)
+    # the int8 output is exactly the f32 output times fp32(1 / s_y), the product taken exactly
+    # (fp64 holds the product of two fp32 values) and rounded once
     inv = np.float32(1.0) / s_y
-    expect = np.clip(np.rint(y32.astype(np.float32) * inv), -127, 127)
+    expect = np.clip(np.rint(y32.astype(np.float64) * np.float64(inv)), -127, 127)
     assert np.array_equal(yq, expect)
 
 

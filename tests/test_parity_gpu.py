@@ -94,14 +94,35 @@ def test_small_prefill_int8_output(Q):
 
 
 def test_int8_output_is_the_fp32_output_requantized():
-    # the int8 epilogue must be q = clamp(rint(y * fp32(1/s_y))) of the very y the f32 path writes
+    # the int8 epilogue must be q = clamp(rint(y * fp32(1/s_y))) of the very y the f32 path
+    # writes, the product taken exactly (fp64 holds the product of two fp32 values) and rounded
+    # once
     case = mk(1, 333, 4, 2, 128, 128, law="laplace_outliers_all", seed=5)
     y32, _ = gpu_scan(case, y_dtype="f32")
     s_y = np.float32(np.abs(y32).max() / 100.0)
     yq, _ = gpu_scan(case, y_dtype="i8", y_scale=float(s_y))
     inv = np.float32(1.0) / s_y
-    ref = np.clip(np.rint(y32.astype(np.float32) * inv), -127, 127).astype(np.int8)
+    ref = np.clip(np.rint(y32.astype(np.float64) * np.float64(inv)), -127, 127).astype(np.int8)
     assert np.array_equal(yq, ref)
+
+
+def test_int8_rounding_rule_at_full_size():
+    """The 8B-shaped prefill with s_y = 0.05: at this size some products y * fp32(1/s_y) fall
+    close enough to a half-integer that rounding them to fp32 first would move the code.  The
+    epilogue rounds the exact product once, in every one of the 2^28 outputs."""
+    case = W.make_prefill_config(3)
+    y32, _ = gpu_scan(case, y_dtype="f32", init=False, final=False)
+    yq, _ = gpu_scan(case, y_dtype="i8", y_scale=0.05, init=False, final=False)
+    inv = np.float32(1.0) / np.float32(0.05)
+    once = twice = 0
+    flat32, flatq = y32.reshape(-1, 1 << 20), yq.reshape(-1, 1 << 20)
+    for a, q in zip(flat32, flatq):
+        ref1 = np.clip(np.rint(a.astype(np.float64) * np.float64(inv)), -127, 127).astype(np.int8)
+        ref2 = np.clip(np.rint(a * inv), -127, 127).astype(np.int8)   # fp32 product first
+        once += int((q != ref1).sum())
+        twice += int((ref1 != ref2).sum())
+    assert once == 0, f"{once} int8 outputs differ from the one-rounding rule"
+    assert twice > 0, "no output distinguishes the two roundings: the check has no power here"
 
 
 # ---------------------------------------------------------------------------------------
