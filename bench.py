@@ -49,7 +49,7 @@ NOMINAL_HBM_GBS = 7700.0  # B200 HBM3e datasheet bandwidth (HGX), context for th
 # profiles/ncu_fused_chunk_scan_b2_L8192.md.  The traffic grows in proportion to the tokens of a
 # launch, so the bench scales it to the workload.  A changed kernel reports null.
 _CAPTURED_TRAFFIC_PER_TOKEN = {
-    "d0ae31f7d1c82131495dfc905ac9833d6cd97c6b7fe9a63ed92414a83e90d084": (179.526656e6 + 108.476160e6) / 16384,
+    "f49754942ee3a1e403d29bf7941f7579f5176cb7effce65f49bab0607a1226b3": (179.271424e6 + 108.001792e6) / 16384,
 }
 
 
