@@ -219,3 +219,28 @@ def test_decode_steps_are_exact_on_the_readout_family(_lib, N, hadamard):
         torch.cuda.synchronize()
         assert np.array_equal(y.cpu().numpy().astype(np.float64), y_ref), f"step {step}: y differs"
     assert np.array_equal(st.cpu().numpy().astype(np.float64), ref)
+
+
+def test_packed_family_matches_the_closed_form_per_sequence():
+    """CPU: every token t < L of every packed sequence is carried by exactly one (head, column)
+    of each group, and the oracle on each sequence is the closed form of the dense family."""
+    lengths = [130, 1, 0, 64, 200]
+    case, cu = W.make_exact_readout_varlen(lengths, 2, 32, seed=3)
+    P, G = case.headdim, case.ngroups
+    per_group = case.nheads // G
+    for i, L in enumerate(lengths):
+        if L == 0:  # an empty sequence carries no token
+            continue
+        a = int(cu[i])
+        xs = case.x[0, a:a + L]  # [L, H, P]
+        for g in range(G):
+            ones = xs[:, g * per_group:(g + 1) * per_group].reshape(L, -1).sum(axis=1)
+            assert np.array_equal(ones, np.ones(L)), f"sequence {i}, group {g}: one-hot broken"
+        sub = W.PrefillCase(
+            name="seq", batch=1, seqlen=L, nheads=case.nheads, headdim=P, dstate=case.dstate,
+            ngroups=G, chunk_size=case.chunk_size, x=case.x[:, a:a + L], B=case.B[:, a:a + L],
+            C=case.C[:, a:a + L], dt=case.dt[:, a:a + L], A=case.A, D=case.D,
+            x_scale=case.x_scale, B_scale=case.B_scale, C_scale=case.C_scale)
+        y = oracle.scan(sub.x, sub.B, sub.C, sub.dt, sub.A, sub.D, sub.x_scale, sub.B_scale,
+                        sub.C_scale)[0]
+        assert np.array_equal(y, _closed_form(sub, None)), f"sequence {i}: oracle != closed form"
